@@ -1,0 +1,487 @@
+#!/usr/bin/env python
+"""Benchmark: paged-KV decode step (append + split-KV decode) on B200.
+
+One step = the whole hot path over one batch: append this step's new K/V
+through the page table, then decode attention over every cached token.  The
+default workload is the Llama-3-8B-shaped batch (64 sequences, context
+U[128,4096], page size 64, 32 q / 8 kv heads, head_dim 128, bf16).  Inputs are
+seeded synthetic data resident in HBM; the KV pool (~0.55 GB) exceeds the
+126 MB L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..5]
+    python bench.py --impl reference ...   # the CPU oracle on the host cores
+
+Prints ONE JSON line (rank 0).  ``value`` is whole-job achieved HBM GB/s of
+algorithmic bytes (K/V + scales + Q/out + page-table entries + appended
+rows) per step time; tokens/s is reported beside it.  Multi-GPU runs are
+weak scaling: each rank runs its own batch, no data-path collective.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged-KV decode attention: achieved HBM GB/s (% of B200 peak), tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--num-ctas", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-seqs", type=int, default=64)
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), \
+            "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+# ------------------------------------------------------------ byte counts
+def decode_bytes(w, rows=None) -> int:
+    """Algorithmic bytes of decode over sequences ``rows`` (default: decode rows)."""
+    rows = w.decode_rows if rows is None else np.asarray(rows)
+    la = w.lens_after[rows].astype(np.int64)
+    P = w.page_size
+    kv = int(la.sum()) * w.num_kv_heads * w.head_dim * 2 * w.elem_bytes
+    pages = int(((la + P - 1) // P).sum())
+    scales = pages * w.num_kv_heads * 2 * 4 if w.kv_dtype == "e4m3" else 0
+    qo = 2 * len(rows) * w.num_q_heads * w.head_dim * 2
+    return kv + scales + qo + pages * 4
+
+
+def append_bytes(w) -> int:
+    t = int(w.new_lens.sum())
+    return t * w.num_kv_heads * w.head_dim * 2 * (2 + w.elem_bytes)
+
+
+def prefill_flops(w) -> int:
+    tot = 0
+    for b in w.chunk_rows:
+        L, n = int(w.lens_after[b]), int(w.new_lens[b])
+        tot += sum(L - n + i + 1 for i in range(n))
+    return 4 * w.num_q_heads * w.head_dim * tot
+
+
+# ------------------------------------------------------------ clock sampler
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        0x0000000000000004: "sw_power_cap",
+        0x0000000000000008: "hw_slowdown",
+        0x0000000000000020: "sw_thermal_slowdown",
+        0x0000000000000040: "hw_thermal_slowdown",
+        0x0000000000000080: "hw_power_brake_slowdown",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples, self.reasons = [], set()
+        self.period = period_s
+        self._stop = threading.Event()
+        self.max_mhz = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nvml = None
+
+    def _run(self):
+        n = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM))
+                mask = n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nvml:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.nvml:
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ setup
+def setup_device_state(w, device):
+    """Pool filled through the library's own append (context tokens)."""
+    import torch
+    import paged_kv_cache_476_b200 as pkv
+    import workloads
+
+    shape = w.pool_shape()
+    if w.kv_dtype == "e4m3":
+        k_pool = torch.full(shape, workloads.E4M3_NAN_CODE, dtype=torch.uint8, device=device)
+        v_pool = torch.full(shape, workloads.E4M3_NAN_CODE, dtype=torch.uint8, device=device)
+        k_scale = torch.ones((w.num_pages, w.num_kv_heads), dtype=torch.float32, device=device)
+        v_scale = torch.ones_like(k_scale)
+    else:
+        k_pool = torch.full(shape, workloads.BF16_NAN_BITS, dtype=torch.int16,
+                            device=device).view(torch.bfloat16)
+        v_pool = torch.full(shape, workloads.BF16_NAN_BITS, dtype=torch.int16,
+                            device=device).view(torch.bfloat16)
+        k_scale = v_scale = None
+    flags = torch.zeros(1, dtype=torch.int32, device=device)
+    cache = pkv.PagedKVCache(k_pool, v_pool, w.kv_dtype, k_scale, v_scale, flags)
+    table = torch.from_numpy(w.page_table).to(device)
+    k_new, v_new = [], []
+    for b in range(w.batch):
+        k, v = w.kv_seq(b)
+        c = int(w.ctx_lens[b])
+        if w.kv_dtype == "e4m3":
+            pages, ks, vs = w.kv_scales_for(b, k, v)
+            idx = torch.from_numpy(pages.astype(np.int64)).to(device)
+            k_scale[idx] = torch.from_numpy(ks).to(device)
+            v_scale[idx] = torch.from_numpy(vs).to(device)
+        if c:
+            pkv.paged_kv_append(cache, table[b:b + 1].contiguous(),
+                                torch.zeros(1, dtype=torch.int32, device=device),
+                                torch.tensor([0, c], dtype=torch.int32, device=device),
+                                k[:c].to(device), v[:c].to(device))
+        k_new.append(k[c:])
+        v_new.append(v[c:])
+    torch.cuda.synchronize()
+    st = {
+        "cache": cache, "flags": flags, "table": table,
+        "ctx_lens": torch.from_numpy(w.ctx_lens).to(device),
+        "cu_new": torch.from_numpy(w.cu_new()).to(device),
+        "k_new": torch.cat(k_new).to(device), "v_new": torch.cat(v_new).to(device),
+    }
+    rows = torch.from_numpy(w.decode_rows).to(device)
+    st["dec_q"] = w.q_decode().to(device)
+    st["dec_table"] = table[rows].contiguous()
+    st["dec_lens"] = torch.from_numpy(w.lens_after[w.decode_rows]).to(device)
+    st["dec_max"] = int(w.lens_after[w.decode_rows].max()) if len(w.decode_rows) else 0
+    st["dec_out"] = torch.empty_like(st["dec_q"])
+    st["dec_lse"] = torch.empty(st["dec_q"].shape[:2], dtype=torch.float32, device=device)
+    if len(w.chunk_rows):
+        crow = torch.from_numpy(w.chunk_rows).to(device)
+        st["pf_q"] = w.q_chunks().to(device)
+        st["pf_table"] = table[crow].contiguous()
+        st["pf_lens"] = torch.from_numpy(w.lens_after[w.chunk_rows]).to(device)
+        st["pf_cu"] = torch.from_numpy(w.cu_q_chunks()).to(device)
+        st["pf_max"] = int(w.new_lens[w.chunk_rows].max())
+        st["pf_out"] = torch.empty_like(st["pf_q"])
+        st["pf_lse"] = torch.empty(st["pf_q"].shape[:2], dtype=torch.float32, device=device)
+    return st
+
+
+def run_ours(args, rank, world, device, dist):
+    import torch
+    import paged_kv_cache_476_b200 as pkv
+    import workloads
+
+    w = workloads.config(args.config)
+    st = setup_device_state(w, device)
+    cache = st["cache"]
+    ws = pkv.decode_workspace(cache, len(w.decode_rows), w.num_q_heads, st["dec_max"],
+                              args.num_ctas)
+    stream = torch.cuda.current_stream()
+    has_pf = len(w.chunk_rows) > 0
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        pkv.paged_kv_append(cache, st["table"], st["ctx_lens"], st["cu_new"], st["k_new"],
+                            st["v_new"])
+        if ev is not None:
+            ev[1].record(stream)
+        if len(w.decode_rows):
+            pkv.paged_decode_attention(cache, st["dec_q"], st["dec_table"], st["dec_lens"],
+                                       st["dec_max"], w.softmax_scale, out=st["dec_out"],
+                                       lse=st["dec_lse"], workspace=ws, num_ctas=args.num_ctas)
+        if ev is not None:
+            ev[2].record(stream)
+        if has_pf:
+            pkv.paged_prefill_chunk_attention(cache, st["pf_q"], st["pf_cu"], st["pf_table"],
+                                              st["pf_lens"], st["pf_max"], w.softmax_scale,
+                                              out=st["pf_out"], lse=st["pf_lse"])
+        if ev is not None:
+            ev[3].record(stream)
+
+    launches_per_step = 1 + (1 if len(w.decode_rows) else 0) + (1 if has_pf else 0)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if int(st["flags"].item()) != 0:
+        raise RuntimeError(f"device error flags {int(st['flags'].item()):#x}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    elapsed = t0.elapsed_time(t1) / 1e3  # seconds
+    dec_s = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps / 1e3
+    app_s = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps / 1e3
+    pf_s = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps / 1e3
+    if dist:
+        import torch.distributed as tdist
+
+        t = torch.tensor([elapsed], device=device)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        elapsed = float(t.item())
+
+    # ---------------------------------------------------------------- e2e
+    # Through the public API with host buffers: per step, H2D of the step's
+    # inputs (q, new K/V, lengths, page table) from pinned memory and D2H of
+    # the attention output, all inside the timed region.
+    names = ("dec_q", "k_new", "v_new", "table", "ctx_lens", "dec_lens", "dec_table")
+    offs, total = {}, 0
+    for k in names:
+        offs[k] = total
+        total += (st[k].numel() * st[k].element_size() + 255) // 256 * 256
+    h_buf = torch.empty(total, dtype=torch.uint8).pin_memory()
+    d_buf = torch.empty(total, dtype=torch.uint8, device=device)
+    d = {}
+    for k in names:
+        n = st[k].numel() * st[k].element_size()
+        h_buf[offs[k]:offs[k] + n].copy_(st[k].contiguous().view(-1).view(torch.uint8).cpu())
+        d[k] = d_buf[offs[k]:offs[k] + n].view(st[k].dtype).view(st[k].shape)
+    h_out = torch.empty(st["dec_out"].shape, dtype=st["dec_out"].dtype).pin_memory()
+    e_steps = max(1, min(args.steps, 200))
+
+    def e2e_step():
+        d_buf.copy_(h_buf, non_blocking=True)  # one H2D copy of every step input
+        pkv.paged_kv_append(cache, d["table"], d["ctx_lens"], st["cu_new"], d["k_new"],
+                            d["v_new"])
+        pkv.paged_decode_attention(cache, d["dec_q"], d["dec_table"], d["dec_lens"], st["dec_max"],
+                                   w.softmax_scale, out=st["dec_out"], lse=st["dec_lse"],
+                                   workspace=ws, num_ctas=args.num_ctas)
+        h_out.copy_(st["dec_out"], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_s = e0.elapsed_time(e1) / 1e3 / e_steps
+    if dist:
+        import torch.distributed as tdist
+
+        t = torch.tensor([e2e_s], device=device)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        e2e_s = float(t.item())
+    h2d = sum(st[k].numel() * st[k].element_size() for k in names)
+    d2h = h_out.numel() * h_out.element_size()
+
+    flags = int(st["flags"].item())
+    step_bytes = decode_bytes(w) + append_bytes(w)
+    step_s = elapsed / args.steps
+    hbm_peak, tf_peak, peak_kind = peaks()
+    dbytes = decode_bytes(w)
+    achieved = dbytes / dec_s / 1e9
+    res = {
+        "metric": METRIC,
+        "value": round(world * step_bytes / step_s / 1e9, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_s * 1e3, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.kv_dtype == "bf16" else "e4m3-kv/bf16-q",
+        "data": "synthetic (seeded N(0,1) bf16 K/V/Q, permuted pages, NaN sentinels)",
+        "tokens_per_s": round(world * len(w.decode_rows) / step_s, 1),
+        "config": {
+            "workload": w.name,
+            "batch": int(len(w.decode_rows)),
+            "page_size": w.page_size,
+            "heads_q_kv": [w.num_q_heads, w.num_kv_heads],
+            "head_dim": w.head_dim,
+            "kv_tokens": int(w.decode_kv_tokens()),
+            "step_bytes": int(step_bytes),
+            "parallelism": f"dp{world} (independent batches)",
+            "l2": f"KV pool {w.pool_bytes() * 2 / 1e6:.0f} MB > 126 MB L2; no flush",
+            "seed": w.seed,
+        },
+        "kernels_ms": {"append": round(app_s * 1e3, 5), "decode": round(dec_s * 1e3, 5),
+                       "prefill": round(pf_s * 1e3, 5) if has_pf else None},
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "decode_kernel",
+            "achieved": round(achieved, 1),
+            "peak": hbm_peak,
+            "unit": "GB/s",
+            "frac": round(achieved / hbm_peak, 4),
+            "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth)",
+            "traffic": None,
+            "algorithmic_bytes_per_launch": int(dbytes),
+        },
+        "e2e": {"value": round(world * step_bytes / e2e_s / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "ms_per_step": round(e2e_s * 1e3, 5)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+        "device_error_flags": flags,
+    }
+    if has_pf:
+        pf = prefill_flops(w)
+        res["prefill"] = {"tflops": round(pf / pf_s / 1e12, 2) if pf_s > 0 else None,
+                          "peak_tflops": tf_peak, "flops_per_launch": int(pf)}
+    return w, res
+
+
+# ----------------------------------------------------------- CPU oracle
+def oracle_sample(w, n_seqs: int):
+    """Decode rows for a bounded CPU sample: spread over the length range."""
+    rows = w.decode_rows
+    order = rows[np.argsort(w.lens_after[rows], kind="stable")]
+    idx = np.linspace(0, len(order) - 1, num=min(n_seqs, len(order))).round().astype(int)
+    return np.unique(order[idx])
+
+
+def run_oracle(w, n_seqs: int, repeats: int = 1):
+    """Time the oracle (append of the step's tokens + decode) on a sample."""
+    import oracle
+
+    sample = oracle_sample(w, n_seqs)
+    c = oracle.cache_for(w, seq_ids=sample, include_new=False)
+    q = oracle.bf16_bits(w.q_decode())
+    k_new, v_new = w.new_kv(rows=sample)
+    cu = np.concatenate([[0], np.cumsum(w.new_lens[sample])]).astype(np.int32)
+    pos = {int(b): i for i, b in enumerate(w.decode_rows)}
+    qi = np.array([pos[int(b)] for b in sample])
+    times = []
+    for _ in range(repeats):
+        t = time.perf_counter()
+        c.append(w.page_table[sample], w.ctx_lens[sample], cu, oracle.bf16_bits(k_new),
+                 oracle.bf16_bits(v_new))
+        c.decode(q[qi], w.page_table[sample], w.lens_after[sample], w.softmax_scale)
+        times.append(time.perf_counter() - t)
+    dt = statistics.median(times)
+    nbytes = decode_bytes(w, rows=sample) + int(w.new_lens[sample].sum()) * w.num_kv_heads * \
+        w.head_dim * 2 * (2 + w.elem_bytes)
+    return {
+        "value": round(nbytes / dt / 1e9, 4),
+        "unit": "GB/s",
+        "cores": oracle.num_threads(),
+        "kind": "oracle",
+        "sample": f"{len(sample)} of {len(w.decode_rows)} sequences (lengths spread over the "
+                  f"range, {int(w.lens_after[sample].sum())} tokens): append + decode, fp64 C "
+                  f"with OpenMP, median of {repeats}",
+        "seconds": round(dt, 3),
+        "tokens_per_s": round(len(sample) / dt, 3),
+    }
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        # The reference arm is the CPU oracle; under torchrun only rank 0 works.
+        if rank != 0:
+            return 0
+        import workloads
+
+        w = workloads.config(args.config)
+        n_seqs = args.cpu_sample_seqs
+        for _ in range(args.warmup):
+            pass  # the oracle has no warm-up state worth timing separately
+        rep = max(1, min(args.steps, 3))
+        cb = run_oracle(w, n_seqs, repeats=rep)
+        res = {
+            "metric": METRIC, "value": cb["value"], "unit": "GB/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(cb["seconds"] * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "sample": cb["sample"]},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(res))
+        return 0
+
+    import torch
+
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as tdist
+
+        torch.cuda.set_device(local)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    device = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(device)
+    w, res = run_ours(args, rank, world, device, dist)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = run_oracle(w, args.cpu_sample_seqs, repeats=5)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,207 @@
+/*
+ * paged_kv.h -- C ABI of libpagedkv.so: attention over a paged KV cache for an
+ * in-flight batch, on NVIDIA B200 (sm_100a).
+ *
+ * The operation (pages on TensorRT-LLM):
+ *  - TensorRT-LLM concept page (compassingai.com), "關鍵機制 / PagedAttention
+ *    及 KV 快取管理": each sequence's K/V lives in fixed-size pages (64 or 128
+ *    tokens); a per-sequence page table maps logical token positions to
+ *    physical pages, so no maximum length is reserved up front.
+ *  - same page, "技術原理 / 編譯期圖最佳化": page-table lookups sit on every KV
+ *    read and write of the attention operator.
+ *  - same page, "執行時執行模型": each forward pass of the in-flight batch
+ *    appends the new tokens' K/V and attends over the pages.
+ *  - same page, "關鍵效能引數": context (prefill) tokens are processed in
+ *    parallel over the paged cache.
+ *  - yololab.net guide, "FP8 與極致量化": FP8 storage halves the bytes moved.
+ *
+ * Conventions shared by every entry point:
+ *  - All array pointers are DEVICE memory owned by the caller; the library
+ *    allocates nothing and keeps no state between calls (except the counters
+ *    inside a caller-owned decode workspace, see below).
+ *  - Pools: separate K and V pools, each [num_pages][num_kv_heads][page_size]
+ *    [head_dim], row-major, element type bf16 or FP8 E4M3 (1 byte).  Base
+ *    addresses must be 16-byte aligned.
+ *  - FP8 scales: one fp32 per (page, kv head) for K and one for V, layout
+ *    [num_pages][num_kv_heads]; the stored value of an element is
+ *    decode_e4m3(code) * scale.  Scales must be finite and in (0, 2^15].
+ *    The caller chooses them (e.g. absmax/448 of what the page will hold);
+ *    the library reads them and never updates them.
+ *  - Page table: int32 [batch][max_pages_per_seq], row-major; entry j holds the
+ *    physical page of tokens [j*page_size, (j+1)*page_size).  Entries past the
+ *    last page a sequence needs are ignored (-1 by convention).
+ *  - GQA: q head h reads kv head h / gqa_group (contiguous groups).
+ *  - Supported: page_size in {64, 128}; head_dim in {64, 128};
+ *    gqa_group in {1, 2, 4, 8}; bf16 Q/K/V/out; K/V pools bf16 or E4M3.
+ *  - Asynchronous: a call validates its arguments on the host, returns a
+ *    negative pkv_status before launching anything if they are wrong, and
+ *    otherwise enqueues its kernels on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream) and returns PKV_OK.  Launch failures return
+ *    PKV_ERR_CUDA.  Data-dependent errors (bad page ids, lengths past the page
+ *    table, a bounded wait that gave up) are detected on the device: the
+ *    offending tokens are skipped and, when cache->error_flags is non-NULL,
+ *    the matching PKV_FLAG_* bit is OR-ed into it.  Kernels never trap.
+ *  - Not done by the library: page allocation (the caller owns the pool and
+ *    the table), positional encoding (K arrives post-rotary), scale choice.
+ */
+#ifndef PAGED_KV_H
+#define PAGED_KV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PKV_OK = 0,
+  PKV_ERR_NULL = -1,        /* a required pointer is NULL */
+  PKV_ERR_SHAPE = -2,       /* a count or size is negative or inconsistent */
+  PKV_ERR_PAGE_SIZE = -3,   /* page_size not in {64, 128} */
+  PKV_ERR_HEAD_DIM = -4,    /* head_dim not in {64, 128} */
+  PKV_ERR_GQA = -5,         /* num_q_heads != gqa_group*num_kv_heads, or group unsupported */
+  PKV_ERR_DTYPE = -6,       /* unknown kv_dtype, or E4M3 without scales */
+  PKV_ERR_WORKSPACE = -7,   /* decode workspace NULL, misaligned or too small */
+  PKV_ERR_CUDA = -8,        /* a CUDA runtime call or kernel launch failed */
+  PKV_ERR_ALIGN = -9,       /* a pointer that must be 16-byte aligned is not */
+  PKV_ERR_UNSUPPORTED = -10 /* a valid combination this build does not implement */
+} pkv_status;
+
+typedef enum { PKV_KV_BF16 = 0, PKV_KV_FP8_E4M3 = 1 } pkv_kv_dtype;
+
+/* Device-side error bits OR-ed into pkv_cache.error_flags. */
+#define PKV_FLAG_BAD_PAGE 0x1    /* a page-table entry outside [0, num_pages) */
+#define PKV_FLAG_BAD_LENGTH 0x2  /* a length < 0, past max_pages_per_seq*page_size, or a
+                                    chunk longer than its sequence */
+#define PKV_FLAG_TIMEOUT 0x4     /* a bounded wait inside a kernel gave up */
+#define PKV_FLAG_BAD_SCALE 0x8   /* an FP8 scale outside (0, 2^15] */
+
+/* The paged KV cache: pools, optional FP8 scales, geometry. */
+typedef struct pkv_cache {
+  void* k_pool;          /* [num_pages][num_kv_heads][page_size][head_dim] */
+  void* v_pool;          /* same shape as k_pool */
+  const float* k_scale;  /* [num_pages][num_kv_heads] fp32, E4M3 only (else NULL) */
+  const float* v_scale;  /* [num_pages][num_kv_heads] fp32, E4M3 only (else NULL) */
+  int32_t num_pages;     /* >= 1 */
+  int32_t page_size;     /* tokens per page: 64 or 128 */
+  int32_t num_kv_heads;  /* >= 1 */
+  int32_t head_dim;      /* 64 or 128 */
+  int32_t kv_dtype;      /* pkv_kv_dtype */
+  int32_t* error_flags;  /* optional device int32; NULL disables reporting */
+} pkv_cache;
+
+/*
+ * Paged KV append (the paged store).  Writes the K/V of this step's new tokens
+ * into their pages: new token j of sequence b sits at logical position
+ * pos = seq_lens_before[b] + (j - cu_new_tokens[b]) and is stored in page
+ * page_table[b][pos / page_size], slot pos % page_size.  bf16 pools receive
+ * the input bits unchanged; E4M3 pools receive
+ * e4m3_round_nearest_even_satfinite(fp32(x) / scale[page][kv_head]) with an
+ * IEEE fp32 division.  Source: concept page "PagedAttention 及 KV 快取管理"
+ * and "執行時執行模型" (attention updates the KV pages).
+ *   page_table        int32 [batch][max_pages_per_seq]
+ *   seq_lens_before   int32 [batch], tokens already cached
+ *   cu_new_tokens     int32 [batch+1], exclusive prefix sum of new tokens
+ *   total_new_tokens  == cu_new_tokens[batch] (host copy, sizes the grid)
+ *   k_new, v_new      bf16 [total_new_tokens][num_kv_heads][head_dim]
+ * Tokens whose page entry is invalid are skipped (PKV_FLAG_BAD_PAGE).
+ */
+int paged_kv_append(const pkv_cache* cache, const int32_t* page_table, int32_t max_pages_per_seq,
+                    const int32_t* seq_lens_before, const int32_t* cu_new_tokens, int32_t batch,
+                    int32_t total_new_tokens, const void* k_new, const void* v_new,
+                    void* stream);
+
+/*
+ * Split planning for decode (host only, no CUDA calls).  Decode runs as one
+ * persistent wave of C CTAs.  The work list is every (sequence, kv head) unit
+ * cut into 64-token tiles, concatenated in (sequence, kv head) order; CTA c
+ * takes the contiguous range [c*T/C, (c+1)*T/C) of the T tiles, so every CTA
+ * streams the same number of KV bytes whatever the length mix.  A unit that a
+ * range boundary cuts becomes several split-KV partials merged in the same
+ * launch.  C = num_ctas if num_ctas > 0, else num_sms * ctas_per_sm; C never
+ * exceeds the tiles of the largest batch the arguments allow.
+ * Output: *out_ctas = C >= 1.
+ */
+int paged_decode_plan(int32_t batch, int32_t num_kv_heads, int32_t max_seq_len,
+                      int32_t num_sms, int32_t num_ctas, int32_t ctas_per_sm,
+                      int32_t* out_ctas);
+
+/*
+ * Bytes of decode workspace for these arguments, sized for the current
+ * device (call it with the device that will run the decode current).
+ * Returns 0 on bad arguments.  The workspace holds the split partials
+ * ((units + C) slots of G x (head_dim + 2) floats, units = batch *
+ * num_kv_heads) and one counter per unit.  It must be ZERO-FILLED before its first use; every completed call
+ * leaves the counters at zero again.  Calls that share a workspace must not
+ * overlap on the GPU.
+ */
+size_t paged_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                    int32_t head_dim, int32_t max_seq_len, int32_t num_ctas);
+
+/*
+ * Split-KV decode attention: one query token per sequence attends over all
+ * seq_lens[b] tokens of its pages.  For q head h (kv head g = h / gqa_group):
+ *   s_t = softmax_scale * q[b][h] . K_b[t],   t < seq_lens[b]
+ *   out[b][h] = sum_t exp(s_t - m) V_b[t] / sum_t exp(s_t - m)   (bf16)
+ *   lse[b][h] = m + ln(sum_t exp(s_t - m))                       (fp32)
+ * computed as online-softmax partials over page ranges (see
+ * paged_decode_plan), merged in the same launch by the last CTA that
+ * finishes a piece of each (sequence, kv head).  A sequence of length 0
+ * yields out = 0 and lse = -inf.  Source: concept page "執行時執行模型"
+ * (attention reads the KV pages each step) and "PagedAttention 及 KV 快取管理".
+ *   q             bf16 [batch][num_q_heads][head_dim]
+ *   seq_lens      int32 [batch], tokens per sequence AFTER this step's append
+ *   max_seq_len   host upper bound of seq_lens (plans the grid)
+ *   out           bf16 [batch][num_q_heads][head_dim]
+ *   lse           fp32 [batch][num_q_heads], or NULL
+ *   workspace     16-byte aligned, >= paged_decode_workspace_bytes(...) bytes
+ *   num_ctas      0 = automatic plan; > 0 forces the CTA count (see plan)
+ */
+int paged_decode_attention(const pkv_cache* cache, const void* q, int32_t num_q_heads,
+                           int32_t gqa_group, const int32_t* page_table,
+                           int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
+                           int32_t max_seq_len, float softmax_scale, void* out, float* lse,
+                           void* workspace, size_t workspace_bytes, int32_t num_ctas,
+                           void* stream);
+
+/*
+ * Causal prefill-chunk attention over the paged cache.  Chunk c owns the
+ * queries [cu_q_lens[c], cu_q_lens[c+1]) of the packed q and has seq_lens[c]
+ * tokens cached AFTER its append (its own new tokens included).  Query i of a
+ * chunk with n queries sits at position p = seq_lens[c] - n + i and attends to
+ * keys 0..p inclusive:
+ *   out[row][h] = softmax_t<=p(softmax_scale * q[row][h] . K_c[t]) V_c   (bf16)
+ *   lse[row][h] = ln sum_t<=p exp(softmax_scale * q[row][h] . K_c[t])    (fp32)
+ * QK^T and PV run on the tcgen05 tensor cores.  Source: concept page
+ * "關鍵效能引數" (context tokens processed in parallel over pages, with
+ * FlashAttention) and ab123.xyz post (FA-2 with PagedAttention for long
+ * sequences) -- both prior art; this is an sm_100a design.
+ *   q          bf16 [total_q][num_q_heads][head_dim], total_q = cu_q_lens[num_chunks]
+ *   cu_q_lens  int32 [num_chunks+1]
+ *   page_table int32 [num_chunks][max_pages_per_seq]
+ *   seq_lens   int32 [num_chunks]
+ *   total_q    host copy of cu_q_lens[num_chunks] (rows of q and out)
+ *   max_q_len  host upper bound of any chunk's query count (plans the grid)
+ * This build runs prefill on bf16 pools; E4M3 pools return PKV_ERR_UNSUPPORTED.
+ *   out        bf16 [total_q][num_q_heads][head_dim]
+ *   lse        fp32 [total_q][num_q_heads], or NULL
+ */
+int paged_prefill_chunk_attention(const pkv_cache* cache, const void* q, int32_t num_q_heads,
+                                  int32_t gqa_group, const int32_t* cu_q_lens,
+                                  const int32_t* page_table, int32_t max_pages_per_seq,
+                                  const int32_t* seq_lens, int32_t num_chunks, int32_t total_q,
+                                  int32_t max_q_len, float softmax_scale, void* out, float* lse,
+                                  void* stream);
+
+/* Human-readable name of a pkv_status value (static storage). */
+const char* pkv_status_string(int status);
+
+/* ABI version of this library: (major << 16) | minor. */
+int pkv_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGED_KV_H */

@@ -1,0 +1,263 @@
+"""Attention over a paged KV cache on B200: Python binding of ``libpagedkv.so``.
+
+A thin ctypes layer over the C ABI in ``include/paged_kv.h``: it checks and
+marshals torch tensors (device memory, streams) into plain pointers and sizes
+and calls the library.  Every step of the computation runs in the library's
+CUDA kernels; there is no CPU or PyTorch fallback.  If the library is missing
+or cannot load, importing this package raises.
+
+Entry points (same names as the C ABI):
+    paged_kv_append                 paged store of new tokens' K/V (bf16 or E4M3)
+    paged_decode_attention          split-KV decode, persistent and balanced
+    paged_prefill_chunk_attention   causal prefill chunks on tcgen05
+    paged_decode_workspace_bytes, paged_decode_plan, pkv_status_string
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libpagedkv.so")
+
+PKV_KV_BF16 = 0
+PKV_KV_FP8_E4M3 = 1
+PKV_FLAG_BAD_PAGE = 0x1
+PKV_FLAG_BAD_LENGTH = 0x2
+PKV_FLAG_TIMEOUT = 0x4
+PKV_FLAG_BAD_SCALE = 0x8
+
+# Every symbol include/paged_kv.h declares.
+EXPORTED = (
+    "paged_kv_append",
+    "paged_decode_plan",
+    "paged_decode_workspace_bytes",
+    "paged_decode_attention",
+    "paged_prefill_chunk_attention",
+    "pkv_status_string",
+    "pkv_abi_version",
+)
+
+
+class PkvCache(ctypes.Structure):
+    """Mirror of ``struct pkv_cache``."""
+
+    _fields_ = [
+        ("k_pool", ctypes.c_void_p),
+        ("v_pool", ctypes.c_void_p),
+        ("k_scale", ctypes.c_void_p),
+        ("v_scale", ctypes.c_void_p),
+        ("num_pages", ctypes.c_int32),
+        ("page_size", ctypes.c_int32),
+        ("num_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("kv_dtype", ctypes.c_int32),
+        ("error_flags", ctypes.c_void_p),
+    ]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_476_b200.build` "
+            "(there is no fallback path)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, SZ, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_float
+    cp = ctypes.POINTER(PkvCache)
+    lib.paged_kv_append.argtypes = [cp, P, I32, P, P, I32, I32, P, P, P]
+    lib.paged_kv_append.restype = ctypes.c_int
+    lib.paged_decode_plan.argtypes = [I32, I32, I32, I32, I32, I32, ctypes.POINTER(I32)]
+    lib.paged_decode_plan.restype = ctypes.c_int
+    lib.paged_decode_workspace_bytes.argtypes = [I32, I32, I32, I32, I32, I32]
+    lib.paged_decode_workspace_bytes.restype = SZ
+    lib.paged_decode_attention.argtypes = [cp, P, I32, I32, P, I32, P, I32, I32, F, P, P, P, SZ,
+                                           I32, P]
+    lib.paged_decode_attention.restype = ctypes.c_int
+    lib.paged_prefill_chunk_attention.argtypes = [cp, P, I32, I32, P, P, I32, P, I32, I32, I32,
+                                                  F, P, P, P]
+    lib.paged_prefill_chunk_attention.restype = ctypes.c_int
+    lib.pkv_status_string.argtypes = [ctypes.c_int]
+    lib.pkv_status_string.restype = ctypes.c_char_p
+    lib.pkv_abi_version.restype = ctypes.c_int
+    return lib
+
+
+_lib = _load()
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def pkv_status_string(status: int) -> str:
+    return _lib.pkv_status_string(int(status)).decode()
+
+
+class PagedKVError(RuntimeError):
+    def __init__(self, what: str, status: int):
+        super().__init__(f"{what} failed: {pkv_status_string(status)} (status {status})")
+        self.status = status
+
+
+def _check(what: str, status: int):
+    if status != 0:
+        raise PagedKVError(what, status)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dev(name: str, t: torch.Tensor, dtype=None, ndim=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise ValueError(f"{name} must have dtype {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
+    return t
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+class PagedKVCache:
+    """Caller-owned paged KV pool: K and V ``[num_pages, Hkv, page_size, head_dim]``.
+
+    ``kv_dtype`` is ``"bf16"`` (torch.bfloat16 pools) or ``"e4m3"`` (uint8 or
+    float8_e4m3fn pools plus fp32 ``k_scale``/``v_scale`` ``[num_pages, Hkv]``).
+    ``error_flags`` is an optional int32 device scalar that kernels OR
+    ``PKV_FLAG_*`` bits into.
+    """
+
+    def __init__(self, k_pool, v_pool, kv_dtype="bf16", k_scale=None, v_scale=None,
+                 error_flags=None):
+        if kv_dtype not in ("bf16", "e4m3"):
+            raise ValueError("kv_dtype must be 'bf16' or 'e4m3'")
+        dt = torch.bfloat16 if kv_dtype == "bf16" else (torch.uint8, torch.float8_e4m3fn)
+        _dev("k_pool", k_pool, dt, 4)
+        _dev("v_pool", v_pool, dt, 4)
+        if k_pool.shape != v_pool.shape:
+            raise ValueError("k_pool and v_pool shapes differ")
+        if kv_dtype == "e4m3":
+            if k_scale is None or v_scale is None:
+                raise ValueError("E4M3 pools need k_scale and v_scale")
+            _dev("k_scale", k_scale, torch.float32, 2)
+            _dev("v_scale", v_scale, torch.float32, 2)
+        if error_flags is not None:
+            _dev("error_flags", error_flags, torch.int32)
+        self.k_pool, self.v_pool = k_pool, v_pool
+        self.k_scale, self.v_scale = k_scale, v_scale
+        self.error_flags = error_flags
+        self.kv_dtype = kv_dtype
+        self.num_pages, self.num_kv_heads, self.page_size, self.head_dim = k_pool.shape
+        self._c = PkvCache(k_pool.data_ptr(), v_pool.data_ptr(),
+                           None if k_scale is None else k_scale.data_ptr(),
+                           None if v_scale is None else v_scale.data_ptr(),
+                           self.num_pages, self.page_size, self.num_kv_heads, self.head_dim,
+                           PKV_KV_FP8_E4M3 if kv_dtype == "e4m3" else PKV_KV_BF16,
+                           None if error_flags is None else error_flags.data_ptr())
+
+    @property
+    def c_struct(self) -> PkvCache:
+        return self._c
+
+
+def paged_kv_append(cache: PagedKVCache, page_table, seq_lens_before, cu_new_tokens, k_new,
+                    v_new, total_new_tokens: Optional[int] = None, stream=None) -> None:
+    """Store new tokens' K/V (bf16 ``[T, Hkv, D]``) into their pages."""
+    _dev("page_table", page_table, torch.int32, 2)
+    _dev("seq_lens_before", seq_lens_before, torch.int32, 1)
+    _dev("cu_new_tokens", cu_new_tokens, torch.int32, 1)
+    _dev("k_new", k_new, torch.bfloat16, 3)
+    _dev("v_new", v_new, torch.bfloat16, 3)
+    T = k_new.shape[0] if total_new_tokens is None else int(total_new_tokens)
+    st = _lib.paged_kv_append(ctypes.byref(cache.c_struct), _ptr(page_table),
+                              page_table.shape[1], _ptr(seq_lens_before), _ptr(cu_new_tokens),
+                              seq_lens_before.shape[0], T, _ptr(k_new), _ptr(v_new),
+                              _stream(stream))
+    _check("paged_kv_append", st)
+
+
+def paged_decode_plan(batch, num_kv_heads, max_seq_len, num_sms, num_ctas=0, ctas_per_sm=1):
+    out = ctypes.c_int32(0)
+    _check("paged_decode_plan", _lib.paged_decode_plan(batch, num_kv_heads, max_seq_len,
+                                                       num_sms, num_ctas, ctas_per_sm,
+                                                       ctypes.byref(out)))
+    return out.value
+
+
+def paged_decode_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim, max_seq_len,
+                                 num_ctas=0) -> int:
+    n = _lib.paged_decode_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim,
+                                          max_seq_len, num_ctas)
+    if n == 0:
+        raise PagedKVError("paged_decode_workspace_bytes", -2)
+    return int(n)
+
+
+def decode_workspace(cache: PagedKVCache, batch, num_q_heads, max_seq_len, num_ctas=0):
+    """A zero-filled workspace tensor for paged_decode_attention."""
+    n = paged_decode_workspace_bytes(batch, num_q_heads, cache.num_kv_heads, cache.head_dim,
+                                     max_seq_len, num_ctas)
+    return torch.zeros(n, dtype=torch.uint8, device=cache.k_pool.device)
+
+
+def paged_decode_attention(cache: PagedKVCache, q, page_table, seq_lens, max_seq_len: int,
+                           softmax_scale: Optional[float] = None, out=None, lse=None,
+                           workspace=None, num_ctas: int = 0, want_lse: bool = True,
+                           stream=None):
+    """Decode attention of ``q`` bf16 ``[B, Hq, D]`` over the paged cache.
+
+    Returns ``(out bf16 [B, Hq, D], lse fp32 [B, Hq] or None)``.
+    """
+    _dev("q", q, torch.bfloat16, 3)
+    _dev("page_table", page_table, torch.int32, 2)
+    _dev("seq_lens", seq_lens, torch.int32, 1)
+    B, Hq, D = q.shape
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = decode_workspace(cache, B, Hq, max_seq_len, num_ctas)
+    st = _lib.paged_decode_attention(
+        ctypes.byref(cache.c_struct), _ptr(q), Hq, Hq // cache.num_kv_heads, _ptr(page_table),
+        page_table.shape[1], _ptr(seq_lens), B, int(max_seq_len), float(softmax_scale),
+        _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), int(num_ctas), _stream(stream))
+    _check("paged_decode_attention", st)
+    return out, lse
+
+
+def paged_prefill_chunk_attention(cache: PagedKVCache, q, cu_q_lens, page_table, seq_lens,
+                                  max_q_len: int, softmax_scale: Optional[float] = None,
+                                  out=None, lse=None, want_lse: bool = True, stream=None):
+    """Causal chunk attention of packed ``q`` bf16 ``[Tq, Hq, D]`` over the paged cache."""
+    _dev("q", q, torch.bfloat16, 3)
+    _dev("cu_q_lens", cu_q_lens, torch.int32, 1)
+    _dev("page_table", page_table, torch.int32, 2)
+    _dev("seq_lens", seq_lens, torch.int32, 1)
+    T, Hq, D = q.shape
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
+    st = _lib.paged_prefill_chunk_attention(
+        ctypes.byref(cache.c_struct), _ptr(q), Hq, Hq // cache.num_kv_heads, _ptr(cu_q_lens),
+        _ptr(page_table), page_table.shape[1], _ptr(seq_lens), seq_lens.shape[0], T,
+        int(max_q_len), float(softmax_scale), _ptr(out), _ptr(lse), _stream(stream))
+    _check("paged_prefill_chunk_attention", st)
+    return out, lse

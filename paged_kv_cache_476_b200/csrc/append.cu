@@ -1,0 +1,102 @@
+// Paged KV append: the paged store of this step's new tokens.
+//
+// TensorRT-LLM concept page, "PagedAttention 及 KV 快取管理" and
+// "編譯期圖最佳化": the K/V of a token is written to the physical page that the
+// sequence's page table names for the token's logical position.
+//
+// One thread moves one 16-byte vector (8 bf16) of one token's K or V row:
+// loads are coalesced over [token][kv head][d]; each warp writes whole
+// 16-byte chunks of a contiguous page row.  bf16 pools receive the bits;
+// E4M3 pools receive e4m3_rne_satfinite(x / scale) computed with an IEEE
+// fp32 division and the hardware satfinite conversion.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace pkv {
+
+
+// Index of the sequence owning new token `tok`: the last b with cu_new[b] <= tok.
+__device__ __forceinline__ int owner_of(const int32_t* cu_new, int batch, int tok) {
+  int lo = 0, hi = batch - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (__ldg(cu_new + mid) <= tok)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo;
+}
+
+template <bool kFp8>
+__global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
+  const int vecs_per_row = p.head_dim / 8;                 // 16-byte vectors per (token, head)
+  const int64_t per_token = (int64_t)p.num_kv_heads * vecs_per_row;
+  const int64_t total = (int64_t)p.total_new * per_token;  // vectors of K (and of V)
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < 2 * total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const bool is_v = i >= total;
+    const int64_t e = is_v ? i - total : i;
+    const int tok = static_cast<int>(e / per_token);
+    const int rem = static_cast<int>(e - (int64_t)tok * per_token);
+    const int g = rem / vecs_per_row;
+    const int vec = rem - g * vecs_per_row;
+
+    const int b = owner_of(p.cu_new, p.batch, tok);
+    const int64_t pos = (int64_t)__ldg(p.seq_lens_before + b) + (tok - __ldg(p.cu_new + b));
+    const int64_t j = pos / p.page_size;
+    if (pos < 0 || j >= p.max_pages) {
+      if (vec == 0 && g == 0 && !is_v) flag_error(p.flags, PKV_FLAG_BAD_LENGTH);
+      continue;
+    }
+    const int32_t page = __ldg(p.page_table + (int64_t)b * p.max_pages + j);
+    if (page < 0 || page >= p.num_pages) {
+      if (vec == 0 && g == 0 && !is_v) flag_error(p.flags, PKV_FLAG_BAD_PAGE);
+      continue;
+    }
+    const int slot = static_cast<int>(pos - j * p.page_size);
+    const uint4 src = __ldg((is_v ? p.v_new : p.k_new) + e);
+    // element index of the first of the 8 values inside the pool
+    const int64_t dst_elem =
+        (((int64_t)page * p.num_kv_heads + g) * p.page_size + slot) * p.head_dim + vec * 8;
+    uint8_t* pool = is_v ? p.v_pool : p.k_pool;
+    if constexpr (!kFp8) {
+      *reinterpret_cast<uint4*>(pool + dst_elem * 2) = src;
+    } else {
+      const float s = __ldg((is_v ? p.v_scale : p.k_scale) + (int64_t)page * p.num_kv_heads + g);
+      if (!(s > 0.f && s <= 32768.f)) {
+        if (vec == 0) flag_error(p.flags, PKV_FLAG_BAD_SCALE);
+      }
+      const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&src);
+      uint32_t w[2];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float2 f = __bfloat1622float2(x[k]);
+        f.x = __fdiv_rn(f.x, s);
+        f.y = __fdiv_rn(f.y, s);
+        const uint16_t two = __nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
+        if (k & 1)
+          w[k >> 1] |= static_cast<uint32_t>(two) << 16;
+        else
+          w[k >> 1] = two;
+      }
+      *reinterpret_cast<uint2*>(pool + dst_elem) = make_uint2(w[0], w[1]);
+    }
+  }
+}
+
+cudaError_t launch_append(const AppendParams& p, bool fp8, int num_sms, cudaStream_t stream) {
+  const int64_t vectors = 2LL * p.total_new * p.num_kv_heads * (p.head_dim / 8);
+  if (vectors == 0) return cudaSuccess;
+  const int threads = 256;
+  int64_t blocks = (vectors + threads - 1) / threads;
+  const int64_t cap = (int64_t)num_sms * 8;
+  if (blocks > cap) blocks = cap;
+  if (fp8)
+    append_kernel<true><<<(unsigned)blocks, threads, 0, stream>>>(p);
+  else
+    append_kernel<false><<<(unsigned)blocks, threads, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace pkv

@@ -1,0 +1,694 @@
+// Split-KV decode attention over a paged KV cache (sm_100a).
+//
+// What it computes (TensorRT-LLM concept page, "執行時執行模型": every step the
+// attention operator reads the KV pages; "PagedAttention 及 KV 快取管理": pages
+// are found through a per-sequence page table): for each sequence b and q head
+// h, out = softmax(scale * q K_b^T) V_b over the seq_lens[b] cached tokens.
+//
+// Design (B200-first, HBM-bound):
+//  * Work list.  Each (sequence, kv head) pair is a unit; a unit's tokens are
+//    cut into 64-token tiles.  The units' tiles, concatenated in (b, g) order,
+//    are split into C equal contiguous ranges, one per CTA, with C = SMs x
+//    resident CTAs per SM: one persistent wave, no tail of unequal splits.
+//  * A range cuts a unit into segments.  A segment computes an online-softmax
+//    partial (m, l, unnormalised o) for the unit's G = Hq/Hkv q heads.  A
+//    segment that covers its whole unit writes the output directly; otherwise
+//    it stores its partial and bumps the unit's counter, and the last segment
+//    to arrive merges all of them (the split-KV reduction, same launch).
+//  * Warp roles: one producer warp walks the range and issues TMA loads of
+//    the K and V tile (page-table indirected, 128-byte swizzled) into a
+//    multi-stage mbarrier ring, plus a bulk copy of Q at each segment start;
+//    four consumer warps each take 16 of a tile's 64 tokens and run
+//    S = Q K^T and O += P V on mma.sync (bf16, or f16 for E4M3 K/V which
+//    converts exactly), with the online softmax in registers.
+//  * E4M3 K/V: K codes are converted to f16 in registers after ldmatrix (the
+//    d order inside each 16-wide block is permuted identically in Q); V codes
+//    are converted into a per-warp f16 tile for the transposed ldmatrix.  The
+//    per-(page, head) scales fold into the scores (K) and into P (V).
+//  * Every wait is bounded; a bad page id or length is skipped and flagged.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace pkv {
+
+constexpr int kTile = 64;           // tokens per pipeline tile
+constexpr int kConsumerWarps = 4;   // 16 tokens of each tile per warp
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kMaxGroup = 8;
+
+// TileInfo.flags
+constexpr int kSegFirst = 1;   // first tile of a segment: reset state, Q in this stage
+constexpr int kSegLast = 2;    // last tile of a segment: flush after it
+constexpr int kUnitWhole = 4;  // the segment is the whole unit: write out directly
+constexpr int kBadTile = 8;    // page id invalid: tile skipped
+
+
+struct TileInfo {
+  int32_t b, g, tile, valid;  // valid = tokens of this tile below the length
+  int32_t flags;
+  int32_t slot;      // partial slot of this CTA's segment
+  int32_t seg_base;  // first partial slot of the unit
+  int32_t nseg;      // segments of the unit
+  float ks, vs;      // E4M3 scales of the tile's page
+};
+
+template <int D, bool kFp8>
+struct Layout {
+  static constexpr int kEB = kFp8 ? 1 : 2;
+  static constexpr int kRowB = D * kEB;                        // bytes of a token row
+  static constexpr int kBoxRowB = kRowB >= 128 ? 128 : kRowB;  // TMA box inner bytes
+  static constexpr int kNumBox = kRowB / kBoxRowB;             // boxes per tile row
+  static constexpr int kBoxB = kTile * kBoxRowB;
+  static constexpr int kTileB = kNumBox * kBoxB;  // one K (or V) tile
+  static constexpr int kStageB = 2 * kTileB;
+  static constexpr int kQB = kMaxGroup * D * 2;    // Q slice per stage
+  static constexpr int kConvB = 16 * D * 2;        // per-warp f16 V tile (E4M3 only)
+  static constexpr bool kSw64 = kBoxRowB == 64;
+};
+
+// Byte address of 16-byte chunk `chunk` of row `row` in a TMA-swizzled tile
+// made of kNumBox boxes of [rows][kBoxRowB].
+template <int kBoxRowB, int kRows>
+__device__ __forceinline__ uint32_t tile_addr(uint32_t base, int row, int chunk) {
+  constexpr int kChunksPerBox = kBoxRowB / 16;
+  const int box = chunk / kChunksPerBox;
+  const int c = chunk % kChunksPerBox;
+  const uint32_t off = row * kBoxRowB + c * 16;
+  const uint32_t sw = kBoxRowB == 128 ? swz128(off) : swz64(off);
+  return base + box * (kRows * kBoxRowB) + sw;
+}
+
+// CTA (of C <= T over T tiles) whose range [c*T/C, (c+1)*T/C) holds global
+// tile x.  With C <= T every range holds at least one tile.
+__device__ __forceinline__ int64_t cta_of(int64_t x, int64_t C, int64_t T) {
+  return ((x + 1) * C - 1) / T;
+}
+
+__device__ __forceinline__ int tiles_of(int32_t len) { return (len + kTile - 1) / kTile; }
+
+__device__ __forceinline__ int32_t clamp_len(const DecodeParams& p, int32_t len, bool report) {
+  const int32_t cap = p.max_pages * p.page_size;
+  if (len < 0 || len > cap) {
+    if (report) flag_error(p.flags, PKV_FLAG_BAD_LENGTH);
+    return len < 0 ? 0 : cap;
+  }
+  return len;
+}
+
+// A CTA-internal barrier among the consumer warps built on an mbarrier, so
+// that every wait is bounded (a named barrier could wait forever).
+struct ConsumerSync {
+  uint64_t* bar;
+  uint32_t phase;
+  __device__ __forceinline__ bool sync(int32_t* flags) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+    const bool ok = mbar_wait(bar, phase, flags);
+    phase ^= 1;
+    return ok;
+  }
+};
+
+template <int D, bool kFp8, int kStages>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                  const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
+  using Ly = Layout<D, kFp8>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte align the dynamic window (the swizzle pattern needs it).
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* tiles = smem;
+  uint8_t* qbuf = tiles + kStages * Ly::kStageB;
+  uint8_t* conv = qbuf + kStages * Ly::kQB;
+  float* red_o = reinterpret_cast<float*>(conv + (kFp8 ? kConsumerWarps * Ly::kConvB : 0));
+  float* red_m = red_o + kConsumerWarps * kMaxGroup * D;
+  float* red_l = red_m + kConsumerWarps * kMaxGroup;
+  uint64_t* full = reinterpret_cast<uint64_t*>(red_l + kConsumerWarps * kMaxGroup);
+  uint64_t* empty = full + kStages;
+  uint64_t* merge_bar = empty + kStages;
+  TileInfo* info = reinterpret_cast<TileInfo*>(merge_bar + 1);
+  int32_t* s_misc = reinterpret_cast<int32_t*>(info + kStages);  // [0]=n tiles, [1]=is_last
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int G = p.group;
+  const int Hkv = p.num_kv_heads;
+  const int64_t C = gridDim.x;
+  const int64_t c = blockIdx.x;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    mbar_init(merge_bar, kConsumerWarps);
+    fence_barrier_init();
+  }
+
+  // ------------------------------------------------ producer: plan + loads
+  int64_t n_tiles = 0;
+  int pb = 0, pg = 0, pt = 0;  // producer's position (b, g, tile) at the range start
+  int64_t range_start = 0, T = 0, Ce = 1;
+  if (warp == kConsumerWarps) {
+    // Total tiles over all units.
+    int64_t tot = 0;
+    for (int base = 0; base < p.batch; base += 32) {
+      const int b = base + lane;
+      const int t = b < p.batch ? tiles_of(clamp_len(p, __ldg(p.seq_lens + b), c == 0)) : 0;
+      tot += t;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    T = tot * Hkv;
+    // Only min(C, T) CTAs take work, so that every working range is
+    // non-empty and a unit's segment count equals the CTAs that touch it.
+    Ce = C < T ? C : T;
+    if (c < Ce) {
+      range_start = (c * T) / Ce;
+      n_tiles = ((c + 1) * T) / Ce - range_start;
+    }
+    // Empty sequences (length 0): out = 0, lse = -inf, written by one CTA each.
+    for (int b = (int)((c * p.batch) / C); b < (int)(((c + 1) * p.batch) / C); ++b) {
+      if (clamp_len(p, __ldg(p.seq_lens + b), false) == 0) {
+        for (int i = lane; i < p.num_q_heads * D; i += 32)
+          p.out[(int64_t)b * p.num_q_heads * D + i] = __float2bfloat16(0.f);
+        if (p.lse)
+          for (int h = lane; h < p.num_q_heads; h += 32)
+            p.lse[(int64_t)b * p.num_q_heads + h] = -INFINITY;
+      }
+    }
+    if (n_tiles > 0) {
+      // Locate (b, g, tile) of global tile range_start.
+      int64_t run = 0;
+      for (int base = 0; base < p.batch; base += 32) {
+        const int b = base + lane;
+        const int t = b < p.batch ? tiles_of(clamp_len(p, __ldg(p.seq_lens + b), false)) : 0;
+        int incl = t;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const int chunk = __shfl_sync(0xffffffffu, incl, 31);
+        if (run + (int64_t)chunk * Hkv > range_start) {
+          const bool hit = run + (int64_t)incl * Hkv > range_start;
+          const unsigned m = __ballot_sync(0xffffffffu, hit);
+          const int l0 = __ffs(m) - 1;
+          const int t0 = __shfl_sync(0xffffffffu, t, l0);
+          const int e0 = __shfl_sync(0xffffffffu, incl - t, l0);
+          pb = base + l0;
+          const int64_t off = range_start - (run + (int64_t)e0 * Hkv);
+          pg = (int)(off / t0);
+          pt = (int)(off - (int64_t)pg * t0);
+          break;
+        }
+        run += (int64_t)chunk * Hkv;
+      }
+    }
+    if (lane == 0) s_misc[0] = (int)n_tiles;
+  }
+  __syncthreads();
+  n_tiles = s_misc[0];
+  if (n_tiles == 0) return;
+
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------ producer loop
+    const uint64_t pol = policy_evict_first();
+    if (lane == 0) {
+      tma_prefetch_desc(&tmap_k);
+      tma_prefetch_desc(&tmap_v);
+    }
+    const int tiles_per_page = p.page_size / kTile;
+    int b = pb, g = pg, t = pt;
+    int len = clamp_len(p, __ldg(p.seq_lens + b), false);
+    int ntile = tiles_of(len);
+    int seg_first_t = t;
+    // page ids (and E4M3 scales) of 32 consecutive pages, one per lane
+    int cache_key = -1, cache_j0 = 0;
+    int my_pid = 0;
+    float my_ks = 1.f, my_vs = 1.f;
+    int64_t x = range_start;  // global tile index
+    int issued = 0;
+    bool ok = true;
+    for (int64_t i = 0; i < n_tiles; ++i, ++x) {
+      const int stage = (int)(i % kStages);
+      if (i >= kStages) {
+        if (!mbar_wait(&empty[stage], (uint32_t)((i / kStages - 1) & 1), p.flags)) {
+          ok = false;
+          break;
+        }
+      }
+      const int j = t / tiles_per_page;
+      const int sub = t - j * tiles_per_page;
+      const int pages_b = (len + p.page_size - 1) / p.page_size;
+      const int key = kFp8 ? b * Hkv + g : b;
+      if (cache_key != key || j < cache_j0 || j >= cache_j0 + 32) {
+        cache_key = key;
+        cache_j0 = j;
+        const int jj = j + lane;
+        my_pid = jj < pages_b ? __ldg(p.page_table + (int64_t)b * p.max_pages + jj) : 0;
+        if constexpr (kFp8) {
+          if (jj < pages_b && my_pid >= 0 && my_pid < p.num_pages) {
+            my_ks = __ldg(p.k_scale + (int64_t)my_pid * Hkv + g);
+            my_vs = __ldg(p.v_scale + (int64_t)my_pid * Hkv + g);
+          }
+        }
+      }
+      int pid = __shfl_sync(0xffffffffu, my_pid, j - cache_j0);
+      float ks = 1.f, vs = 1.f;
+      if constexpr (kFp8) {
+        ks = __shfl_sync(0xffffffffu, my_ks, j - cache_j0);
+        vs = __shfl_sync(0xffffffffu, my_vs, j - cache_j0);
+      }
+      bool bad = pid < 0 || pid >= p.num_pages;
+      if constexpr (kFp8) {
+        if (!bad && !(ks > 0.f && ks <= 32768.f && vs > 0.f && vs <= 32768.f)) {
+          bad = true;
+          if (lane == 0) flag_error(p.flags, PKV_FLAG_BAD_SCALE);
+        }
+      }
+      if (pid < 0 || pid >= p.num_pages) {
+        if (lane == 0) flag_error(p.flags, PKV_FLAG_BAD_PAGE);
+      }
+      if (bad) pid = 0;
+      const bool first = (i == 0) || (t == 0);
+      if (first) seg_first_t = t;
+      const bool last = (i == n_tiles - 1) || (t == ntile - 1);
+      if (lane == 0) {
+        TileInfo ti;
+        ti.b = b;
+        ti.g = g;
+        ti.tile = t;
+        ti.valid = min(kTile, len - t * kTile);
+        ti.flags = (first ? kSegFirst : 0) | (last ? kSegLast : 0) | (bad ? kBadTile : 0);
+        if (last && seg_first_t == 0 && t == ntile - 1) ti.flags |= kUnitWhole;
+        const int64_t u = (int64_t)b * Hkv + g;
+        const int64_t x_unit = x - t;  // global index of the unit's first tile
+        const int64_t c_first = cta_of(x_unit, Ce, T);
+        const int64_t c_last = cta_of(x_unit + ntile - 1, Ce, T);
+        ti.seg_base = (int)(u + c_first);
+        ti.nseg = (int)(c_last - c_first + 1);
+        ti.slot = (int)(u + c);
+        ti.ks = ks;
+        ti.vs = vs;
+        info[stage] = ti;
+        const uint32_t qbytes = first ? (uint32_t)(G * D * 2) : 0u;
+        mbar_arrive_expect_tx(&full[stage], (uint32_t)Ly::kStageB + qbytes);
+        const int32_t y = (int32_t)(((int64_t)pid * Hkv + g) * p.page_size + sub * kTile);
+        uint8_t* kdst = tiles + stage * Ly::kStageB;
+        uint8_t* vdst = kdst + Ly::kTileB;
+#pragma unroll
+        for (int bx = 0; bx < Ly::kNumBox; ++bx) {
+          const int32_t xc = bx * (Ly::kBoxRowB / Ly::kEB);
+          tma_load_2d(kdst + bx * Ly::kBoxB, &tmap_k, xc, y, &full[stage], pol);
+          tma_load_2d(vdst + bx * Ly::kBoxB, &tmap_v, xc, y, &full[stage], pol);
+        }
+        if (first) {
+          const __nv_bfloat16* src = p.q + ((int64_t)b * p.num_q_heads + (int64_t)g * G) * D;
+          asm volatile(
+              "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, "
+              "[%3];" ::"r"(smem_u32(qbuf + stage * Ly::kQB)),
+              "l"(reinterpret_cast<uint64_t>(src)), "r"(qbytes), "r"(smem_u32(&full[stage]))
+              : "memory");
+        }
+      }
+      __syncwarp();
+      ++issued;
+      // advance to the next tile of the work list
+      if (++t == ntile) {
+        t = 0;
+        if (++g == Hkv) {
+          g = 0;
+          do {
+            ++b;
+          } while (b < p.batch && tiles_of(clamp_len(p, __ldg(p.seq_lens + b), false)) == 0);
+          if (b < p.batch) {
+            len = clamp_len(p, __ldg(p.seq_lens + b), false);
+            ntile = tiles_of(len);
+          }
+        }
+      }
+    }
+    // Drain: wait (bounded) until the last issued loads have landed, so no
+    // bulk copy is in flight into this CTA's shared memory when it exits.
+    const int64_t lo = issued > kStages ? issued - kStages : 0;
+    for (int64_t k = lo; k < issued; ++k)
+      mbar_wait(&full[k % kStages], (uint32_t)((k / kStages) & 1), p.flags);
+    (void)ok;
+    return;
+  }
+
+  // ---------------------------------------------------------- consumers
+  const int gid = lane >> 2;   // row of the mma fragment = q head within the group
+  const int tid4 = lane & 3;
+  const int mat = lane >> 3;   // which 8x8 matrix this lane addresses in ldmatrix.x4
+  const int mrow = lane & 7;
+  const bool row_ok = gid < G;
+  ConsumerSync csync{merge_bar, 0};
+
+  constexpr int KS = D / 16;  // k-steps over head_dim
+  uint32_t qa[KS][2];         // A fragments of Q: rows gid, two k halves
+  float o[D / 8][4];
+  float m_run = -INFINITY, l_part = 0.f;
+  float qk_mul = p.scale_log2;  // multiplier of the raw scores into log2 units
+
+  for (int64_t i = 0; i < n_tiles; ++i) {
+    const int stage = (int)(i % kStages);
+    if (!mbar_wait(&full[stage], (uint32_t)((i / kStages) & 1), p.flags)) return;
+    const TileInfo ti = info[stage];
+    const uint8_t* qs = qbuf + stage * Ly::kQB;
+    if (ti.flags & kSegFirst) {
+      m_run = -INFINITY;
+      l_part = 0.f;
+#pragma unroll
+      for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+      if constexpr (!kFp8) {
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+          const uint32_t* qrow = reinterpret_cast<const uint32_t*>(qs + gid * D * 2);
+          qa[kk][0] = row_ok ? qrow[(16 * kk + 2 * tid4) / 2] : 0u;
+          qa[kk][1] = row_ok ? qrow[(16 * kk + 8 + 2 * tid4) / 2] : 0u;
+        }
+        qk_mul = p.scale_log2;
+      } else {
+        // f16 Q with a per-row power-of-two prescale; inside each 16-wide d
+        // block, the fragment's k pair (2*tid4, +1) holds d = 4*tid4 + {0,1}
+        // and the pair (2*tid4+8, +9) holds d = 4*tid4 + {2,3}, matching the
+        // byte order of the E4M3 K rows delivered by ldmatrix.
+        float amax = 0.f;
+        float qv[KS][4];
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+          const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(qs) + gid * D;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            qv[kk][e] = row_ok ? __bfloat162float(qrow[16 * kk + 4 * tid4 + e]) : 0.f;
+            amax = fmaxf(amax, fabsf(qv[kk][e]));
+          }
+        }
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        int ex = 0;
+        if (amax > 0.f) {
+          frexpf(amax, &ex);  // amax < 2^ex
+          ex = 14 - ex;       // amax * 2^ex < 2^14
+          ex = max(-100, min(100, ex));
+        }
+        const float pre = ldexpf(1.f, ex);
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+          qa[kk][0] = pack_f16(qv[kk][0] * pre, qv[kk][1] * pre);
+          qa[kk][1] = pack_f16(qv[kk][2] * pre, qv[kk][3] * pre);
+        }
+        qk_mul = p.scale_log2 * ldexpf(1.f, -ex);
+      }
+    }
+
+    const int valid = (ti.flags & kBadTile) ? 0 : ti.valid - 16 * warp;  // tokens of my 16
+    if (valid > 0) {
+      const uint32_t kbase = smem_u32(tiles + stage * Ly::kStageB);
+      const uint32_t vbase = kbase + Ly::kTileB;
+      // ---- S = Q K^T over my 16 tokens (two n-tiles of 8) ----
+      float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      if constexpr (!kFp8) {
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+          const int row = 16 * warp + mrow + (mat >> 1) * 8;
+          const int chunk = 2 * kk + (mat & 1);
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(tile_addr<Ly::kBoxRowB, kTile>(kbase, row, chunk), b0, b1, b2, b3);
+          mma_bf16(s[0], qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
+          mma_bf16(s[1], qa[kk][0], 0u, qa[kk][1], 0u, b2, b3);
+        }
+      } else {
+#pragma unroll
+        for (int kp = 0; kp < KS / 2; ++kp) {
+          // matrices: (tokens 0-7, chunk 2kp), (0-7, 2kp+1), (8-15, 2kp), (8-15, 2kp+1)
+          const int row = 16 * warp + mrow + (mat >> 1) * 8;
+          const int chunk = 2 * kp + (mat & 1);
+          uint32_t r0, r1, r2, r3;
+          ldsm_x4(tile_addr<Ly::kBoxRowB, kTile>(kbase, row, chunk), r0, r1, r2, r3);
+          mma_f16(s[0], qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, e4m3x2_to_f16x2(r0 & 0xffff),
+                  e4m3x2_to_f16x2(r0 >> 16));
+          mma_f16(s[0], qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u,
+                  e4m3x2_to_f16x2(r1 & 0xffff), e4m3x2_to_f16x2(r1 >> 16));
+          mma_f16(s[1], qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, e4m3x2_to_f16x2(r2 & 0xffff),
+                  e4m3x2_to_f16x2(r2 >> 16));
+          mma_f16(s[1], qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u,
+                  e4m3x2_to_f16x2(r3 & 0xffff), e4m3x2_to_f16x2(r3 >> 16));
+        }
+      }
+      // ---- online softmax on row gid (log2 domain) ----
+      const float mul = kFp8 ? qk_mul * ti.ks : qk_mul;
+      float x[4];
+#pragma unroll
+      for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int tok = 8 * n + 2 * tid4 + e;
+          x[2 * n + e] = tok < valid ? s[n][e] * mul : -INFINITY;
+        }
+      float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float m_new = fmaxf(m_run, mx);  // finite: valid > 0
+      const float alpha = fast_exp2(m_run - m_new);
+      float pr[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) pr[e] = fast_exp2(x[e] - m_new);
+      l_part = l_part * alpha + (pr[0] + pr[1]) + (pr[2] + pr[3]);
+      m_run = m_new;
+#pragma unroll
+      for (int n = 0; n < D / 8; ++n) {
+        o[n][0] *= alpha;
+        o[n][1] *= alpha;
+      }
+      // ---- O += P V over my 16 tokens ----
+      uint32_t pa0, pa2;
+      if constexpr (!kFp8) {
+        pa0 = pack_bf16(pr[0], pr[1]);
+        pa2 = pack_bf16(pr[2], pr[3]);
+      } else {
+        pa0 = pack_f16(pr[0] * ti.vs, pr[1] * ti.vs);
+        pa2 = pack_f16(pr[2] * ti.vs, pr[3] * ti.vs);
+      }
+      // V rows past the length may hold anything (NaN); zero them in the
+      // fragments so that 0 * NaN never reaches the accumulator.
+      uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;
+      if (valid < 16) {
+        vm0 = (2 * tid4 < valid ? 0x0000ffffu : 0u) | (2 * tid4 + 1 < valid ? 0xffff0000u : 0u);
+        vm1 = (2 * tid4 + 8 < valid ? 0x0000ffffu : 0u) |
+              (2 * tid4 + 9 < valid ? 0xffff0000u : 0u);
+      }
+      uint32_t vsrc;
+      if constexpr (!kFp8) {
+        vsrc = vbase;
+      } else {
+        // E4M3 -> f16 copy of my 16 V rows into my conversion tile, laid out
+        // like a bf16 tile (256-byte rows as two 128-byte swizzled boxes).
+        uint8_t* cv = conv + warp * Ly::kConvB;
+        const uint32_t cbase = smem_u32(cv);
+        constexpr int kChunks = 16 * D / 16;  // 16-byte E4M3 chunks of my rows
+#pragma unroll
+        for (int k = 0; k < kChunks / 32; ++k) {
+          const int ci = lane + 32 * k;
+          const int r = ci / (D / 16);
+          const int ch = ci % (D / 16);
+          uint4 raw;
+          const uint32_t src = tile_addr<Ly::kBoxRowB, kTile>(vbase, 16 * warp + r, ch);
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(raw.x), "=r"(raw.y), "=r"(raw.z), "=r"(raw.w)
+                       : "r"(src));
+          uint4 h0, h1;
+          h0.x = e4m3x2_to_f16x2(raw.x & 0xffff);
+          h0.y = e4m3x2_to_f16x2(raw.x >> 16);
+          h0.z = e4m3x2_to_f16x2(raw.y & 0xffff);
+          h0.w = e4m3x2_to_f16x2(raw.y >> 16);
+          h1.x = e4m3x2_to_f16x2(raw.z & 0xffff);
+          h1.y = e4m3x2_to_f16x2(raw.z >> 16);
+          h1.z = e4m3x2_to_f16x2(raw.w & 0xffff);
+          h1.w = e4m3x2_to_f16x2(raw.w >> 16);
+          const uint32_t d0 = tile_addr<128, 16>(cbase, r, 2 * ch);
+          const uint32_t d1 = tile_addr<128, 16>(cbase, r, 2 * ch + 1);
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(d0), "r"(h0.x),
+                       "r"(h0.y), "r"(h0.z), "r"(h0.w)
+                       : "memory");
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(d1), "r"(h1.x),
+                       "r"(h1.y), "r"(h1.z), "r"(h1.w)
+                       : "memory");
+        }
+        __syncwarp();
+        vsrc = cbase;
+      }
+#pragma unroll
+      for (int dp = 0; dp < D / 16; ++dp) {
+        // matrices: (tokens 0-7, d-chunk 2dp), (8-15, 2dp), (0-7, 2dp+1), (8-15, 2dp+1)
+        const int chunk = 2 * dp + (mat >> 1);
+        uint32_t v0, v1, v2, v3;
+        if constexpr (!kFp8) {
+          const int row = 16 * warp + mrow + (mat & 1) * 8;
+          ldsm_x4_t(tile_addr<Ly::kBoxRowB, kTile>(vsrc, row, chunk), v0, v1, v2, v3);
+        } else {
+          const int row = mrow + (mat & 1) * 8;
+          ldsm_x4_t(tile_addr<128, 16>(vsrc, row, chunk), v0, v1, v2, v3);
+        }
+        v0 &= vm0;
+        v2 &= vm0;
+        v1 &= vm1;
+        v3 &= vm1;
+        if constexpr (!kFp8) {
+          mma_bf16(o[2 * dp], pa0, 0u, pa2, 0u, v0, v1);
+          mma_bf16(o[2 * dp + 1], pa0, 0u, pa2, 0u, v2, v3);
+        } else {
+          mma_f16(o[2 * dp], pa0, 0u, pa2, 0u, v0, v1);
+          mma_f16(o[2 * dp + 1], pa0, 0u, pa2, 0u, v2, v3);
+        }
+      }
+    }
+    // release the stage (all of this warp's reads of it are done)
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stage]);
+
+    if (!(ti.flags & kSegLast)) continue;
+
+    // ----------------------------------------------------------- flush
+    float l_row = l_part;
+    l_row += __shfl_xor_sync(0xffffffffu, l_row, 1);
+    l_row += __shfl_xor_sync(0xffffffffu, l_row, 2);
+    if (row_ok) {
+      if (tid4 == 0) {
+        red_m[warp * kMaxGroup + gid] = m_run;
+        red_l[warp * kMaxGroup + gid] = l_row;
+      }
+      float* ro = red_o + (warp * kMaxGroup + gid) * D;
+#pragma unroll
+      for (int n = 0; n < D / 8; ++n)
+        *reinterpret_cast<float2*>(ro + 8 * n + 2 * tid4) = make_float2(o[n][0], o[n][1]);
+    }
+    if (!csync.sync(p.flags)) return;
+    const bool whole = ti.flags & kUnitWhole;
+    const int ctid = threadIdx.x;  // 0..127
+    for (int e = ctid; e < G * D; e += kConsumerWarps * 32) {
+      const int row = e / D;
+      const int d = e - row * D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red_m[w * kMaxGroup + row]);
+      float num = 0.f, den = 0.f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float mw = red_m[w * kMaxGroup + row];
+          if (mw == -INFINITY) continue;
+          const float sc = exp2f(mw - M);
+          num += sc * red_o[(w * kMaxGroup + row) * D + d];
+          den += sc * red_l[w * kMaxGroup + row];
+        }
+      }
+      const int h = ti.g * G + row;
+      const int64_t orow = (int64_t)ti.b * p.num_q_heads + h;
+      if (whole) {
+        p.out[orow * D + d] = __float2bfloat16(den > 0.f ? num / den : 0.f);
+        if (d == 0 && p.lse)
+          p.lse[orow] = den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
+      } else {
+        p.part_o[((int64_t)ti.slot * G + row) * D + d] = num;
+        if (d == 0) p.part_ml[(int64_t)ti.slot * G + row] = make_float2(M, den);
+      }
+    }
+    if (!whole) {
+      __threadfence();
+      if (!csync.sync(p.flags)) return;
+      if (ctid == 0) {
+        const int u = ti.b * Hkv + ti.g;
+        const int old = atomicAdd(p.counters + u, 1);
+        s_misc[1] = (old == ti.nseg - 1);
+      }
+      if (!csync.sync(p.flags)) return;
+      if (s_misc[1]) {
+        __threadfence();
+        for (int e = ctid; e < G * D; e += kConsumerWarps * 32) {
+          const int row = e / D;
+          const int d = e - row * D;
+          float M = -INFINITY;
+          for (int s = 0; s < ti.nseg; ++s)
+            M = fmaxf(M, __ldcg(&p.part_ml[(int64_t)(ti.seg_base + s) * G + row]).x);
+          float num = 0.f, den = 0.f;
+          if (M != -INFINITY) {
+            for (int s = 0; s < ti.nseg; ++s) {
+              const float2 ml = __ldcg(&p.part_ml[(int64_t)(ti.seg_base + s) * G + row]);
+              if (ml.x == -INFINITY) continue;
+              const float sc = exp2f(ml.x - M);
+              num += sc * __ldcg(&p.part_o[((int64_t)(ti.seg_base + s) * G + row) * D + d]);
+              den += sc * ml.y;
+            }
+          }
+          const int64_t orow = (int64_t)ti.b * p.num_q_heads + ti.g * G + row;
+          p.out[orow * D + d] = __float2bfloat16(den > 0.f ? num / den : 0.f);
+          if (d == 0 && p.lse)
+            p.lse[orow] = den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
+        }
+        if (ctid == 0) p.counters[ti.b * Hkv + ti.g] = 0;  // leave the workspace clean
+      }
+    }
+    if (!csync.sync(p.flags)) return;  // the reduction buffers may be reused
+  }
+}
+
+// ------------------------------------------------------------- host side
+template <int D, bool kFp8, int kStages>
+size_t decode_smem_bytes() {
+  using Ly = Layout<D, kFp8>;
+  size_t s = 1024;  // alignment slack
+  s += (size_t)kStages * Ly::kStageB + (size_t)kStages * Ly::kQB;
+  if (kFp8) s += (size_t)kConsumerWarps * Ly::kConvB;
+  s += sizeof(float) * (kConsumerWarps * kMaxGroup * D + 2 * kConsumerWarps * kMaxGroup);
+  s += sizeof(TileInfo) * kStages;
+  s += sizeof(uint64_t) * (2 * kStages + 1) + 2 * sizeof(int32_t);
+  return s;
+}
+
+template <int D, bool kFp8, int kStages>
+cudaError_t decode_prepare(int* ctas_per_sm) {
+  auto k = decode_kernel<D, kFp8, kStages>;
+  const size_t smem = decode_smem_bytes<D, kFp8, kStages>();
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, k, kThreads, smem);
+}
+
+template <int D, bool kFp8, int kStages>
+cudaError_t decode_launch(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
+                          int num_ctas, cudaStream_t stream) {
+  const size_t smem = decode_smem_bytes<D, kFp8, kStages>();
+  decode_kernel<D, kFp8, kStages><<<num_ctas, kThreads, smem, stream>>>(tk, tv, p);
+  return cudaGetLastError();
+}
+
+// Pipeline depth per variant: enough bytes in flight per SM to cover HBM
+// latency at two resident CTAs per SM.
+constexpr int kStagesBf16D128 = 3;
+constexpr int kStagesBf16D64 = 4;
+constexpr int kStagesFp8D128 = 4;
+constexpr int kStagesFp8D64 = 4;
+
+cudaError_t decode_occupancy(int head_dim, bool fp8, int* ctas_per_sm) {
+  if (!fp8 && head_dim == 128) return decode_prepare<128, false, kStagesBf16D128>(ctas_per_sm);
+  if (!fp8 && head_dim == 64) return decode_prepare<64, false, kStagesBf16D64>(ctas_per_sm);
+  if (fp8 && head_dim == 128) return decode_prepare<128, true, kStagesFp8D128>(ctas_per_sm);
+  return decode_prepare<64, true, kStagesFp8D64>(ctas_per_sm);
+}
+
+cudaError_t decode_run(int head_dim, bool fp8, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const DecodeParams& p, int num_ctas, cudaStream_t stream) {
+  if (!fp8 && head_dim == 128)
+    return decode_launch<128, false, kStagesBf16D128>(tk, tv, p, num_ctas, stream);
+  if (!fp8 && head_dim == 64)
+    return decode_launch<64, false, kStagesBf16D64>(tk, tv, p, num_ctas, stream);
+  if (fp8 && head_dim == 128)
+    return decode_launch<128, true, kStagesFp8D128>(tk, tv, p, num_ctas, stream);
+  return decode_launch<64, true, kStagesFp8D64>(tk, tv, p, num_ctas, stream);
+}
+
+}  // namespace pkv

@@ -1,0 +1,70 @@
+// Internal interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/paged_kv.h"
+
+namespace pkv {
+
+struct AppendParams {
+  uint8_t* k_pool;
+  uint8_t* v_pool;
+  const float* k_scale;
+  const float* v_scale;
+  const int32_t* page_table;
+  const int32_t* seq_lens_before;
+  const int32_t* cu_new;
+  const uint4* k_new;  // [T][Hkv][D] bf16, as 16-byte vectors
+  const uint4* v_new;
+  int32_t* flags;
+  int32_t batch;
+  int32_t total_new;
+  int32_t max_pages;
+  int32_t num_pages;
+  int32_t page_size;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+};
+
+struct DecodeParams {
+  const __nv_bfloat16* q;  // [B][Hq][D]
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  const float* k_scale;  // [pages][Hkv] (E4M3)
+  const float* v_scale;
+  __nv_bfloat16* out;  // [B][Hq][D]
+  float* lse;          // [B][Hq] or null
+  float* part_o;       // [U + C][G][D]
+  float2* part_ml;     // [U + C][G]
+  int32_t* counters;   // [U]
+  int32_t* flags;
+  int32_t batch;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t group;
+  int32_t max_pages;
+  int32_t num_pages;
+  int32_t page_size;
+  float scale_log2;  // softmax_scale * log2(e)
+};
+
+cudaError_t launch_append(const AppendParams& p, bool fp8, int num_sms, cudaStream_t stream);
+cudaError_t decode_occupancy(int head_dim, bool fp8, int* ctas_per_sm);
+cudaError_t decode_run(int head_dim, bool fp8, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const DecodeParams& p, int num_ctas, cudaStream_t stream);
+
+int check_cache(const pkv_cache* c);
+int check_group(const pkv_cache* c, int32_t num_q_heads, int32_t gqa_group);
+int encode_pool_map(CUtensorMap* map, void* base, bool fp8, int64_t rows, int row_elems,
+                    int box_cols, int box_rows);
+int prefill_entry(const pkv_cache* cache, const void* q, int32_t num_q_heads, int32_t gqa_group,
+                  const int32_t* cu_q_lens, const int32_t* page_table, int32_t max_pages_per_seq,
+                  const int32_t* seq_lens, int32_t num_chunks, int32_t total_q,
+                  int32_t max_q_len, float softmax_scale, void* out, float* lse,
+                  cudaStream_t stream);
+
+}  // namespace pkv

@@ -53,7 +53,7 @@ _STREAM_QCHUNK = 3
 
 def _torch_gen(seed: int, stream: int, index: int) -> torch.Generator:
     g = torch.Generator(device="cpu")
-    g.manual_seed((seed * 1_000_003 + stream * 65_537 + index) % (2**63 - 1))
+    g.manual_seed(int((int(seed) * 1_000_003 + int(stream) * 65_537 + int(index)) % (2**63 - 1)))
     return g
 
 
