@@ -87,13 +87,14 @@ int encode_pool_map(CUtensorMap* map, void* base, bool fp8, int64_t rows, int ro
   return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_CUDA;
 }
 
-static int decode_ctas_per_sm(int head_dim, bool fp8, int* out) {
+static int decode_ctas_per_sm(int head_dim, bool fp8, int group, int* out) {
   // cached per variant: the occupancy of a kernel does not change at run time
-  static int cache[2][2] = {{0, 0}, {0, 0}};
-  int& slot = cache[head_dim == 128][fp8];
+  static int cache[2][2][4] = {};
+  const int gi = group == 1 ? 0 : group == 2 ? 1 : group == 4 ? 2 : 3;
+  int& slot = cache[head_dim == 128][fp8][gi];
   if (slot == 0) {
     int n = 0;
-    if (decode_occupancy(head_dim, fp8, &n) != cudaSuccess || n < 1) return PKV_ERR_CUDA;
+    if (decode_occupancy(head_dim, fp8, group, &n) != cudaSuccess || n < 1) return PKV_ERR_CUDA;
     slot = n;
   }
   *out = slot;
@@ -224,7 +225,7 @@ int paged_decode_attention(const pkv_cache* cache, const void* q, int32_t num_q_
   const bool fp8 = cache->kv_dtype == PKV_KV_FP8_E4M3;
   int sms = 0, per_sm = 0;
   if ((st = device_sms(&sms))) return st;
-  if ((st = decode_ctas_per_sm(cache->head_dim, fp8, &per_sm))) return st;
+  if ((st = decode_ctas_per_sm(cache->head_dim, fp8, gqa_group, &per_sm))) return st;
   if (per_sm > kMaxDecodeCtasPerSm) per_sm = kMaxDecodeCtasPerSm;
   int32_t ctas = 0;
   if ((st = paged_decode_plan(batch, cache->num_kv_heads, max_seq_len, sms, num_ctas, per_sm,

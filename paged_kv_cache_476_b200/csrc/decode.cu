@@ -61,10 +61,43 @@ struct Layout {
   static constexpr int kBoxB = kTile * kBoxRowB;
   static constexpr int kTileB = kNumBox * kBoxB;  // one K (or V) tile
   static constexpr int kStageB = 2 * kTileB;
-  static constexpr int kQB = kMaxGroup * D * 2;    // Q slice per stage
-  static constexpr int kConvB = 16 * D * 2;        // per-warp f16 V tile (E4M3 only)
-  static constexpr bool kSw64 = kBoxRowB == 64;
+  static constexpr int kConvB = 16 * D * 2;  // per-warp f16 V tile (E4M3 only)
 };
+
+// Shared-memory carve-up; the Q slices and the reduction buffers are sized
+// by the GQA group so that two CTAs fit on one SM.
+struct SmemPlan {
+  uint32_t q, conv, red_o, red_m, red_l, bars, info, misc, total;
+};
+
+__host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+
+template <int D, bool kFp8, int kStages>
+__host__ __device__ inline SmemPlan smem_plan(int G) {
+  using Ly = Layout<D, kFp8>;
+  SmemPlan s;
+  uint32_t o = kStages * Ly::kStageB;
+  s.q = o;
+  o += kStages * align_up(G * D * 2, 128);
+  o = align_up(o, 1024);
+  s.conv = o;
+  if (kFp8) o += kConsumerWarps * Ly::kConvB;
+  s.red_o = o;
+  o += kConsumerWarps * G * D * 4;
+  s.red_m = o;
+  o += kConsumerWarps * G * 4;
+  s.red_l = o;
+  o += kConsumerWarps * G * 4;
+  o = align_up(o, 8);
+  s.bars = o;
+  o += (2 * kStages + 1) * 8;
+  s.info = o;
+  o += kStages * sizeof(TileInfo);
+  s.misc = o;
+  o += 2 * sizeof(int32_t);
+  s.total = o;
+  return s;
+}
 
 // Byte address of 16-byte chunk `chunk` of row `row` in a TMA-swizzled tile
 // made of kNumBox boxes of [rows][kBoxRowB].
@@ -110,7 +143,7 @@ struct ConsumerSync {
 };
 
 template <int D, bool kFp8, int kStages>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
   using Ly = Layout<D, kFp8>;
@@ -118,21 +151,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   // 1024-byte align the dynamic window (the swizzle pattern needs it).
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
+  const int G = p.group;
+  const SmemPlan sp = smem_plan<D, kFp8, kStages>(G);
+  const uint32_t kQStride = align_up(G * D * 2, 128);
   uint8_t* tiles = smem;
-  uint8_t* qbuf = tiles + kStages * Ly::kStageB;
-  uint8_t* conv = qbuf + kStages * Ly::kQB;
-  float* red_o = reinterpret_cast<float*>(conv + (kFp8 ? kConsumerWarps * Ly::kConvB : 0));
-  float* red_m = red_o + kConsumerWarps * kMaxGroup * D;
-  float* red_l = red_m + kConsumerWarps * kMaxGroup;
-  uint64_t* full = reinterpret_cast<uint64_t*>(red_l + kConsumerWarps * kMaxGroup);
+  uint8_t* qbuf = smem + sp.q;
+  uint8_t* conv = smem + sp.conv;
+  float* red_o = reinterpret_cast<float*>(smem + sp.red_o);
+  float* red_m = reinterpret_cast<float*>(smem + sp.red_m);
+  float* red_l = reinterpret_cast<float*>(smem + sp.red_l);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + sp.bars);
   uint64_t* empty = full + kStages;
   uint64_t* merge_bar = empty + kStages;
-  TileInfo* info = reinterpret_cast<TileInfo*>(merge_bar + 1);
-  int32_t* s_misc = reinterpret_cast<int32_t*>(info + kStages);  // [0]=n tiles, [1]=is_last
+  TileInfo* info = reinterpret_cast<TileInfo*>(smem + sp.info);
+  int32_t* s_misc = reinterpret_cast<int32_t*>(smem + sp.misc);  // [0]=n tiles, [1]=is_last
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int G = p.group;
   const int Hkv = p.num_kv_heads;
   const int64_t C = gridDim.x;
   const int64_t c = blockIdx.x;
@@ -229,6 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int my_pid = 0;
     float my_ks = 1.f, my_vs = 1.f;
     int64_t x = range_start;  // global tile index
+    int u_seg_base = 0, u_nseg = 1, u_slot = 0;
     int issued = 0;
     bool ok = true;
     for (int64_t i = 0; i < n_tiles; ++i, ++x) {
@@ -283,13 +319,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         ti.valid = min(kTile, len - t * kTile);
         ti.flags = (first ? kSegFirst : 0) | (last ? kSegLast : 0) | (bad ? kBadTile : 0);
         if (last && seg_first_t == 0 && t == ntile - 1) ti.flags |= kUnitWhole;
-        const int64_t u = (int64_t)b * Hkv + g;
-        const int64_t x_unit = x - t;  // global index of the unit's first tile
-        const int64_t c_first = cta_of(x_unit, Ce, T);
-        const int64_t c_last = cta_of(x_unit + ntile - 1, Ce, T);
-        ti.seg_base = (int)(u + c_first);
-        ti.nseg = (int)(c_last - c_first + 1);
-        ti.slot = (int)(u + c);
+        if (first) {
+          // once per unit: which CTAs share it, hence its partial slots
+          const int64_t u = (int64_t)b * Hkv + g;
+          const int64_t x_unit = x - t;  // global index of the unit's first tile
+          const int64_t c_first = cta_of(x_unit, Ce, T);
+          const int64_t c_last = cta_of(x_unit + ntile - 1, Ce, T);
+          u_seg_base = (int)(u + c_first);
+          u_nseg = (int)(c_last - c_first + 1);
+          u_slot = (int)(u + c);
+        }
+        ti.seg_base = u_seg_base;
+        ti.nseg = u_nseg;
+        ti.slot = u_slot;
         ti.ks = ks;
         ti.vs = vs;
         info[stage] = ti;
@@ -308,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const __nv_bfloat16* src = p.q + ((int64_t)b * p.num_q_heads + (int64_t)g * G) * D;
           asm volatile(
               "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, "
-              "[%3];" ::"r"(smem_u32(qbuf + stage * Ly::kQB)),
+              "[%3];" ::"r"(smem_u32(qbuf + stage * kQStride)),
               "l"(reinterpret_cast<uint64_t>(src)), "r"(qbytes), "r"(smem_u32(&full[stage]))
               : "memory");
         }
@@ -357,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int stage = (int)(i % kStages);
     if (!mbar_wait(&full[stage], (uint32_t)((i / kStages) & 1), p.flags)) return;
     const TileInfo ti = info[stage];
-    const uint8_t* qs = qbuf + stage * Ly::kQB;
+    const uint8_t* qs = qbuf + stage * kQStride;
     if (ti.flags & kSegFirst) {
       m_run = -INFINITY;
       l_part = 0.f;
@@ -412,15 +454,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- S = Q K^T over my 16 tokens (two n-tiles of 8) ----
       float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
       if constexpr (!kFp8) {
+        // two independent accumulation chains per n-tile (even / odd k-steps)
+        float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
         for (int kk = 0; kk < KS; ++kk) {
           const int row = 16 * warp + mrow + (mat >> 1) * 8;
           const int chunk = 2 * kk + (mat & 1);
           uint32_t b0, b1, b2, b3;
           ldsm_x4(tile_addr<Ly::kBoxRowB, kTile>(kbase, row, chunk), b0, b1, b2, b3);
-          mma_bf16(s[0], qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
-          mma_bf16(s[1], qa[kk][0], 0u, qa[kk][1], 0u, b2, b3);
+          float(*acc)[4] = (kk & 1) ? s2 : s;
+          mma_bf16(acc[0], qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
+          mma_bf16(acc[1], qa[kk][0], 0u, qa[kk][1], 0u, b2, b3);
         }
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s[n][e] += s2[n][e];
       } else {
 #pragma unroll
         for (int kp = 0; kp < KS / 2; ++kp) {
@@ -558,10 +607,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     l_row += __shfl_xor_sync(0xffffffffu, l_row, 2);
     if (row_ok) {
       if (tid4 == 0) {
-        red_m[warp * kMaxGroup + gid] = m_run;
-        red_l[warp * kMaxGroup + gid] = l_row;
+        red_m[warp * G + gid] = m_run;
+        red_l[warp * G + gid] = l_row;
       }
-      float* ro = red_o + (warp * kMaxGroup + gid) * D;
+      float* ro = red_o + (warp * G + gid) * D;
 #pragma unroll
       for (int n = 0; n < D / 8; ++n)
         *reinterpret_cast<float2*>(ro + 8 * n + 2 * tid4) = make_float2(o[n][0], o[n][1]);
@@ -574,16 +623,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int d = e - row * D;
       float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red_m[w * kMaxGroup + row]);
+      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red_m[w * G + row]);
       float num = 0.f, den = 0.f;
       if (M != -INFINITY) {
 #pragma unroll
         for (int w = 0; w < kConsumerWarps; ++w) {
-          const float mw = red_m[w * kMaxGroup + row];
+          const float mw = red_m[w * G + row];
           if (mw == -INFINITY) continue;
           const float sc = exp2f(mw - M);
-          num += sc * red_o[(w * kMaxGroup + row) * D + d];
-          den += sc * red_l[w * kMaxGroup + row];
+          num += sc * red_o[(w * G + row) * D + d];
+          den += sc * red_l[w * G + row];
         }
       }
       const int h = ti.g * G + row;
@@ -638,22 +687,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------- host side
 template <int D, bool kFp8, int kStages>
-size_t decode_smem_bytes() {
-  using Ly = Layout<D, kFp8>;
-  size_t s = 1024;  // alignment slack
-  s += (size_t)kStages * Ly::kStageB + (size_t)kStages * Ly::kQB;
-  if (kFp8) s += (size_t)kConsumerWarps * Ly::kConvB;
-  s += sizeof(float) * (kConsumerWarps * kMaxGroup * D + 2 * kConsumerWarps * kMaxGroup);
-  s += sizeof(TileInfo) * kStages;
-  s += sizeof(uint64_t) * (2 * kStages + 1) + 2 * sizeof(int32_t);
-  return s;
+size_t decode_smem_bytes(int G) {
+  return 1024 + smem_plan<D, kFp8, kStages>(G).total;  // + alignment slack
 }
 
 template <int D, bool kFp8, int kStages>
-cudaError_t decode_prepare(int* ctas_per_sm) {
+cudaError_t decode_prepare(int G, int* ctas_per_sm) {
   auto k = decode_kernel<D, kFp8, kStages>;
-  const size_t smem = decode_smem_bytes<D, kFp8, kStages>();
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const size_t smem = decode_smem_bytes<D, kFp8, kStages>(G);
+  // The attribute belongs to the instantiation, which serves every group
+  // size: allow the largest footprint once, not the one of this call.
+  const size_t most = decode_smem_bytes<D, kFp8, kStages>(kMaxGroup);
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most);
   if (e != cudaSuccess) return e;
   return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, k, kThreads, smem);
 }
@@ -661,34 +706,54 @@ cudaError_t decode_prepare(int* ctas_per_sm) {
 template <int D, bool kFp8, int kStages>
 cudaError_t decode_launch(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                           int num_ctas, cudaStream_t stream) {
-  const size_t smem = decode_smem_bytes<D, kFp8, kStages>();
+  const size_t smem = decode_smem_bytes<D, kFp8, kStages>(p.group);
   decode_kernel<D, kFp8, kStages><<<num_ctas, kThreads, smem, stream>>>(tk, tv, p);
   return cudaGetLastError();
 }
 
-// Pipeline depth per variant: enough bytes in flight per SM to cover HBM
-// latency at two resident CTAs per SM.
-constexpr int kStagesBf16D128 = 3;
-constexpr int kStagesBf16D64 = 4;
-constexpr int kStagesFp8D128 = 4;
-constexpr int kStagesFp8D64 = 4;
+// Deepest ring that still lets two CTAs share an SM (228 KB of shared
+// memory per SM, 1 KB of it reserved per CTA).
+constexpr size_t kSmemPerCtaFor2 = 113 * 1024;
 
-cudaError_t decode_occupancy(int head_dim, bool fp8, int* ctas_per_sm) {
-  if (!fp8 && head_dim == 128) return decode_prepare<128, false, kStagesBf16D128>(ctas_per_sm);
-  if (!fp8 && head_dim == 64) return decode_prepare<64, false, kStagesBf16D64>(ctas_per_sm);
-  if (fp8 && head_dim == 128) return decode_prepare<128, true, kStagesFp8D128>(ctas_per_sm);
-  return decode_prepare<64, true, kStagesFp8D64>(ctas_per_sm);
+template <int D, bool kFp8>
+int pick_stages(int G) {
+  if (decode_smem_bytes<D, kFp8, 4>(G) <= kSmemPerCtaFor2) return 4;
+  if (decode_smem_bytes<D, kFp8, 3>(G) <= kSmemPerCtaFor2) return 3;
+  return 2;
+}
+
+template <int D, bool kFp8>
+cudaError_t occupancy_for(int G, int* n) {
+  switch (pick_stages<D, kFp8>(G)) {
+    case 4: return decode_prepare<D, kFp8, 4>(G, n);
+    case 3: return decode_prepare<D, kFp8, 3>(G, n);
+    default: return decode_prepare<D, kFp8, 2>(G, n);
+  }
+}
+
+template <int D, bool kFp8>
+cudaError_t run_for(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
+                    int num_ctas, cudaStream_t stream) {
+  switch (pick_stages<D, kFp8>(p.group)) {
+    case 4: return decode_launch<D, kFp8, 4>(tk, tv, p, num_ctas, stream);
+    case 3: return decode_launch<D, kFp8, 3>(tk, tv, p, num_ctas, stream);
+    default: return decode_launch<D, kFp8, 2>(tk, tv, p, num_ctas, stream);
+  }
+}
+
+cudaError_t decode_occupancy(int head_dim, bool fp8, int group, int* ctas_per_sm) {
+  if (!fp8 && head_dim == 128) return occupancy_for<128, false>(group, ctas_per_sm);
+  if (!fp8 && head_dim == 64) return occupancy_for<64, false>(group, ctas_per_sm);
+  if (fp8 && head_dim == 128) return occupancy_for<128, true>(group, ctas_per_sm);
+  return occupancy_for<64, true>(group, ctas_per_sm);
 }
 
 cudaError_t decode_run(int head_dim, bool fp8, const CUtensorMap& tk, const CUtensorMap& tv,
                        const DecodeParams& p, int num_ctas, cudaStream_t stream) {
-  if (!fp8 && head_dim == 128)
-    return decode_launch<128, false, kStagesBf16D128>(tk, tv, p, num_ctas, stream);
-  if (!fp8 && head_dim == 64)
-    return decode_launch<64, false, kStagesBf16D64>(tk, tv, p, num_ctas, stream);
-  if (fp8 && head_dim == 128)
-    return decode_launch<128, true, kStagesFp8D128>(tk, tv, p, num_ctas, stream);
-  return decode_launch<64, true, kStagesFp8D64>(tk, tv, p, num_ctas, stream);
+  if (!fp8 && head_dim == 128) return run_for<128, false>(tk, tv, p, num_ctas, stream);
+  if (!fp8 && head_dim == 64) return run_for<64, false>(tk, tv, p, num_ctas, stream);
+  if (fp8 && head_dim == 128) return run_for<128, true>(tk, tv, p, num_ctas, stream);
+  return run_for<64, true>(tk, tv, p, num_ctas, stream);
 }
 
 }  // namespace pkv

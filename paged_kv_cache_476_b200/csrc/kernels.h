@@ -53,7 +53,7 @@ struct DecodeParams {
 };
 
 cudaError_t launch_append(const AppendParams& p, bool fp8, int num_sms, cudaStream_t stream);
-cudaError_t decode_occupancy(int head_dim, bool fp8, int* ctas_per_sm);
+cudaError_t decode_occupancy(int head_dim, bool fp8, int group, int* ctas_per_sm);
 cudaError_t decode_run(int head_dim, bool fp8, const CUtensorMap& tk, const CUtensorMap& tv,
                        const DecodeParams& p, int num_ctas, cudaStream_t stream);
 
