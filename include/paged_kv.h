@@ -65,7 +65,8 @@ typedef enum {
   PKV_ERR_WORKSPACE = -7,   /* decode workspace NULL, misaligned or too small */
   PKV_ERR_CUDA = -8,        /* a CUDA runtime call or kernel launch failed */
   PKV_ERR_ALIGN = -9,       /* a pointer that must be 16-byte aligned is not */
-  PKV_ERR_UNSUPPORTED = -10 /* a valid combination this build does not implement */
+  PKV_ERR_UNSUPPORTED = -10, /* a valid combination this build does not implement */
+  PKV_ERR_SCRATCH_LIMIT = -11 /* request needs more than the static decode scratch */
 } pkv_status;
 
 typedef enum { PKV_KV_BF16 = 0, PKV_KV_FP8_E4M3 = 1 } pkv_kv_dtype;
@@ -193,6 +194,35 @@ int paged_prefill_chunk_attention(const pkv_cache* cache, const void* q, int32_t
                                   const int32_t* seq_lens, int32_t num_chunks, int32_t total_q,
                                   int32_t max_q_len, float softmax_scale, void* out, float* lse,
                                   void* stream);
+
+/*
+ * Decode attention without any device allocation.  The paper has no
+ * counterpart: this entry point exists for callers that cannot call
+ * cudaMalloc or take memory from an allocator (code handed only input and
+ * output pointers by a host framework or plugin interface, code running where
+ * allocation is forbidden, or code that must not change the device's
+ * allocation state).  It computes exactly what paged_decode_attention
+ * computes, with the same arguments minus the workspace: the split partials
+ * and counters live in a scratch array inside the library, a file-scope
+ * __device__ array of PKV_NOALLOC_SCRATCH_BYTES (16 MiB) that every GPU which
+ * loads the library holds until the process exits.
+ *  - Sizes whose workspace (paged_decode_workspace_bytes) exceeds the array
+ *    are rejected with PKV_ERR_SCRATCH_LIMIT before anything is enqueued.
+ *  - Each call clears the part of the array it uses with an asynchronous
+ *    memset on `stream`, then launches; it allocates nothing and calls no
+ *    allocating library routine.
+ *  - All calls on a device share the array and it keeps the last call's
+ *    contents: calls whose executions overlap on the GPU (unordered streams)
+ *    race and give wrong results.  Order them on one stream.
+ *  - The first call on a device looks up the array's device address with that
+ *    device current; make that first call before any stream capture.
+ */
+#define PKV_NOALLOC_SCRATCH_BYTES (16u << 20)
+int paged_decode_attention_noalloc(const pkv_cache* cache, const void* q, int32_t num_q_heads,
+                                   int32_t gqa_group, const int32_t* page_table,
+                                   int32_t max_pages_per_seq, const int32_t* seq_lens,
+                                   int32_t batch, int32_t max_seq_len, float softmax_scale,
+                                   void* out, float* lse, int32_t num_ctas, void* stream);
 
 /* Human-readable name of a pkv_status value (static storage). */
 const char* pkv_status_string(int status);

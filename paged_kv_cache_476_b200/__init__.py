@@ -40,7 +40,11 @@ EXPORTED = (
     "paged_prefill_chunk_attention",
     "pkv_status_string",
     "pkv_abi_version",
+    "paged_decode_attention_noalloc",
 )
+
+# Size of the library's static decode scratch (see paged_decode_attention_noalloc).
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class PkvCache(ctypes.Structure):
@@ -63,9 +67,13 @@ class PkvCache(ctypes.Structure):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_476_b200.build` "
+            f"{LIB_PATH} is missing: build it with `python paged_kv_cache_476_b200/build.py` "
             "(there is no fallback path)")
     lib = ctypes.CDLL(LIB_PATH)
+    missing = [n for n in EXPORTED if not hasattr(lib, n)]
+    if missing:
+        raise ImportError(f"{LIB_PATH} is stale (missing {missing}): rebuild it with "
+                          "`python paged_kv_cache_476_b200/build.py`")
     P, I32, SZ, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_float
     cp = ctypes.POINTER(PkvCache)
     lib.paged_kv_append.argtypes = [cp, P, I32, P, P, I32, I32, P, P, P]
@@ -80,6 +88,9 @@ def _load() -> ctypes.CDLL:
     lib.paged_prefill_chunk_attention.argtypes = [cp, P, I32, I32, P, P, I32, P, I32, I32, I32,
                                                   F, P, P, P]
     lib.paged_prefill_chunk_attention.restype = ctypes.c_int
+    lib.paged_decode_attention_noalloc.argtypes = [cp, P, I32, I32, P, I32, P, I32, I32, F, P, P,
+                                                   I32, P]
+    lib.paged_decode_attention_noalloc.restype = ctypes.c_int
     lib.pkv_status_string.argtypes = [ctypes.c_int]
     lib.pkv_status_string.restype = ctypes.c_char_p
     lib.pkv_abi_version.restype = ctypes.c_int
@@ -260,4 +271,35 @@ def paged_prefill_chunk_attention(cache: PagedKVCache, q, cu_q_lens, page_table,
         _ptr(page_table), page_table.shape[1], _ptr(seq_lens), seq_lens.shape[0], T,
         int(max_q_len), float(softmax_scale), _ptr(out), _ptr(lse), _stream(stream))
     _check("paged_prefill_chunk_attention", st)
+    return out, lse
+
+
+def paged_decode_attention_noalloc(cache: PagedKVCache, q, page_table, seq_lens,
+                                   max_seq_len: int, softmax_scale: Optional[float] = None,
+                                   out=None, lse=None, num_ctas: int = 0, want_lse: bool = True,
+                                   stream=None):
+    """Decode attention that allocates no device memory inside the library.
+
+    For callers that cannot provide a workspace: the split partials live in a
+    16 MiB scratch array inside ``libpagedkv.so`` that each GPU holds until
+    the process exits.  Calls share that array, so calls that overlap on the
+    GPU race; keep them on one stream.  ``out``/``lse`` are still the
+    caller's (allocated here only if not given).  Same results as
+    ``paged_decode_attention``.
+    """
+    _dev("q", q, torch.bfloat16, 3)
+    _dev("page_table", page_table, torch.int32, 2)
+    _dev("seq_lens", seq_lens, torch.int32, 1)
+    B, Hq, D = q.shape
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    st = _lib.paged_decode_attention_noalloc(
+        ctypes.byref(cache.c_struct), _ptr(q), Hq, Hq // cache.num_kv_heads, _ptr(page_table),
+        page_table.shape[1], _ptr(seq_lens), B, int(max_seq_len), float(softmax_scale),
+        _ptr(out), _ptr(lse), int(num_ctas), _stream(stream))
+    _check("paged_decode_attention_noalloc", st)
     return out, lse

@@ -1,6 +1,7 @@
 """Build libpagedkv.so in-tree with nvcc for sm_100a.
 
-Usage: ``python -m paged_kv_cache_476_b200.build [--force]``.  Each ``.cu``
+Usage: ``python paged_kv_cache_476_b200/build.py [--force]`` (run it as a
+file: importing the package first would load a possibly stale library).  Each ``.cu``
 under ``csrc/`` compiles to an object in ``_build/`` (in parallel), then the
 objects link into ``paged_kv_cache_476_b200/libpagedkv.so`` with the CUDA
 runtime linked statically.  nvcc cross-compiles, so no GPU is needed.

@@ -125,6 +125,8 @@ const char* pkv_status_string(int status) {
     case PKV_ERR_CUDA: return "a CUDA call or kernel launch failed";
     case PKV_ERR_ALIGN: return "a pointer that must be 16-byte aligned is not";
     case PKV_ERR_UNSUPPORTED: return "this combination is not implemented";
+    case PKV_ERR_SCRATCH_LIMIT:
+      return "the request needs more decode scratch than the library's static 16 MiB array";
     default: return "unknown status";
   }
 }
