@@ -17,8 +17,7 @@
  *
  * Conventions shared by every entry point:
  *  - All array pointers are DEVICE memory owned by the caller; the library
- *    allocates nothing and keeps no state between calls (except the counters
- *    inside a caller-owned decode workspace, see below).
+ *    allocates nothing and keeps no state between calls.
  *  - Pools: separate K and V pools, each [num_pages][num_kv_heads][page_size]
  *    [head_dim], row-major, element type bf16 or FP8 E4M3 (1 byte).  Base
  *    addresses must be 16-byte aligned.
@@ -133,9 +132,9 @@ int paged_decode_plan(int32_t batch, int32_t num_kv_heads, int32_t max_seq_len,
  * device (call it with the device that will run the decode current).
  * Returns 0 on bad arguments.  The workspace holds the split partials
  * ((units + C) slots of G x (head_dim + 2) floats, units = batch *
- * num_kv_heads) and one counter per unit.  It must be ZERO-FILLED before its first use; every completed call
- * leaves the counters at zero again.  Calls that share a workspace must not
- * overlap on the GPU.
+ * num_kv_heads) and one (first slot, segment count) record per unit.  It
+ * needs no initialisation: every call writes each value it later reads.
+ * Calls that share a workspace must not overlap on the GPU.
  */
 size_t paged_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
                                     int32_t head_dim, int32_t max_seq_len, int32_t num_ctas);
@@ -147,8 +146,9 @@ size_t paged_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t 
  *   out[b][h] = sum_t exp(s_t - m) V_b[t] / sum_t exp(s_t - m)   (bf16)
  *   lse[b][h] = m + ln(sum_t exp(s_t - m))                       (fp32)
  * computed as online-softmax partials over page ranges (see
- * paged_decode_plan), merged in the same launch by the last CTA that
- * finishes a piece of each (sequence, kv head).  A sequence of length 0
+ * paged_decode_plan); the pieces of a (sequence, kv head) cut across CTAs
+ * are merged by a second kernel enqueued by the same call (a programmatic
+ * dependent launch, so its launch overlaps the first).  A sequence of length 0
  * yields out = 0 and lse = -inf.  Source: concept page "執行時執行模型"
  * (attention reads the KV pages each step) and "PagedAttention 及 KV 快取管理".
  *   q             bf16 [batch][num_q_heads][head_dim]
@@ -203,14 +203,14 @@ int paged_prefill_chunk_attention(const pkv_cache* cache, const void* q, int32_t
  * allocation is forbidden, or code that must not change the device's
  * allocation state).  It computes exactly what paged_decode_attention
  * computes, with the same arguments minus the workspace: the split partials
- * and counters live in a scratch array inside the library, a file-scope
+ * and per-unit records live in a scratch array inside the library, a file-scope
  * __device__ array of PKV_NOALLOC_SCRATCH_BYTES (16 MiB) that every GPU which
  * loads the library holds until the process exits.
  *  - Sizes whose workspace (paged_decode_workspace_bytes) exceeds the array
  *    are rejected with PKV_ERR_SCRATCH_LIMIT before anything is enqueued.
- *  - Each call clears the part of the array it uses with an asynchronous
- *    memset on `stream`, then launches; it allocates nothing and calls no
- *    allocating library routine.
+ *  - Nothing in the array needs to start at zero: each call writes every
+ *    value it later reads.  A call allocates nothing and calls no allocating
+ *    library routine.
  *  - All calls on a device share the array and it keeps the last call's
  *    contents: calls whose executions overlap on the GPU (unordered streams)
  *    race and give wrong results.  Order them on one stream.

@@ -200,7 +200,7 @@ size_t paged_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t 
   bytes = (bytes + 15) & ~size_t(15);
   bytes += slots * G * 2 * sizeof(float);  // partial (m, l)
   bytes = (bytes + 15) & ~size_t(15);
-  bytes += units * sizeof(int32_t);  // counters
+  bytes += units * sizeof(int2);  // per-unit (first slot, segments)
   return (bytes + 255) & ~size_t(255);
 }
 
@@ -254,7 +254,7 @@ int paged_decode_attention(const pkv_cache* cache, const void* q, int32_t num_q_
   float2* part_ml = reinterpret_cast<float2*>(ws + off);
   off += slots * G * 2 * sizeof(float);
   off = (off + 15) & ~size_t(15);
-  int32_t* counters = reinterpret_cast<int32_t*>(ws + off);
+  int2* unit_info = reinterpret_cast<int2*>(ws + off);
 
   DecodeParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -266,7 +266,7 @@ int paged_decode_attention(const pkv_cache* cache, const void* q, int32_t num_q_
   p.lse = lse;
   p.part_o = part_o;
   p.part_ml = part_ml;
-  p.counters = counters;
+  p.unit_info = unit_info;
   p.flags = cache->error_flags;
   p.batch = batch;
   p.num_q_heads = num_q_heads;

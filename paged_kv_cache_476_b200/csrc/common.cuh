@@ -21,10 +21,9 @@
 
 namespace pkv {
 
-// Tries of an mbarrier wait before it is declared stuck.  A try can suspend
-// the thread for a hardware-chosen interval, so this bounds the wait at
-// roughly a second or two, far beyond any legitimate latency.
-constexpr uint32_t kWaitTries = 1u << 22;
+// A bounded wait gives up after this many nanoseconds (%globaltimer), far
+// beyond any legitimate latency, and reports PKV_FLAG_TIMEOUT.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 __device__ __forceinline__ void flag_error(int32_t* flags, int bit) {
   if (flags) atomicOr(flags, bit);
@@ -67,11 +66,39 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity to complete.  Returns
-// false (and raises PKV_FLAG_TIMEOUT) if it never does.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* flags) {
-  for (uint32_t i = 0; i < kWaitTries; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity,
+                                                    uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait for the phase with the given parity to complete.  With
+// suspend_ns > 0 a waiting thread may sleep up to that long per try (it is
+// woken when the phase completes), so an idle warp costs no issue slots.
+// Returns false (and raises PKV_FLAG_TIMEOUT) after kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* flags,
+                                          uint32_t suspend_ns = 0) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    const bool ok =
+        suspend_ns ? mbar_try_wait_sleep(bar, parity, suspend_ns) : mbar_try_wait(bar, parity);
+    if (ok) return true;
+    if (global_ns() - t0 > kWaitLimitNs) break;
+  }
   flag_error(flags, PKV_FLAG_TIMEOUT);
   return false;
 }

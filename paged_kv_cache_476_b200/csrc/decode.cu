@@ -13,14 +13,16 @@
 //  * A range cuts a unit into segments.  A segment computes an online-softmax
 //    partial (m, l, unnormalised o) for the unit's G = Hq/Hkv q heads.  A
 //    segment that covers its whole unit writes the output directly; otherwise
-//    it stores its partial and bumps the unit's counter, and the last segment
-//    to arrive merges all of them (the split-KV reduction, same launch).
+//    it stores its partial, and a small merge kernel (a programmatic
+//    dependent launch, one warp per unit) combines the pieces afterwards.
 //  * Warp roles: one producer warp walks the range and issues TMA loads of
 //    the K and V tile (page-table indirected, 128-byte swizzled) into a
 //    multi-stage mbarrier ring, plus a bulk copy of Q at each segment start;
 //    four consumer warps each take 16 of a tile's 64 tokens and run
-//    S = Q K^T and O += P V on mma.sync (bf16, or f16 for E4M3 K/V which
-//    converts exactly), with the online softmax in registers.
+//    S = Q K^T and O^T += V^T P^T on mma.sync (bf16, or f16 for E4M3 K/V
+//    which converts exactly), with the online softmax in registers; a flush
+//    warp turns the consumers' per-warp snapshots at each segment end into
+//    the output or a split partial while the consumers stream on.
 //  * E4M3 K/V: K codes are converted to f16 in registers after ldmatrix (the
 //    d order inside each 16-wide block is permuted identically in Q); V codes
 //    are converted into a per-warp f16 tile for the transposed ldmatrix.  The
@@ -33,8 +35,17 @@ namespace pkv {
 
 constexpr int kTile = 64;           // tokens per pipeline tile
 constexpr int kConsumerWarps = 4;   // 16 tokens of each tile per warp
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kProducerWarp = kConsumerWarps;
+constexpr int kFlushWarp = kConsumerWarps + 1;
+constexpr int kThreads = (kConsumerWarps + 2) * 32;
 constexpr int kMaxGroup = 8;
+// Suspend hints (ns) of the waits: the flush warp idles for long stretches.
+#ifndef PKV_FLUSH_SLEEP_NS
+#define PKV_FLUSH_SLEEP_NS 20000
+#endif
+#ifndef PKV_PIPE_SLEEP_NS
+#define PKV_PIPE_SLEEP_NS 0
+#endif
 
 // TileInfo.flags
 constexpr int kSegFirst = 1;   // first tile of a segment: reset state, Q in this stage
@@ -50,6 +61,11 @@ struct TileInfo {
   int32_t seg_base;  // first partial slot of the unit
   int32_t nseg;      // segments of the unit
   float ks, vs;      // E4M3 scales of the tile's page
+};
+
+// What the consumers hand to the flush warp at the end of a segment.
+struct FlushDesc {
+  int32_t b, g, slot, seg_base, nseg, whole, final;
 };
 
 template <int D, bool kFp8>
@@ -90,9 +106,9 @@ __host__ __device__ inline SmemPlan smem_plan(int G) {
   o += kConsumerWarps * G * 4;
   o = align_up(o, 8);
   s.bars = o;
-  o += (2 * kStages + 1) * 8;
+  o += (2 * kStages + 2) * 8;
   s.info = o;
-  o += kStages * sizeof(TileInfo);
+  o += kStages * sizeof(TileInfo) + sizeof(FlushDesc);
   s.misc = o;
   o += 2 * sizeof(int32_t);
   s.total = o;
@@ -128,20 +144,6 @@ __device__ __forceinline__ int32_t clamp_len(const DecodeParams& p, int32_t len,
   return len;
 }
 
-// A CTA-internal barrier among the consumer warps built on an mbarrier, so
-// that every wait is bounded (a named barrier could wait forever).
-struct ConsumerSync {
-  uint64_t* bar;
-  uint32_t phase;
-  __device__ __forceinline__ bool sync(int32_t* flags) {
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-    const bool ok = mbar_wait(bar, phase, flags);
-    phase ^= 1;
-    return ok;
-  }
-};
-
 template <int D, bool kFp8, int kStages>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
@@ -162,13 +164,18 @@ __global__ void __launch_bounds__(kThreads, 2)
   float* red_l = reinterpret_cast<float*>(smem + sp.red_l);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + sp.bars);
   uint64_t* empty = full + kStages;
-  uint64_t* merge_bar = empty + kStages;
+  uint64_t* red_full = empty + kStages;   // consumers -> flush warp: a snapshot is ready
+  uint64_t* red_empty = red_full + 1;     // flush warp -> consumers: snapshot consumed
   TileInfo* info = reinterpret_cast<TileInfo*>(smem + sp.info);
+  FlushDesc* desc = reinterpret_cast<FlushDesc*>(info + kStages);
   int32_t* s_misc = reinterpret_cast<int32_t*>(smem + sp.misc);  // [0]=n tiles, [1]=is_last
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int Hkv = p.num_kv_heads;
+  // The merge kernel that follows waits for this grid's completion itself;
+  // letting it launch now hides its launch latency behind this kernel.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t C = gridDim.x;
   const int64_t c = blockIdx.x;
 
@@ -177,7 +184,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kConsumerWarps);
     }
-    mbar_init(merge_bar, kConsumerWarps);
+    mbar_init(red_full, kConsumerWarps);
+    mbar_init(red_empty, 1);
     fence_barrier_init();
   }
 
@@ -185,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   int64_t n_tiles = 0;
   int pb = 0, pg = 0, pt = 0;  // producer's position (b, g, tile) at the range start
   int64_t range_start = 0, T = 0, Ce = 1;
-  if (warp == kConsumerWarps) {
+  if (warp == kProducerWarp) {
     // Total tiles over all units.
     int64_t tot = 0;
     for (int base = 0; base < p.batch; base += 32) {
@@ -247,7 +255,53 @@ __global__ void __launch_bounds__(kThreads, 2)
   n_tiles = s_misc[0];
   if (n_tiles == 0) return;
 
-  if (warp == kConsumerWarps) {
+  if (warp == kFlushWarp) {
+    // ---------------------------------------------------------- flush warp
+    // Turns each segment's per-warp snapshots into the output (whole unit)
+    // or a split partial, then settles the unit's counter and, as the last
+    // segment of a unit, merges its partials.  All of it overlaps the
+    // consumers, which keep streaming the next segment.
+    for (int k = 0;; ++k) {
+      if (!mbar_wait(red_full, (uint32_t)(k & 1), p.flags, PKV_FLUSH_SLEEP_NS)) return;
+      const FlushDesc fd = *desc;
+      for (int r = 0; r < G; ++r) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red_m[w * G + r]);
+        float sc[kConsumerWarps];
+        float den = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float mw = red_m[w * G + r];
+          sc[w] = (M == -INFINITY || mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
+          den += sc[w] * red_l[w * G + r];
+        }
+        const int64_t orow = (int64_t)fd.b * p.num_q_heads + fd.g * G + r;
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        for (int d = lane; d < D; d += 32) {
+          float num = 0.f;
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) num += sc[w] * red_o[(w * G + r) * D + d];
+          if (fd.whole)
+            p.out[orow * D + d] = __float2bfloat16(num * inv);
+          else
+            p.part_o[((int64_t)fd.slot * G + r) * D + d] = num;
+        }
+        if (lane == 0) {
+          if (fd.whole) {
+            if (p.lse) p.lse[orow] = den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
+          } else {
+            p.part_ml[(int64_t)fd.slot * G + r] = make_float2(M, den);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(red_empty);  // the snapshot buffers are free again
+      if (fd.final) return;
+    }
+  }
+
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------ producer loop
     const uint64_t pol = policy_evict_first();
     if (lane == 0) {
@@ -270,7 +324,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int64_t i = 0; i < n_tiles; ++i, ++x) {
       const int stage = (int)(i % kStages);
       if (i >= kStages) {
-        if (!mbar_wait(&empty[stage], (uint32_t)((i / kStages - 1) & 1), p.flags)) {
+        if (!mbar_wait(&empty[stage], (uint32_t)((i / kStages - 1) & 1), p.flags,
+                       PKV_PIPE_SLEEP_NS)) {
           ok = false;
           break;
         }
@@ -328,6 +383,9 @@ __global__ void __launch_bounds__(kThreads, 2)
           u_seg_base = (int)(u + c_first);
           u_nseg = (int)(c_last - c_first + 1);
           u_slot = (int)(u + c);
+          // the CTA holding the unit's first tile tells the merge kernel
+          // where the unit's partials are (nseg == 1: written whole)
+          if (t == 0) p.unit_info[u] = make_int2(u_seg_base, u_nseg);
         }
         ti.seg_base = u_seg_base;
         ti.nseg = u_nseg;
@@ -387,24 +445,32 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int mat = lane >> 3;   // which 8x8 matrix this lane addresses in ldmatrix.x4
   const int mrow = lane & 7;
   const bool row_ok = gid < G;
-  ConsumerSync csync{merge_bar, 0};
+  int nflush = 0;
 
   constexpr int KS = D / 16;  // k-steps over head_dim
   uint32_t qa[KS][2];         // A fragments of Q: rows gid, two k halves
-  float o[D / 8][4];
+  // O^T accumulators: PV runs as O^T = V^T P^T (M = head_dim, N = 8 heads).
+  // ot[m][0..1] = O[heads 2*tid4, 2*tid4+1][d = 16m + gid], ot[m][2..3] the same at d + 8.
+  float ot[D / 16][4];
   float m_run = -INFINITY, l_part = 0.f;
   float qk_mul = p.scale_log2;  // multiplier of the raw scores into log2 units
 
   for (int64_t i = 0; i < n_tiles; ++i) {
     const int stage = (int)(i % kStages);
-    if (!mbar_wait(&full[stage], (uint32_t)((i / kStages) & 1), p.flags)) return;
-    const TileInfo ti = info[stage];
+    if (!mbar_wait(&full[stage], (uint32_t)((i / kStages) & 1), p.flags, PKV_PIPE_SLEEP_NS))
+      return;
+    // only what the tile's math needs lives in registers; the segment
+    // bookkeeping is read from the (still unreleased) stage at hand-off
+    const int t_flags = info[stage].flags;
+    const int t_valid = info[stage].valid;
+    const float t_ks = kFp8 ? info[stage].ks : 1.f;
+    const float t_vs = kFp8 ? info[stage].vs : 1.f;
     const uint8_t* qs = qbuf + stage * kQStride;
-    if (ti.flags & kSegFirst) {
+    if (t_flags & kSegFirst) {
       m_run = -INFINITY;
       l_part = 0.f;
 #pragma unroll
-      for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+      for (int m = 0; m < D / 16; ++m) ot[m][0] = ot[m][1] = ot[m][2] = ot[m][3] = 0.f;
       if constexpr (!kFp8) {
 #pragma unroll
         for (int kk = 0; kk < KS; ++kk) {
@@ -447,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
 
-    const int valid = (ti.flags & kBadTile) ? 0 : ti.valid - 16 * warp;  // tokens of my 16
+    const int valid = (t_flags & kBadTile) ? 0 : t_valid - 16 * warp;  // tokens of my 16
     if (valid > 0) {
       const uint32_t kbase = smem_u32(tiles + stage * Ly::kStageB);
       const uint32_t vbase = kbase + Ly::kTileB;
@@ -489,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
       // ---- online softmax on row gid (log2 domain) ----
-      const float mul = kFp8 ? qk_mul * ti.ks : qk_mul;
+      const float mul = kFp8 ? qk_mul * t_ks : qk_mul;
       float x[4];
 #pragma unroll
       for (int n = 0; n < 2; ++n)
@@ -508,19 +574,24 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int e = 0; e < 4; ++e) pr[e] = fast_exp2(x[e] - m_new);
       l_part = l_part * alpha + (pr[0] + pr[1]) + (pr[2] + pr[3]);
       m_run = m_new;
+      // alpha belongs to head gid; O^T columns are heads 2*tid4 and 2*tid4+1
+      const float a_lo = __shfl_sync(0xffffffffu, alpha, 8 * tid4);
+      const float a_hi = __shfl_sync(0xffffffffu, alpha, 8 * tid4 + 4);
 #pragma unroll
-      for (int n = 0; n < D / 8; ++n) {
-        o[n][0] *= alpha;
-        o[n][1] *= alpha;
+      for (int m = 0; m < D / 16; ++m) {
+        ot[m][0] *= a_lo;
+        ot[m][1] *= a_hi;
+        ot[m][2] *= a_lo;
+        ot[m][3] *= a_hi;
       }
-      // ---- O += P V over my 16 tokens ----
+      // ---- O^T += V^T P^T over my 16 tokens (P^T comes straight from S) ----
       uint32_t pa0, pa2;
       if constexpr (!kFp8) {
         pa0 = pack_bf16(pr[0], pr[1]);
         pa2 = pack_bf16(pr[2], pr[3]);
       } else {
-        pa0 = pack_f16(pr[0] * ti.vs, pr[1] * ti.vs);
-        pa2 = pack_f16(pr[2] * ti.vs, pr[3] * ti.vs);
+        pa0 = pack_f16(pr[0] * t_vs, pr[1] * t_vs);
+        pa2 = pack_f16(pr[2] * t_vs, pr[3] * t_vs);
       }
       // V rows past the length may hold anything (NaN); zero them in the
       // fragments so that 0 * NaN never reaches the accumulator.
@@ -571,117 +642,169 @@ __global__ void __launch_bounds__(kThreads, 2)
         vsrc = cbase;
       }
 #pragma unroll
-      for (int dp = 0; dp < D / 16; ++dp) {
-        // matrices: (tokens 0-7, d-chunk 2dp), (8-15, 2dp), (0-7, 2dp+1), (8-15, 2dp+1)
-        const int chunk = 2 * dp + (mat >> 1);
-        uint32_t v0, v1, v2, v3;
+      for (int m = 0; m < D / 16; ++m) {
+        // A = V^T rows d 16m..16m+15: matrices (tokens 0-7, chunk 2m), (0-7, 2m+1),
+        // (8-15, 2m), (8-15, 2m+1), transposed on load
+        const int chunk = 2 * m + (mat & 1);
+        uint32_t a0, a1, a2, a3;
         if constexpr (!kFp8) {
-          const int row = 16 * warp + mrow + (mat & 1) * 8;
-          ldsm_x4_t(tile_addr<Ly::kBoxRowB, kTile>(vsrc, row, chunk), v0, v1, v2, v3);
+          const int row = 16 * warp + mrow + (mat >> 1) * 8;
+          ldsm_x4_t(tile_addr<Ly::kBoxRowB, kTile>(vsrc, row, chunk), a0, a1, a2, a3);
         } else {
-          const int row = mrow + (mat & 1) * 8;
-          ldsm_x4_t(tile_addr<128, 16>(vsrc, row, chunk), v0, v1, v2, v3);
+          const int row = mrow + (mat >> 1) * 8;
+          ldsm_x4_t(tile_addr<128, 16>(vsrc, row, chunk), a0, a1, a2, a3);
         }
-        v0 &= vm0;
-        v2 &= vm0;
-        v1 &= vm1;
-        v3 &= vm1;
-        if constexpr (!kFp8) {
-          mma_bf16(o[2 * dp], pa0, 0u, pa2, 0u, v0, v1);
-          mma_bf16(o[2 * dp + 1], pa0, 0u, pa2, 0u, v2, v3);
-        } else {
-          mma_f16(o[2 * dp], pa0, 0u, pa2, 0u, v0, v1);
-          mma_f16(o[2 * dp + 1], pa0, 0u, pa2, 0u, v2, v3);
+        a0 &= vm0;
+        a1 &= vm0;
+        a2 &= vm1;
+        a3 &= vm1;
+        if constexpr (!kFp8)
+          mma_bf16(ot[m], a0, a1, a2, a3, pa0, pa2);
+        else
+          mma_f16(ot[m], a0, a1, a2, a3, pa0, pa2);
+      }
+    }
+    if (t_flags & kSegLast) {
+    // ------------------------------------------- hand the segment over
+    // Snapshot this warp's (m, l, o) for the flush warp and go on streaming.
+    float l_row = l_part;
+    l_row += __shfl_xor_sync(0xffffffffu, l_row, 1);
+    l_row += __shfl_xor_sync(0xffffffffu, l_row, 2);
+    if (nflush > 0 && !mbar_wait(red_empty, (uint32_t)((nflush - 1) & 1), p.flags)) return;
+    if (row_ok && tid4 == 0) {
+      red_m[warp * G + gid] = m_run;
+      red_l[warp * G + gid] = l_row;
+    }
+    {
+      const int h0 = 2 * tid4, h1 = 2 * tid4 + 1;
+      float* r0 = red_o + (warp * G + h0) * D;
+      float* r1 = red_o + (warp * G + h1) * D;
+#pragma unroll
+      for (int m = 0; m < D / 16; ++m) {
+        const int d = 16 * m + gid;
+        if (h0 < G) {
+          r0[d] = ot[m][0];
+          r0[d + 8] = ot[m][2];
+        }
+        if (h1 < G) {
+          r1[d] = ot[m][1];
+          r1[d + 8] = ot[m][3];
         }
       }
+    }
+    if (warp == 0 && lane == 0) {
+      const TileInfo& ti = info[stage];
+      FlushDesc fd;
+      fd.b = ti.b;
+      fd.g = ti.g;
+      fd.slot = ti.slot;
+      fd.seg_base = ti.seg_base;
+      fd.nseg = ti.nseg;
+      fd.whole = (t_flags & kUnitWhole) ? 1 : 0;
+      fd.final = (i == n_tiles - 1) ? 1 : 0;
+      *desc = fd;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(red_full);
+    ++nflush;
     }
     // release the stage (all of this warp's reads of it are done)
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[stage]);
+  }
+}
 
-    if (!(ti.flags & kSegLast)) continue;
+// --------------------------------------------------------- split reduce
+// One warp per (sequence, kv head) unit whose tiles were cut across CTAs:
+// out = sum_i e^{m_i - M} o_i / sum_i e^{m_i - M} l_i, lse = M + ln(...), in
+// the log2 domain of the partials.  Launched as a programmatic dependent of
+// the decode kernel: it may start early and waits for the decode grid's
+// completion (and memory) before reading any partial.
+template <int D, int G>
+__global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int lane = threadIdx.x & 31;
+  const int u = blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (u >= p.batch * p.num_kv_heads) return;
+  const int b = u / p.num_kv_heads;
+  const int g = u - b * p.num_kv_heads;
+  const int2 info = p.unit_info[u];
+  if (clamp_len(p, __ldg(p.seq_lens + b), false) == 0) return;  // written by the decode kernel
+  const int n = info.y;
+  if (n <= 1) return;  // whole unit: written by the decode kernel
+  constexpr int GD = G * D;
+  constexpr int kJ = GD / 32;  // elements of the unit's output per lane
+  const int64_t mlb = (int64_t)info.x * G;
+  const float* po = p.part_o + (int64_t)info.x * GD;
+  // Every load of a segment (its G (m, l) pairs and this lane's kJ partial
+  // outputs) is independent, so a segment costs one memory round trip and
+  // consecutive segments overlap.
+  float mrow[G], lrow[G], num[kJ];
+#pragma unroll
+  for (int r = 0; r < G; ++r) {
+    mrow[r] = -INFINITY;
+    lrow[r] = 0.f;
+  }
+#pragma unroll
+  for (int j = 0; j < kJ; ++j) num[j] = 0.f;
+  // pass over segments with a running (online) max per row
+#pragma unroll 2
+  for (int sgm = 0; sgm < n; ++sgm) {
+    float2 ml[G];
+    float ov[kJ];
+#pragma unroll
+    for (int r = 0; r < G; ++r) ml[r] = __ldcg(&p.part_ml[mlb + (int64_t)sgm * G + r]);
+#pragma unroll
+    for (int j = 0; j < kJ; ++j) ov[j] = __ldcg(po + (int64_t)sgm * GD + lane + 32 * j);
+    float sc_old[G], sc_new[G];
+#pragma unroll
+    for (int r = 0; r < G; ++r) {
+      const float m_new = fmaxf(mrow[r], ml[r].x);
+      sc_old[r] = mrow[r] == -INFINITY ? 0.f : fast_exp2(mrow[r] - m_new);
+      sc_new[r] = ml[r].x == -INFINITY ? 0.f : fast_exp2(ml[r].x - m_new);
+      lrow[r] = lrow[r] * sc_old[r] + ml[r].y * sc_new[r];
+      mrow[r] = m_new;
+    }
+#pragma unroll
+    for (int j = 0; j < kJ; ++j) {
+      constexpr int kPerRow = D / 32;
+      const int r = j / kPerRow;
+      num[j] = num[j] * sc_old[r] + ov[j] * sc_new[r];
+    }
+  }
+  __nv_bfloat16* ob = p.out + ((int64_t)b * p.num_q_heads + g * G) * D;
+#pragma unroll
+  for (int j = 0; j < kJ; ++j) {
+    constexpr int kPerRow = D / 32;
+    const int r = j / kPerRow;
+    ob[lane + 32 * j] = __float2bfloat16(lrow[r] > 0.f ? num[j] / lrow[r] : 0.f);
+  }
+  if (lane == 0 && p.lse) {
+#pragma unroll
+    for (int r = 0; r < G; ++r)
+      p.lse[(int64_t)b * p.num_q_heads + g * G + r] =
+          lrow[r] > 0.f ? (mrow[r] + log2f(lrow[r])) * 0.69314718055994531f : -INFINITY;
+  }
+}
 
-    // ----------------------------------------------------------- flush
-    float l_row = l_part;
-    l_row += __shfl_xor_sync(0xffffffffu, l_row, 1);
-    l_row += __shfl_xor_sync(0xffffffffu, l_row, 2);
-    if (row_ok) {
-      if (tid4 == 0) {
-        red_m[warp * G + gid] = m_run;
-        red_l[warp * G + gid] = l_row;
-      }
-      float* ro = red_o + (warp * G + gid) * D;
-#pragma unroll
-      for (int n = 0; n < D / 8; ++n)
-        *reinterpret_cast<float2*>(ro + 8 * n + 2 * tid4) = make_float2(o[n][0], o[n][1]);
-    }
-    if (!csync.sync(p.flags)) return;
-    const bool whole = ti.flags & kUnitWhole;
-    const int ctid = threadIdx.x;  // 0..127
-    for (int e = ctid; e < G * D; e += kConsumerWarps * 32) {
-      const int row = e / D;
-      const int d = e - row * D;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red_m[w * G + row]);
-      float num = 0.f, den = 0.f;
-      if (M != -INFINITY) {
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
-          const float mw = red_m[w * G + row];
-          if (mw == -INFINITY) continue;
-          const float sc = exp2f(mw - M);
-          num += sc * red_o[(w * G + row) * D + d];
-          den += sc * red_l[w * G + row];
-        }
-      }
-      const int h = ti.g * G + row;
-      const int64_t orow = (int64_t)ti.b * p.num_q_heads + h;
-      if (whole) {
-        p.out[orow * D + d] = __float2bfloat16(den > 0.f ? num / den : 0.f);
-        if (d == 0 && p.lse)
-          p.lse[orow] = den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
-      } else {
-        p.part_o[((int64_t)ti.slot * G + row) * D + d] = num;
-        if (d == 0) p.part_ml[(int64_t)ti.slot * G + row] = make_float2(M, den);
-      }
-    }
-    if (!whole) {
-      __threadfence();
-      if (!csync.sync(p.flags)) return;
-      if (ctid == 0) {
-        const int u = ti.b * Hkv + ti.g;
-        const int old = atomicAdd(p.counters + u, 1);
-        s_misc[1] = (old == ti.nseg - 1);
-      }
-      if (!csync.sync(p.flags)) return;
-      if (s_misc[1]) {
-        __threadfence();
-        for (int e = ctid; e < G * D; e += kConsumerWarps * 32) {
-          const int row = e / D;
-          const int d = e - row * D;
-          float M = -INFINITY;
-          for (int s = 0; s < ti.nseg; ++s)
-            M = fmaxf(M, __ldcg(&p.part_ml[(int64_t)(ti.seg_base + s) * G + row]).x);
-          float num = 0.f, den = 0.f;
-          if (M != -INFINITY) {
-            for (int s = 0; s < ti.nseg; ++s) {
-              const float2 ml = __ldcg(&p.part_ml[(int64_t)(ti.seg_base + s) * G + row]);
-              if (ml.x == -INFINITY) continue;
-              const float sc = exp2f(ml.x - M);
-              num += sc * __ldcg(&p.part_o[((int64_t)(ti.seg_base + s) * G + row) * D + d]);
-              den += sc * ml.y;
-            }
-          }
-          const int64_t orow = (int64_t)ti.b * p.num_q_heads + ti.g * G + row;
-          p.out[orow * D + d] = __float2bfloat16(den > 0.f ? num / den : 0.f);
-          if (d == 0 && p.lse)
-            p.lse[orow] = den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
-        }
-        if (ctid == 0) p.counters[ti.b * Hkv + ti.g] = 0;  // leave the workspace clean
-      }
-    }
-    if (!csync.sync(p.flags)) return;  // the reduction buffers may be reused
+template <int D>
+cudaError_t merge_launch(const DecodeParams& p, cudaStream_t stream) {
+  const int units = p.batch * p.num_kv_heads;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((units + 3) / 4);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  switch (p.group) {
+    case 1: return cudaLaunchKernelEx(&cfg, decode_merge_kernel<D, 1>, p);
+    case 2: return cudaLaunchKernelEx(&cfg, decode_merge_kernel<D, 2>, p);
+    case 4: return cudaLaunchKernelEx(&cfg, decode_merge_kernel<D, 4>, p);
+    default: return cudaLaunchKernelEx(&cfg, decode_merge_kernel<D, 8>, p);
   }
 }
 
@@ -734,11 +857,14 @@ cudaError_t occupancy_for(int G, int* n) {
 template <int D, bool kFp8>
 cudaError_t run_for(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                     int num_ctas, cudaStream_t stream) {
+  cudaError_t e;
   switch (pick_stages<D, kFp8>(p.group)) {
-    case 4: return decode_launch<D, kFp8, 4>(tk, tv, p, num_ctas, stream);
-    case 3: return decode_launch<D, kFp8, 3>(tk, tv, p, num_ctas, stream);
-    default: return decode_launch<D, kFp8, 2>(tk, tv, p, num_ctas, stream);
+    case 4: e = decode_launch<D, kFp8, 4>(tk, tv, p, num_ctas, stream); break;
+    case 3: e = decode_launch<D, kFp8, 3>(tk, tv, p, num_ctas, stream); break;
+    default: e = decode_launch<D, kFp8, 2>(tk, tv, p, num_ctas, stream); break;
   }
+  if (e != cudaSuccess) return e;
+  return merge_launch<D>(p, stream);
 }
 
 cudaError_t decode_occupancy(int head_dim, bool fp8, int group, int* ctas_per_sm) {

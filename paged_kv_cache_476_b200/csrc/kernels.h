@@ -40,7 +40,7 @@ struct DecodeParams {
   float* lse;          // [B][Hq] or null
   float* part_o;       // [U + C][G][D]
   float2* part_ml;     // [U + C][G]
-  int32_t* counters;   // [U]
+  int2* unit_info;     // [U]: (first partial slot, number of segments)
   int32_t* flags;
   int32_t batch;
   int32_t num_q_heads;

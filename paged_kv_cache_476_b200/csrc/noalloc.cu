@@ -1,7 +1,7 @@
 // Decode attention for callers that cannot allocate device memory.
 //
 // paged_decode_attention needs a caller-provided workspace for its split
-// partials and per-unit counters.  Some callers have no way to obtain one:
+// partials and per-unit records.  Some callers have no way to obtain one:
 // code running where cudaMalloc is forbidden or unavailable (inside a host
 // callback or a foreign runtime that owns all allocations, an embedded or
 // plugin context handed only input/output pointers), or code that must not
@@ -15,9 +15,9 @@
 //  * All calls on one device share the array.  Two calls whose executions
 //    overlap on the GPU (different streams, no ordering between them) race
 //    on it and produce wrong results; order them on one stream.
-//  * The array keeps whatever the last call left in it.  Each call clears the
-//    part it uses before launching (an asynchronous memset on the caller's
-//    stream, which allocates nothing).
+//  * The array keeps whatever the last call left in it.  That is harmless:
+//    every value a call reads from it was written earlier by the same call,
+//    so nothing needs to start at zero.
 //  * The first call on a device looks up the array's device address (host
 //    code cannot use the array's name as a device pointer).  Make that first
 //    call before capturing any stream into a CUDA graph.
@@ -29,7 +29,7 @@
 
 namespace pkv {
 
-// Static decode scratch: partials + counters of paged_decode_attention.
+// Static decode scratch: split partials + per-unit records of paged_decode_attention.
 static __device__ __align__(256) uint8_t g_decode_scratch[PKV_NOALLOC_SCRATCH_BYTES];
 
 namespace {
@@ -76,8 +76,6 @@ extern "C" int paged_decode_attention_noalloc(const pkv_cache* cache, const void
   if (need > (size_t)PKV_NOALLOC_SCRATCH_BYTES) return PKV_ERR_SCRATCH_LIMIT;
   void* scratch = nullptr;
   if ((st = scratch_address(&scratch))) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(scratch, 0, need, s) != cudaSuccess) return PKV_ERR_CUDA;
   return paged_decode_attention(cache, q, num_q_heads, gqa_group, page_table, max_pages_per_seq,
                                 seq_lens, batch, max_seq_len, softmax_scale, out, lse, scratch,
                                 (size_t)PKV_NOALLOC_SCRATCH_BYTES, num_ctas, stream);

@@ -10,7 +10,8 @@ This file checks, through the C ABI, that the allocation-free entry point
 returns what the workspace entry point returns (within the tolerance the
 parity tests use: max-abs 1e-2, mean-abs 1e-3, lse 2e-3) on two calls in a
 row and on a following call with a different batch (the scratch keeps the
-previous call's contents), and that sizes beyond the scratch are rejected
+previous call's contents, which the new call must not read), and that sizes
+beyond the scratch are rejected
 before anything runs.  It is named to be collected last.
 """
 import ctypes
