@@ -51,6 +51,31 @@ def parse():
     return ap.parse_args()
 
 
+def decode_traffic():
+    """ncu DRAM bytes per decode call from profiles/, if the sources still match.
+
+    The decode kernel's sources are hashed; a capture taken on other sources
+    is stale and reported as null.
+    """
+    import hashlib
+
+    src = os.path.join(ROOT, "paged_kv_cache_476_b200", "csrc")
+    h = hashlib.sha256()
+    for f in ("decode.cu", "common.cuh", "kernels.h"):
+        with open(os.path.join(src, f), "rb") as fh:
+            h.update(fh.read())
+    sha = h.hexdigest()[:16]
+    try:
+        with open(os.path.join(ROOT, "profiles", "decode_kernel_llama8b_decode.md")) as fh:
+            kv = dict(line.strip().split(": ", 1) for line in fh if ": " in line and
+                      line.startswith(("traffic_bytes_per_call", "source_sha256_16")))
+        if kv.get("source_sha256_16") == sha:
+            return int(kv["traffic_bytes_per_call"])
+    except (OSError, ValueError, KeyError):
+        pass
+    return None
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -362,13 +387,15 @@ def run_ours(args, rank, world, device, dist):
                        "prefill": round(pf_s * 1e3, 5) if has_pf else None},
         "roofline": {
             "bound": "hbm",
-            "kernel": "decode_kernel",
+            "kernel": "decode_kernel + decode_merge_kernel (one paged_decode_attention call)",
             "achieved": round(achieved, 1),
             "peak": hbm_peak,
             "unit": "GB/s",
             "frac": round(achieved / hbm_peak, 4),
             "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth)",
-            "traffic": None,
+            "traffic": decode_traffic() if args.config == 2 else None,
+            "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of "
+                              "decode_kernel + decode_merge_kernel (profiles/)",
             "algorithmic_bytes_per_launch": int(dbytes),
         },
         "e2e": {"value": round(world * step_bytes / e2e_s / 1e9, 2), "unit": "GB/s",
