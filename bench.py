@@ -51,6 +51,26 @@ def parse():
     return ap.parse_args()
 
 
+def max_over_ranks(x: float, dist, device=None) -> float:
+    """Largest value of ``x`` over all ranks (identity without a process group).
+
+    Multi-GPU times are the max over ranks, taken on the device tensors of
+    the rank (NCCL) or on CPU tensors (gloo).
+    """
+    if dist is None:
+        return float(x)
+    import torch
+
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, seconds: float) -> float:
+    """Weak-scaling throughput: units all ranks processed / the slowest rank's time."""
+    return world * units_per_rank / seconds
+
+
 def decode_traffic():
     """ncu DRAM bytes per decode call from profiles/, if the sources still match.
 
@@ -294,12 +314,7 @@ def run_ours(args, rank, world, device, dist):
     dec_s = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps / 1e3
     app_s = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps / 1e3
     pf_s = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps / 1e3
-    if dist:
-        import torch.distributed as tdist
-
-        t = torch.tensor([elapsed], device=device)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        elapsed = float(t.item())
+    elapsed = max_over_ranks(elapsed, dist, device)
 
     # ---------------------------------------------------------------- e2e
     # Through the public API with host buffers: per step, H2D of the step's
@@ -342,12 +357,7 @@ def run_ours(args, rank, world, device, dist):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_s = e0.elapsed_time(e1) / 1e3 / e_steps
-    if dist:
-        import torch.distributed as tdist
-
-        t = torch.tensor([e2e_s], device=device)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        e2e_s = float(t.item())
+    e2e_s = max_over_ranks(e2e_s, dist, device)
     h2d = sum(st[k].numel() * st[k].element_size() for k in names)
     d2h = h_out.numel() * h_out.element_size()
 
@@ -359,7 +369,7 @@ def run_ours(args, rank, world, device, dist):
     achieved = dbytes / dec_s / 1e9
     res = {
         "metric": METRIC,
-        "value": round(world * step_bytes / step_s / 1e9, 2),
+        "value": round(whole_job_rate(step_bytes, world, step_s) / 1e9, 2),
         "unit": "GB/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -370,7 +380,7 @@ def run_ours(args, rank, world, device, dist):
         "vs_baseline": None,
         "dtype": "bf16" if w.kv_dtype == "bf16" else "e4m3-kv/bf16-q",
         "data": "synthetic (seeded N(0,1) bf16 K/V/Q, permuted pages, NaN sentinels)",
-        "tokens_per_s": round(world * len(w.decode_rows) / step_s, 1),
+        "tokens_per_s": round(whole_job_rate(len(w.decode_rows), world, step_s), 1),
         "config": {
             "workload": w.name,
             "batch": int(len(w.decode_rows)),
@@ -398,7 +408,7 @@ def run_ours(args, rank, world, device, dist):
                               "decode_kernel + decode_merge_kernel (profiles/)",
             "algorithmic_bytes_per_launch": int(dbytes),
         },
-        "e2e": {"value": round(world * step_bytes / e2e_s / 1e9, 2), "unit": "GB/s",
+        "e2e": {"value": round(whole_job_rate(step_bytes, world, e2e_s) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "ms_per_step": round(e2e_s * 1e3, 5)},
         "gpu_launches": launches_per_step * args.steps,
