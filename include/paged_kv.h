@@ -184,7 +184,8 @@ int paged_decode_attention(const pkv_cache* cache, const void* q, int32_t num_q_
  *   seq_lens   int32 [num_chunks]
  *   total_q    host copy of cu_q_lens[num_chunks] (rows of q and out)
  *   max_q_len  host upper bound of any chunk's query count (plans the grid)
- * This build runs prefill on bf16 pools; E4M3 pools return PKV_ERR_UNSUPPORTED.
+ * E4M3 pools are converted tile by tile to bf16 in shared memory (exact) and
+ * their per-(page, head) scales applied to the scores (K) and to P (V).
  *   out        bf16 [total_q][num_q_heads][head_dim]
  *   lse        fp32 [total_q][num_q_heads], or NULL
  */

@@ -25,6 +25,11 @@
 //    rescaled in TMEM), write P to TMEM, and finally normalise O.
 //  * V rows past the sequence end (or of a rejected page) are zeroed in
 //    shared memory before their PV product: 0 * NaN would poison O.
+//  * E4M3 pools: two converter warps turn each landed E4M3 tile into a 16-bit
+//    tile (exact) laid out as TMA lays out bf16 tiles: K as bf16 (Q's type),
+//    V as f16.  The per-(page, head) K scales multiply the scores of their
+//    64-key block; the V scales ride on P, kept in f16 (11-bit mantissa) so
+//    that PV is an f16 x f16 product.
 //  * Every wait is bounded; TMEM is freed on every exit path.
 #include "common.cuh"
 #include "kernels.h"
@@ -36,13 +41,17 @@ namespace pf {
 constexpr int kRows = 128;     // M of the Q tile
 constexpr int kKeys = 128;     // N of the S tile (keys per KV tile)
 constexpr int kStages = 2;     // K/V ring depth
-constexpr int kThreads = 192;  // warps 0-3 softmax, 4 producer, 5 MMA
+// warps 0-3 softmax (one TMEM lane = one row per thread), 4 producer, 5 MMA,
+// 6-7 E4M3 -> bf16 converters (E4M3 pools only)
 constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
+constexpr int kConvWarp0 = 6;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP = 384;
 
 struct Params {
+  const float* k_scale;  // [pages][Hkv] (E4M3 pools)
+  const float* v_scale;
   const int32_t* cu_q;
   const int32_t* page_table;
   const int32_t* seq_lens;
@@ -160,49 +169,129 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, ui
   return d;
 }
 
-// Instruction descriptor of kind::f16: bf16 x bf16 -> f32, M x N, operand majors.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn_major) {
-  return (1u << 4)                         // D format f32
-         | (1u << 7)                       // A bf16
-         | (1u << 10)                      // B bf16
-         | ((uint32_t)b_mn_major << 16)    // B major: 0 K, 1 MN
-         | ((uint32_t)(N >> 3) << 17)      // N / 8
-         | ((uint32_t)(M >> 4) << 24);     // M / 16
+// Instruction descriptor of kind::f16 with f32 accumulation: A and B both
+// bf16 (or both f16), M x N, B K- or MN-major.
+__host__ __device__ constexpr uint32_t idesc_f16kind(int M, int N, int b_mn_major, bool bf16) {
+  return (1u << 4)                           // D format f32
+         | ((bf16 ? 1u : 0u) << 7)           // A: 1 bf16, 0 f16
+         | ((bf16 ? 1u : 0u) << 10)          // B: same type as A
+         | ((uint32_t)b_mn_major << 16)      // B major: 0 K, 1 MN
+         | ((uint32_t)(N >> 3) << 17)        // N / 8
+         | ((uint32_t)(M >> 4) << 24);       // M / 16
 }
 
-template <int D>
+template <int D, bool kFp8>
 struct Smem {
-  static constexpr int kHalves = D / 64;          // 128-byte column boxes per row
-  static constexpr int kQB = kRows * D * 2;       // Q tile
-  static constexpr int kTileB = kKeys * D * 2;    // K (or V) tile
-  static constexpr int kHalfB = kKeys * 128;      // one 64-column half of a K/V tile
-  static constexpr int kStageB = 2 * kTileB;
-  static constexpr int kBytes = kQB + kStages * kStageB;
+  static constexpr int kHalves = D / 64;            // 128-byte column boxes per bf16 row
+  static constexpr int kQB = kRows * D * 2;         // Q tile
+  static constexpr int kTileB = kKeys * D * 2;      // bf16 K (or V) tile
+  static constexpr int kHalfB = kKeys * 128;        // one 64-column half of a bf16 tile
+  static constexpr int kTile8B = kKeys * D;         // E4M3 K (or V) tile as it lands
+  static constexpr int kStageB = kFp8 ? 2 * kTile8B : 2 * kTileB;
+  static constexpr int kConvB = kFp8 ? 2 * kTileB : 0;  // converted K, then V
+  static constexpr int kBytes = kQB + kStages * kStageB + kConvB;
+  static constexpr int kThreads = kFp8 ? 256 : 192;  // + two converter warps
 };
 
+// Per-KV-tile facts the producer passes on: rejected 64-key blocks and the
+// E4M3 scales of the (up to two) pages of the tile.
+struct TileFacts {
+  int32_t bad;
+  float ks[2], vs[2];
+};
+constexpr int kFactsRing = 4;
+
+// Shared-memory byte address of 16-byte chunk c (0..D/8-1) of row r of a bf16
+// tile laid out as TMA writes it: 64-column halves kHalfB apart, 128-byte
+// rows, 128-byte swizzle.
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__device__ __forceinline__ uint32_t bf16_chunk(uint32_t base, int r, int c) {
+  return base + (c >> 3) * (kKeys * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+}
+
+// Same for an E4M3 tile as TMA writes it: rows of D bytes, 128-byte swizzle
+// (D = 128) or 64-byte swizzle (D = 64).
+template <int D>
+__device__ __forceinline__ uint32_t e4m3_chunk(uint32_t base, int r, int c) {
+  if constexpr (D == 128)
+    return base + r * 128 + ((c ^ (r & 7)) << 4);
+  else
+    return base + r * 64 + ((c ^ ((r >> 1) & 3)) << 4);
+}
+
+// E4M3 tile -> bf16 or f16 tile (both exact: every E4M3 value is an f16 and a
+// bf16), rows in `zero_mask` (bit per 64-row block) or at/after `zero_from`
+// written as zeros.  64 threads share the work.
+template <int D, bool kToF16>
+__device__ __forceinline__ void convert_tile(uint32_t src, uint32_t dst, int t, int zero_from,
+                                             int zero_mask) {
+  constexpr int kChunks = kKeys * D / 16;  // 16-byte E4M3 chunks
+#pragma unroll 4
+  for (int ci = t; ci < kChunks; ci += 64) {
+    const int r = ci / (D / 16);
+    const int c = ci - r * (D / 16);
+    uint32_t o[8];
+    if (r >= zero_from || ((zero_mask >> (r >> 6)) & 1)) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) o[k] = 0u;
+    } else {
+      uint32_t w[4];
+      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                   : "r"(e4m3_chunk<D>(src, r, c)));
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t h01 = e4m3x2_to_f16x2(w[k] & 0xffff);
+        const uint32_t h23 = e4m3x2_to_f16x2(w[k] >> 16);
+        if constexpr (kToF16) {
+          o[2 * k] = h01;
+          o[2 * k + 1] = h23;
+        } else {
+          const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+          const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+          o[2 * k] = pack_bf16(f01.x, f01.y);
+          o[2 * k + 1] = pack_bf16(f23.x, f23.y);
+        }
+      }
+    }
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(bf16_chunk<D>(dst, r, 2 * c)),
+                 "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3])
+                 : "memory");
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
+                     bf16_chunk<D>(dst, r, 2 * c + 1)),
+                 "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7])
+                 : "memory");
+  }
+}
+
+template <int D, bool kFp8>
+__global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,
                    const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v, const Params p) {
-  using Sm = Smem<D>;
+  using Sm = Smem<D, kFp8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* sq = smem;
-  uint8_t* skv = smem + Sm::kQB;  // stage s: K at s*kStageB, V at +kTileB
+  uint8_t* skv = smem + Sm::kQB;                    // stage s: K at s*kStageB, V after it
+  uint8_t* sconv = skv + kStages * Sm::kStageB;     // E4M3 only: bf16 K, then bf16 V
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sm::kBytes);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;             // [kStages]
-  uint64_t* kv_empty = kv_full + kStages;   // [kStages]
-  uint64_t* s_full = kv_empty + kStages;    // [2]
-  uint64_t* s_free = s_full + 2;            // [2]
+  uint64_t* kv_full = bars + 1;               // [kStages] TMA landed
+  uint64_t* kv_empty = kv_full + kStages;     // [kStages] stage may be refilled
+  uint64_t* s_full = kv_empty + kStages;      // [2]
+  uint64_t* s_free = s_full + 2;              // [2]
   uint64_t* p_full = s_free + 2;
   uint64_t* o_bar = p_full + 1;
   uint64_t* done_bar = o_bar + 1;
-  uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(done_bar + 1);
-  int32_t* stage_bad = reinterpret_cast<int32_t*>(tmem_base_smem + 1);  // [kStages] bit/sub-block
-  int32_t* s_abort = stage_bad + kStages;
+  uint64_t* kc_full = done_bar + 1;           // E4M3: converted K ready / free
+  uint64_t* kc_free = kc_full + 1;
+  uint64_t* vc_full = kc_free + 1;            // E4M3: converted V ready / free
+  uint64_t* vc_free = vc_full + 1;
+  uint64_t* facts_full = vc_free + 1;         // [kFactsRing] producer -> softmax
+  TileFacts* facts = reinterpret_cast<TileFacts*>(facts_full + kFactsRing);
+  uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(facts + kFactsRing);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -231,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_full, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&kv_empty[s], kFp8 ? 2 : 1);  // E4M3: released by the two converter warps
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
@@ -240,7 +329,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(p_full, 4);
     mbar_init(o_bar, 1);
     mbar_init(done_bar, 1);
-    *s_abort = 0;
+    mbar_init(kc_full, 2);
+    mbar_init(kc_free, 1);
+    mbar_init(vc_full, 2);
+    mbar_init(vc_free, 1);
+    for (int s = 0; s < kFactsRing; ++s) mbar_init(&facts_full[s], 1);
     fence_barrier_init();
   }
   if (warp == kMmaWarp) tmem_alloc(tmem_base_smem, kTmemCols);
@@ -261,83 +354,132 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(sq + h * (kRows * 128), &tmap_q, h * 64, g * G, q_begin + qt0, q_full);
     }
     const uint64_t pol = policy_evict_first();
-    (void)pol;
     for (int j = 0; j < n_kv; ++j) {
       const int st = j % kStages;
       if (j >= kStages) {
-        if (!mbar_wait(&kv_empty[st], (uint32_t)((j / kStages - 1) & 1), p.flags)) {
-          *s_abort = 1;
-          break;
-        }
+        if (!mbar_wait(&kv_empty[st], (uint32_t)((j / kStages - 1) & 1), p.flags)) break;
       }
       if (lane == 0) {
         uint8_t* kd = skv + st * Sm::kStageB;
-        uint8_t* vd = kd + Sm::kTileB;
-        int bad = 0;
+        uint8_t* vd = kd + Sm::kStageB / 2;
+        TileFacts tf;
+        tf.bad = 0;
         uint32_t bytes = 0;
         int32_t ys[2] = {0, 0};
         bool live[2] = {false, false};
         for (int sb = 0; sb < 2; ++sb) {
+          tf.ks[sb] = tf.vs[sb] = 1.f;
           const int32_t key0 = j * kKeys + sb * 64;
           if (key0 >= L) continue;
           const int32_t pj = key0 / p.page_size;
           int32_t pid = __ldg(p.page_table + (int64_t)chunk * p.max_pages + pj);
           if (pid < 0 || pid >= p.num_pages) {
             flag_error(p.flags, PKV_FLAG_BAD_PAGE);
-            bad |= 1 << sb;
+            tf.bad |= 1 << sb;
             continue;
+          }
+          if constexpr (kFp8) {
+            const float ks = __ldg(p.k_scale + (int64_t)pid * p.num_kv_heads + g);
+            const float vs = __ldg(p.v_scale + (int64_t)pid * p.num_kv_heads + g);
+            if (!(ks > 0.f && ks <= 32768.f && vs > 0.f && vs <= 32768.f)) {
+              flag_error(p.flags, PKV_FLAG_BAD_SCALE);
+              tf.bad |= 1 << sb;
+              continue;
+            }
+            tf.ks[sb] = ks;
+            tf.vs[sb] = vs;
           }
           ys[sb] = (int32_t)(((int64_t)pid * p.num_kv_heads + g) * p.page_size +
                              key0 % p.page_size);
           live[sb] = true;
-          bytes += 2u * Sm::kHalves * 64u * 128u;
+          bytes += kFp8 ? 2u * 64u * D : 2u * Sm::kHalves * 64u * 128u;
         }
-        stage_bad[st] = bad;
+        facts[j % kFactsRing] = tf;
+        mbar_arrive(&facts_full[j % kFactsRing]);
         mbar_arrive_expect_tx(&kv_full[st], bytes);
         for (int sb = 0; sb < 2; ++sb) {
           if (!live[sb]) continue;
+          if constexpr (kFp8) {
+            tma_load_2d(kd + sb * 64 * D, &tmap_k, 0, ys[sb], &kv_full[st], pol);
+            tma_load_2d(vd + sb * 64 * D, &tmap_v, 0, ys[sb], &kv_full[st], pol);
+          } else {
 #pragma unroll
-          for (int h = 0; h < Sm::kHalves; ++h) {
-            tma_load_2d(kd + h * Sm::kHalfB + sb * 64 * 128, &tmap_k, h * 64, ys[sb],
-                        &kv_full[st], pol);
-            tma_load_2d(vd + h * Sm::kHalfB + sb * 64 * 128, &tmap_v, h * 64, ys[sb],
-                        &kv_full[st], pol);
+            for (int h = 0; h < Sm::kHalves; ++h) {
+              tma_load_2d(kd + h * Sm::kHalfB + sb * 64 * 128, &tmap_k, h * 64, ys[sb],
+                          &kv_full[st], pol);
+              tma_load_2d(vd + h * Sm::kHalfB + sb * 64 * 128, &tmap_v, h * 64, ys[sb],
+                          &kv_full[st], pol);
+            }
           }
         }
       }
       __syncwarp();
     }
+  } else if (kFp8 && warp >= kConvWarp0) {
+    // ------------------------------------------------- E4M3 -> bf16 converters
+    const int t = threadIdx.x - kConvWarp0 * 32;  // 0..63
+    const uint32_t kc = smem_u32(sconv), vc = kc + Sm::kTileB;
+    for (int j = 0; j < n_kv; ++j) {
+      const int st = j % kStages;
+      if (!mbar_wait(&kv_full[st], (uint32_t)((j / kStages) & 1), p.flags)) break;
+      const uint32_t k8 = smem_u32(skv + st * Sm::kStageB), v8 = k8 + Sm::kStageB / 2;
+      const int bad = facts[j % kFactsRing].bad;
+      const int32_t key0 = j * kKeys;
+      const int zero_from = key0 + kKeys > L ? max(0, L - key0) : kKeys;
+      // K (rows that must not count are masked in the scores; keep them finite)
+      if (j >= 1 && !mbar_wait(kc_free, (uint32_t)((j - 1) & 1), p.flags)) break;
+      convert_tile<D, false>(k8, kc, t, zero_from, bad);  // bf16, like Q
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(kc_full);
+      // V (rows that must not count are zeros: 0 * NaN would poison O)
+      if (j >= 1 && !mbar_wait(vc_free, (uint32_t)((j - 1) & 1), p.flags)) break;
+      convert_tile<D, true>(v8, vc, t, zero_from, bad);  // f16, like P
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(vc_full);
+        mbar_arrive(&kv_empty[st]);  // the E4M3 stage may be refilled
+      }
+    }
   } else if (warp == kMmaWarp) {
     // ----------------------------------------------------------------- MMA
-    const uint32_t id_s = idesc_bf16(kRows, kKeys, 0);
-    const uint32_t id_o = idesc_bf16(kRows, D, 1);
+    const uint32_t id_s = idesc_f16kind(kRows, kKeys, 0, true);
+    // E4M3: P (scaled by the V scales) and V are f16 for the PV product
+    const uint32_t id_o = idesc_f16kind(kRows, D, 1, !kFp8);
     const uint32_t q_addr = smem_u32(sq);
     bool ok = mbar_wait(q_full, 0, p.flags);
     auto issue_pv = [&](int i) -> bool {
       const int st = i % kStages;
       if (!mbar_wait(p_full, (uint32_t)(i & 1), p.flags)) return false;
-      tc_fence_after();
-      // zero V rows that must not contribute (past the end, or a rejected page)
-      const int32_t key0 = i * kKeys;
-      const int bad = stage_bad[st];
-      int zlo = kKeys;  // first row to zero (tail)
-      if (key0 + kKeys > L) zlo = max(0, L - key0);
-      if (zlo < kKeys || bad) {
-        uint8_t* vd = skv + st * Sm::kStageB + Sm::kTileB;
-        for (int idx = lane; idx < kKeys * Sm::kHalves * 8; idx += 32) {
-          const int row = idx / (Sm::kHalves * 8);
-          const int rem = idx - row * (Sm::kHalves * 8);
-          const int h = rem >> 3, c = rem & 7;
-          const bool z = row >= zlo || ((bad >> (row >> 6)) & 1);
-          if (z)
-            *reinterpret_cast<uint4*>(vd + h * Sm::kHalfB + row * 128 + c * 16) =
-                make_uint4(0, 0, 0, 0);
+      uint32_t v_addr;
+      if constexpr (kFp8) {
+        if (!mbar_wait(vc_full, (uint32_t)(i & 1), p.flags)) return false;
+        v_addr = smem_u32(sconv) + Sm::kTileB;
+      } else {
+        // zero V rows that must not contribute (past the end, or a rejected page)
+        const int32_t key0 = i * kKeys;
+        const int bad = facts[i % kFactsRing].bad;
+        int zlo = kKeys;
+        if (key0 + kKeys > L) zlo = max(0, L - key0);
+        if (zlo < kKeys || bad) {
+          uint8_t* vd = skv + st * Sm::kStageB + Sm::kTileB;
+          for (int idx = lane; idx < kKeys * Sm::kHalves * 8; idx += 32) {
+            const int row = idx / (Sm::kHalves * 8);
+            const int rem = idx - row * (Sm::kHalves * 8);
+            const int h = rem >> 3, c = rem & 7;
+            const bool z = row >= zlo || ((bad >> (row >> 6)) & 1);
+            if (z)
+              *reinterpret_cast<uint4*>(vd + h * Sm::kHalfB + row * 128 + c * 16) =
+                  make_uint4(0, 0, 0, 0);
+          }
+          fence_async_smem();
+          __syncwarp();
         }
-        fence_async_smem();
-        __syncwarp();
+        v_addr = smem_u32(skv + st * Sm::kStageB + Sm::kTileB);
       }
+      tc_fence_after();
       if (lane == 0) {
-        const uint32_t v_addr = smem_u32(skv + st * Sm::kStageB + Sm::kTileB);
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk) {
           // B = V [keys x d], MN-major: 8-key groups 1024 B apart (SBO), the
@@ -346,7 +488,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts(tmem + kColO, tmem + kColP + kk * 8, bd, id_o, (i > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(o_bar);
-        tc_commit(&kv_empty[st]);
+        if constexpr (kFp8)
+          tc_commit(vc_free);
+        else
+          tc_commit(&kv_empty[st]);
       }
       __syncwarp();
       return true;
@@ -354,14 +499,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = 0; j < n_kv && ok; ++j) {
       const int st = j % kStages;
       const int sb = j & 1;
-      if (!mbar_wait(&kv_full[st], (uint32_t)((j / kStages) & 1), p.flags)) { ok = false; break; }
+      uint32_t k_addr;
+      if constexpr (kFp8) {
+        if (!mbar_wait(kc_full, (uint32_t)(j & 1), p.flags)) { ok = false; break; }
+        k_addr = smem_u32(sconv);
+      } else {
+        if (!mbar_wait(&kv_full[st], (uint32_t)((j / kStages) & 1), p.flags)) { ok = false; break; }
+        k_addr = smem_u32(skv + st * Sm::kStageB);
+      }
       if (j >= 2 && !mbar_wait(&s_free[sb], (uint32_t)((j / 2 - 1) & 1), p.flags)) {
         ok = false;
         break;
       }
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t k_addr = smem_u32(skv + st * Sm::kStageB);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           // A = Q, B = K, both K-major: 16-element K steps advance 32 B inside
@@ -372,16 +523,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ss(tmem + (sb ? kColS1 : kColS0), ad, bd, id_s, kk > 0 ? 1u : 0u);
         }
         tc_commit(&s_full[sb]);
+        if constexpr (kFp8) tc_commit(kc_free);
       }
       __syncwarp();
       if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
     }
     if (ok && n_kv > 0) ok = issue_pv(n_kv - 1);
-    if (!ok) *s_abort = 1;
     // every MMA this thread issued must finish before TMEM is released
     if (lane == 0) tc_commit(done_bar);
     __syncwarp();
-  } else {
+  } else if (warp < 4) {
     // ------------------------------------------------------------- softmax
     const int r = threadIdx.x;  // row = TMEM lane
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
@@ -392,10 +543,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
       const int sb = j & 1;
-      const int st = j % kStages;
       if (!mbar_wait(&s_full[sb], (uint32_t)((j / 2) & 1), p.flags)) { ok = false; break; }
-      if (!mbar_wait(&kv_full[st], (uint32_t)((j / kStages) & 1), p.flags)) { ok = false; break; }
-      const int bad = stage_bad[st];
+      if (!mbar_wait(&facts_full[j % kFactsRing], (uint32_t)((j / kFactsRing) & 1), p.flags)) {
+        ok = false;
+        break;
+      }
+      const TileFacts tf = facts[j % kFactsRing];
       tc_fence_after();
       float s[kKeys];
 #pragma unroll
@@ -406,18 +559,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[sb]);
       // mask: causal diagonal (which also covers keys past the end) and
-      // sub-blocks of a rejected page
+      // blocks of a rejected page; E4M3 K scales per 64-key block
       const int32_t key0 = j * kKeys;
       const bool diag = key0 + kKeys - 1 > p_min;
+      const float mul0 = kFp8 ? p.scale_log2 * tf.ks[0] : p.scale_log2;
+      const float mul1 = kFp8 ? p.scale_log2 * tf.ks[1] : p.scale_log2;
       float mt = -INFINITY;
 #pragma unroll
       for (int c = 0; c < kKeys; ++c) {
         const int32_t key = key0 + c;
-        const bool keep = (!diag || key <= pos) && !((bad >> (c >> 6)) & 1);
-        s[c] = keep ? s[c] * p.scale_log2 : -INFINITY;
+        const bool keep = (!diag || key <= pos) && !((tf.bad >> (c >> 6)) & 1);
+        s[c] = keep ? s[c] * (c < 64 ? mul0 : mul1) : -INFINITY;
         mt = fmaxf(mt, s[c]);
       }
-      const bool need = mt > m_ref + 8.f;  // also true on the first visible tile
+      // The reference max is raised lazily (p <= 2^8) for bf16; for E4M3 at
+      // every increase, so that p * v_scale <= 2^15 fits the f16 P.
+      const bool need = mt > m_ref + (kFp8 ? 0.f : 8.f);  // also true on the first visible tile
       // PV of the previous tile must be done before P is overwritten or O rescaled
       if (j >= 1 && !mbar_wait(o_bar, (uint32_t)((j - 1) & 1), p.flags)) { ok = false; break; }
       tc_fence_after();
@@ -440,6 +597,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       m_ref = m_new;
       // a row with no visible key yet keeps m_ref = -inf: its p must be 0
       const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+      const float pv0 = kFp8 ? tf.vs[0] : 1.f;  // E4M3 V scales ride on P
+      const float pv1 = kFp8 ? tf.vs[1] : 1.f;
       uint32_t pk[kKeys / 2];
       float rs = 0.f;
 #pragma unroll
@@ -447,7 +606,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float p0 = fast_exp2(s[c] - m_use);
         const float p1 = fast_exp2(s[c + 1] - m_use);
         rs += p0 + p1;
-        pk[c / 2] = pack_bf16(p0, p1);
+        if constexpr (kFp8) {
+          const float vsc = c < 64 ? pv0 : pv1;
+          pk[c / 2] = pack_f16(p0 * vsc, p1 * vsc);
+        } else {
+          pk[c / 2] = pack_bf16(p0, p1);
+        }
       }
       l += rs;
 #pragma unroll
@@ -502,24 +666,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D>
+template <int D, bool kFp8>
 size_t smem_bytes() {
-  return 1024 + Smem<D>::kBytes + 16 * sizeof(uint64_t) + 16 * sizeof(int32_t);
+  return 1024 + Smem<D, kFp8>::kBytes + (16 + kFactsRing) * sizeof(uint64_t) +
+         kFactsRing * sizeof(TileFacts) + 16;
 }
 
-template <int D>
+template <int D, bool kFp8>
 cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const Params& p, int q_tiles, cudaStream_t stream) {
-  const size_t smem = smem_bytes<D>();
+  const size_t smem = smem_bytes<D, kFp8>();
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D>,
+    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, kFp8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
   dim3 grid(q_tiles, p.num_kv_heads, p.num_chunks);
-  prefill_kernel<D><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
+  prefill_kernel<D, kFp8><<<grid, Smem<D, kFp8>::kThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
@@ -544,14 +709,18 @@ int prefill_entry(const pkv_cache* cache, const void* q, int32_t num_q_heads, in
   if (!q || !cu_q_lens || !page_table || !seq_lens || !out) return PKV_ERR_NULL;
   if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(out) & 15))
     return PKV_ERR_ALIGN;
-  if (cache->kv_dtype != PKV_KV_BF16) return PKV_ERR_UNSUPPORTED;
+  const bool fp8 = cache->kv_dtype == PKV_KV_FP8_E4M3;
   const int D = cache->head_dim;
   CUtensorMap tq, tk, tv;
   if ((st = encode_q_map(&tq, q, total_q, num_q_heads, D, gqa_group))) return st;
   const int64_t rows = (int64_t)cache->num_pages * cache->num_kv_heads * cache->page_size;
-  if ((st = encode_pool_map(&tk, cache->k_pool, false, rows, D, 64, 64))) return st;
-  if ((st = encode_pool_map(&tv, cache->v_pool, false, rows, D, 64, 64))) return st;
+  // bf16 pools: 64-column boxes; E4M3 pools: one box of the whole D-byte row
+  const int box_cols = fp8 ? D : 64;
+  if ((st = encode_pool_map(&tk, cache->k_pool, fp8, rows, D, box_cols, 64))) return st;
+  if ((st = encode_pool_map(&tv, cache->v_pool, fp8, rows, D, box_cols, 64))) return st;
   pf::Params p;
+  p.k_scale = cache->k_scale;
+  p.v_scale = cache->v_scale;
   p.cu_q = cu_q_lens;
   p.page_table = page_table;
   p.seq_lens = seq_lens;
@@ -568,8 +737,13 @@ int prefill_entry(const pkv_cache* cache, const void* q, int32_t num_q_heads, in
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   const int tq_tokens = pf::kRows / gqa_group;
   const int q_tiles = (max_q_len + tq_tokens - 1) / tq_tokens;
-  cudaError_t e = D == 128 ? pf::launch<128>(tq, tk, tv, p, q_tiles, stream)
-                           : pf::launch<64>(tq, tk, tv, p, q_tiles, stream);
+  cudaError_t e;
+  if (D == 128)
+    e = fp8 ? pf::launch<128, true>(tq, tk, tv, p, q_tiles, stream)
+            : pf::launch<128, false>(tq, tk, tv, p, q_tiles, stream);
+  else
+    e = fp8 ? pf::launch<64, true>(tq, tk, tv, p, q_tiles, stream)
+            : pf::launch<64, false>(tq, tk, tv, p, q_tiles, stream);
   return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 

@@ -2,9 +2,10 @@
 
 Causal chunk attention (query i of a chunk with n queries over L tokens sees
 keys 0..L-n+i): bf16 output within max-abs 1e-2 and mean-abs 1e-3 of the
-fp64 oracle, lse within 2e-3.  Cases cover GQA groups 1..8, head_dim 64/128,
-page sizes 64/128, chunks without context, chunks shorter than a Q tile,
-ragged tails and the in-flight mixed-batch configuration.
+fp64 oracle, lse within 2e-3.  Cases cover bf16 and E4M3 pools (the oracle
+attends over its own bit-identical E4M3 pool), GQA groups 1..8, head_dim
+64/128, page sizes 64/128, chunks without context, chunks shorter than a Q
+tile, ragged tails and the in-flight mixed-batch configuration.
 """
 import numpy as np
 import pytest
@@ -25,21 +26,25 @@ def _oracle_prefill(w):
 
 
 CASES = [
-    # (P, D, Hkv, G, ctx lengths of the chunks, new tokens per chunk)
-    (64, 128, 2, 4, [0, 100, 700], [512, 33, 130]),
-    (64, 128, 1, 8, [5, 0], [17, 1]),
-    (128, 128, 2, 1, [0, 129, 1000], [128, 200, 7]),
-    (64, 64, 2, 2, [63, 64, 0], [65, 1, 300]),
-    (128, 64, 1, 4, [300], [257]),
-    (64, 128, 8, 4, [2048, 0, 777, 1500], [512, 512, 512, 512]),
+    # (kv dtype, P, D, Hkv, G, ctx lengths of the chunks, new tokens per chunk)
+    ("bf16", 64, 128, 2, 4, [0, 100, 700], [512, 33, 130]),
+    ("bf16", 64, 128, 1, 8, [5, 0], [17, 1]),
+    ("bf16", 128, 128, 2, 1, [0, 129, 1000], [128, 200, 7]),
+    ("bf16", 64, 64, 2, 2, [63, 64, 0], [65, 1, 300]),
+    ("bf16", 128, 64, 1, 4, [300], [257]),
+    ("bf16", 64, 128, 8, 4, [2048, 0, 777, 1500], [512, 512, 512, 512]),
+    ("e4m3", 64, 128, 2, 4, [0, 100, 700], [512, 33, 130]),
+    ("e4m3", 128, 128, 1, 8, [5, 0, 300], [17, 1, 129]),
+    ("e4m3", 64, 64, 2, 2, [63, 64, 0], [65, 1, 300]),
+    ("e4m3", 128, 64, 2, 1, [1000], [200]),
 ]
 
 
-@pytest.mark.parametrize("case", CASES, ids=lambda c: f"P{c[0]}-D{c[1]}-G{c[3]}")
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"{c[0]}-P{c[1]}-D{c[2]}-G{c[4]}")
 def test_prefill_matches_oracle(case):
-    P, D, Hkv, G, ctx, new = case
+    dtype, P, D, Hkv, G, ctx, new = case
     w = workloads.build("pf", 21, ctx, new, page_size=P, num_q_heads=Hkv * G, num_kv_heads=Hkv,
-                        head_dim=D, pool_slack=0.3, chunk_rows=range(len(ctx)))
+                        head_dim=D, kv_dtype=dtype, pool_slack=0.3, chunk_rows=range(len(ctx)))
     st = GpuState(w)
     st.append_step()
     out, lse = st.prefill()
@@ -100,6 +105,24 @@ def test_prefill_bad_page_is_masked_and_flagged():
     st.append_step()
     q, cu, table, lens, max_q = st.chunk_inputs()
     table[0, 1] = w.num_pages + 3
+    out, lse = st.pkv.paged_prefill_chunk_attention(st.cache, q, cu, table, lens, max_q,
+                                                    w.softmax_scale)
+    torch.cuda.synchronize()
+    assert int(st.flags.item()) & 0x1
+    assert torch.all(torch.isfinite(out.float()))
+    ref, ref_lse = _oracle_prefill(w)
+    rows = np.arange(int(cu[1].item()), int(cu[2].item()))
+    compare(out, lse, ref, ref_lse, rows=rows)
+
+
+def test_prefill_e4m3_bad_page_is_masked_and_flagged():
+    w = workloads.build("pfbad8", 25, [200, 64], [40, 64], page_size=64, num_q_heads=8,
+                        num_kv_heads=2, head_dim=128, kv_dtype="e4m3", pool_slack=0.5,
+                        chunk_rows=[0, 1])
+    st = GpuState(w)
+    st.append_step()
+    q, cu, table, lens, max_q = st.chunk_inputs()
+    table[0, 1] = -1
     out, lse = st.pkv.paged_prefill_chunk_attention(st.cache, q, cu, table, lens, max_q,
                                                     w.softmax_scale)
     torch.cuda.synchronize()
