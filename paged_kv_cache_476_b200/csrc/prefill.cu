@@ -38,16 +38,19 @@ namespace pkv {
 
 namespace pf {
 
-constexpr int kRows = 128;     // M of the Q tile
+constexpr int kRows = 128;     // M of a Q tile; a CTA holds two Q tiles, A and B
 constexpr int kKeys = 128;     // N of the S tile (keys per KV tile)
 constexpr int kStages = 2;     // K/V ring depth
-// warps 0-3 softmax (one TMEM lane = one row per thread), 4 producer, 5 MMA,
-// 6-7 E4M3 -> bf16 converters (E4M3 pools only)
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kConvWarp0 = 6;
+// warps 0-3 softmax of Q tile A, 4-7 softmax of Q tile B (one TMEM lane =
+// one row per thread), 8 producer, 9 MMA, 10-11 E4M3 converters (E4M3 only)
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kConvWarp0 = 10;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP = 384;
+// TMEM columns: S of tile A and B (P is written over S as 16-bit pairs), O
+// of tile A and B.
+__device__ __forceinline__ uint32_t col_s(int x) { return x ? 128u : 0u; }
+__device__ __forceinline__ uint32_t col_o(int x) { return x ? 384u : 256u; }
 
 struct Params {
   const float* k_scale;  // [pages][Hkv] (E4M3 pools)
@@ -183,14 +186,14 @@ __host__ __device__ constexpr uint32_t idesc_f16kind(int M, int N, int b_mn_majo
 template <int D, bool kFp8>
 struct Smem {
   static constexpr int kHalves = D / 64;            // 128-byte column boxes per bf16 row
-  static constexpr int kQB = kRows * D * 2;         // Q tile
+  static constexpr int kQB = kRows * D * 2;         // one Q tile
   static constexpr int kTileB = kKeys * D * 2;      // bf16 K (or V) tile
   static constexpr int kHalfB = kKeys * 128;        // one 64-column half of a bf16 tile
   static constexpr int kTile8B = kKeys * D;         // E4M3 K (or V) tile as it lands
   static constexpr int kStageB = kFp8 ? 2 * kTile8B : 2 * kTileB;
   static constexpr int kConvB = kFp8 ? 2 * kTileB : 0;  // converted K, then V
-  static constexpr int kBytes = kQB + kStages * kStageB + kConvB;
-  static constexpr int kThreads = kFp8 ? 256 : 192;  // + two converter warps
+  static constexpr int kBytes = 2 * kQB + kStages * kStageB + kConvB;
+  static constexpr int kThreads = kFp8 ? 384 : 320;  // + two converter warps
 };
 
 // Per-KV-tile facts the producer passes on: rejected 64-key blocks and the
@@ -273,18 +276,17 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sq = smem;
-  uint8_t* skv = smem + Sm::kQB;                    // stage s: K at s*kStageB, V after it
-  uint8_t* sconv = skv + kStages * Sm::kStageB;     // E4M3 only: bf16 K, then bf16 V
+  uint8_t* sq = smem;                               // Q tile A, then Q tile B
+  uint8_t* skv = smem + 2 * Sm::kQB;                // stage s: K at s*kStageB, V after it
+  uint8_t* sconv = skv + kStages * Sm::kStageB;     // E4M3 only: 16-bit K, then V
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sm::kBytes);
   uint64_t* q_full = bars + 0;
   uint64_t* kv_full = bars + 1;               // [kStages] TMA landed
   uint64_t* kv_empty = kv_full + kStages;     // [kStages] stage may be refilled
-  uint64_t* s_full = kv_empty + kStages;      // [2]
-  uint64_t* s_free = s_full + 2;              // [2]
-  uint64_t* p_full = s_free + 2;
-  uint64_t* o_bar = p_full + 1;
-  uint64_t* done_bar = o_bar + 1;
+  uint64_t* s_full = kv_empty + kStages;      // [2] S of tile A / B computed
+  uint64_t* p_full = s_full + 2;              // [2] P of tile A / B written
+  uint64_t* o_bar = p_full + 2;               // [2] PV of tile A / B done
+  uint64_t* done_bar = o_bar + 2;
   uint64_t* kc_full = done_bar + 1;           // E4M3: converted K ready / free
   uint64_t* kc_free = kc_full + 1;
   uint64_t* vc_full = kc_free + 1;            // E4M3: converted V ready / free
@@ -296,25 +298,30 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int G = p.group;
-  const int TQ = kRows / G;  // query tokens per tile
+  const int TQ = kRows / G;  // query tokens per Q tile
   const int chunk = blockIdx.z;
   const int g = blockIdx.y;
-  const int qt0 = blockIdx.x * TQ;
+  const int qa0 = blockIdx.x * 2 * TQ;  // first token of tile A; tile B follows
 
   const int32_t q_begin = __ldg(p.cu_q + chunk);
   const int32_t n = __ldg(p.cu_q + chunk + 1) - q_begin;
   int32_t L = __ldg(p.seq_lens + chunk);
-  if (n <= 0 || qt0 >= n) return;  // uniform across the CTA
+  if (n <= 0 || qa0 >= n) return;  // uniform across the CTA
   const int32_t cap = p.max_pages * p.page_size;
   if (L > cap || n > L) {
     if (threadIdx.x == 0) flag_error(p.flags, PKV_FLAG_BAD_LENGTH);
     if (n > cap || L < n) return;  // nothing meaningful to compute
     L = min(L, cap);
   }
-  const int tq_end = min(qt0 + TQ, n);                 // exclusive token bound of this tile
-  const int32_t p_max = L - n + tq_end - 1;            // largest query position
-  const int32_t p_min = L - n + qt0;                   // smallest query position
-  const int n_kv = (p_max + kKeys) / kKeys;            // KV tiles to visit
+  const int q0[2] = {qa0, qa0 + TQ};
+  const bool hasB = q0[1] < n;
+  int nkv[2];
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    const int32_t pmax = L - n + min(q0[x] + TQ, n) - 1;  // largest query position
+    nkv[x] = (x == 0 || hasB) ? (pmax + kKeys) / kKeys : 0;
+  }
+  const int n_kv = max(nkv[0], nkv[1]);  // KV tiles the CTA visits
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -322,12 +329,11 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], kFp8 ? 2 : 1);  // E4M3: released by the two converter warps
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&s_free[s], 4);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&s_full[x], 1);
+      mbar_init(&p_full[x], 4);
+      mbar_init(&o_bar[x], 1);
     }
-    mbar_init(p_full, 4);
-    mbar_init(o_bar, 1);
     mbar_init(done_bar, 1);
     mbar_init(kc_full, 2);
     mbar_init(kc_free, 1);
@@ -348,10 +354,15 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
       tma_prefetch_desc(&tmap_q);
       tma_prefetch_desc(&tmap_k);
       tma_prefetch_desc(&tmap_v);
-      mbar_arrive_expect_tx(q_full, (uint32_t)Sm::kQB);
+      mbar_arrive_expect_tx(q_full, (uint32_t)(hasB ? 2 : 1) * Sm::kQB);
 #pragma unroll
-      for (int h = 0; h < Sm::kHalves; ++h)
-        tma_load_3d(sq + h * (kRows * 128), &tmap_q, h * 64, g * G, q_begin + qt0, q_full);
+      for (int x = 0; x < 2; ++x) {
+        if (x == 1 && !hasB) break;
+#pragma unroll
+        for (int h = 0; h < Sm::kHalves; ++h)
+          tma_load_3d(sq + x * Sm::kQB + h * (kRows * 128), &tmap_q, h * 64, g * G,
+                      q_begin + q0[x], q_full);
+      }
     }
     const uint64_t pol = policy_evict_first();
     for (int j = 0; j < n_kv; ++j) {
@@ -416,7 +427,7 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
       __syncwarp();
     }
   } else if (kFp8 && warp >= kConvWarp0) {
-    // ------------------------------------------------- E4M3 -> bf16 converters
+    // ------------------------------------------------- E4M3 -> 16-bit converters
     const int t = threadIdx.x - kConvWarp0 * 32;  // 0..63
     const uint32_t kc = smem_u32(sconv), vc = kc + Sm::kTileB;
     for (int j = 0; j < n_kv; ++j) {
@@ -444,26 +455,52 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ----------------------------------------------------------------- MMA
+    // Issue order per KV tile j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so the
+    // tensor core always has the other tile's work while a softmax runs.
     const uint32_t id_s = idesc_f16kind(kRows, kKeys, 0, true);
     // E4M3: P (scaled by the V scales) and V are f16 for the PV product
     const uint32_t id_o = idesc_f16kind(kRows, D, 1, !kFp8);
     const uint32_t q_addr = smem_u32(sq);
     bool ok = mbar_wait(q_full, 0, p.flags);
-    auto issue_pv = [&](int i) -> bool {
-      const int st = i % kStages;
-      if (!mbar_wait(p_full, (uint32_t)(i & 1), p.flags)) return false;
-      uint32_t v_addr;
+    auto k_ready = [&](int j, uint32_t* addr) -> bool {
       if constexpr (kFp8) {
-        if (!mbar_wait(vc_full, (uint32_t)(i & 1), p.flags)) return false;
-        v_addr = smem_u32(sconv) + Sm::kTileB;
+        *addr = smem_u32(sconv);
+        return mbar_wait(kc_full, (uint32_t)(j & 1), p.flags);
       } else {
-        // zero V rows that must not contribute (past the end, or a rejected page)
-        const int32_t key0 = i * kKeys;
-        const int bad = facts[i % kFactsRing].bad;
+        *addr = smem_u32(skv + (j % kStages) * Sm::kStageB);
+        return mbar_wait(&kv_full[j % kStages], (uint32_t)((j / kStages) & 1), p.flags);
+      }
+    };
+    auto issue_s = [&](int x, uint32_t k_addr) {
+      tc_fence_after();
+      if (lane == 0) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          // A = Q, B = K, both K-major: 16-element K steps advance 32 B inside
+          // a 128-byte swizzled row; the second 64 columns live kHalfB away.
+          const int h = kk >> 2, w = kk & 3;
+          const uint64_t ad = sdesc(q_addr + x * Sm::kQB + h * (kRows * 128) + w * 32, 16, 1024);
+          const uint64_t bd = sdesc(k_addr + h * Sm::kHalfB + w * 32, 16, 1024);
+          mma_ss(tmem + col_s(x), ad, bd, id_s, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&s_full[x]);
+      }
+      __syncwarp();
+    };
+    // V of tile j, made safe for the PV product (rows past the end or of a
+    // rejected page zeroed); returns false on a timeout
+    auto v_ready = [&](int j, uint32_t* addr) -> bool {
+      if constexpr (kFp8) {
+        *addr = smem_u32(sconv) + Sm::kTileB;
+        return mbar_wait(vc_full, (uint32_t)(j & 1), p.flags);
+      } else {
+        const int st = j % kStages;
+        const int32_t key0 = j * kKeys;
+        const int bad = facts[j % kFactsRing].bad;
         int zlo = kKeys;
         if (key0 + kKeys > L) zlo = max(0, L - key0);
+        uint8_t* vd = skv + st * Sm::kStageB + Sm::kTileB;
         if (zlo < kKeys || bad) {
-          uint8_t* vd = skv + st * Sm::kStageB + Sm::kTileB;
           for (int idx = lane; idx < kKeys * Sm::kHalves * 8; idx += 32) {
             const int row = idx / (Sm::kHalves * 8);
             const int rem = idx - row * (Sm::kHalves * 8);
@@ -476,178 +513,212 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
           fence_async_smem();
           __syncwarp();
         }
-        v_addr = smem_u32(skv + st * Sm::kStageB + Sm::kTileB);
+        *addr = smem_u32(vd);
+        return true;
       }
+    };
+    auto issue_pv = [&](int x, int j, uint32_t v_addr) -> bool {
+      if (!mbar_wait(&p_full[x], (uint32_t)(j & 1), p.flags)) return false;
       tc_fence_after();
       if (lane == 0) {
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk) {
           // B = V [keys x d], MN-major: 8-key groups 1024 B apart (SBO), the
-          // 64-column halves kHalfB apart (LBO).
+          // 64-column halves kHalfB apart (LBO).  A = P, 16-bit pairs in TMEM.
           const uint64_t bd = sdesc(v_addr + kk * 2048, Sm::kHalfB, 1024);
-          mma_ts(tmem + kColO, tmem + kColP + kk * 8, bd, id_o, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + col_o(x), tmem + col_s(x) + kk * 8, bd, id_o,
+                 (j > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(o_bar);
-        if constexpr (kFp8)
-          tc_commit(vc_free);
-        else
-          tc_commit(&kv_empty[st]);
+        tc_commit(&o_bar[x]);
       }
       __syncwarp();
       return true;
     };
+    uint32_t k_addr = 0;
+    if (ok) ok = k_ready(0, &k_addr);
+    if (ok) {
+      issue_s(0, k_addr);
+      if (hasB) issue_s(1, k_addr);
+      if (kFp8 && lane == 0) tc_commit(kc_free);  // K_0 is read by both S products
+      __syncwarp();
+    }
     for (int j = 0; j < n_kv && ok; ++j) {
-      const int st = j % kStages;
-      const int sb = j & 1;
-      uint32_t k_addr;
-      if constexpr (kFp8) {
-        if (!mbar_wait(kc_full, (uint32_t)(j & 1), p.flags)) { ok = false; break; }
-        k_addr = smem_u32(sconv);
-      } else {
-        if (!mbar_wait(&kv_full[st], (uint32_t)((j / kStages) & 1), p.flags)) { ok = false; break; }
-        k_addr = smem_u32(skv + st * Sm::kStageB);
-      }
-      if (j >= 2 && !mbar_wait(&s_free[sb], (uint32_t)((j / 2 - 1) & 1), p.flags)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
+      uint32_t v_addr;
+      if (!(ok = v_ready(j, &v_addr))) break;
+      if (j < nkv[0] && !(ok = issue_pv(0, j, v_addr))) break;
+      const bool next = j + 1 < n_kv;
+      if (next && !(ok = k_ready(j + 1, &k_addr))) break;
+      if (j + 1 < nkv[0]) issue_s(0, k_addr);
+      if (j < nkv[1] && !(ok = issue_pv(1, j, v_addr))) break;
       if (lane == 0) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          // A = Q, B = K, both K-major: 16-element K steps advance 32 B inside
-          // a 128-byte swizzled row; the second 64 columns live kHalfB away.
-          const int h = kk >> 2, w = kk & 3;
-          const uint64_t ad = sdesc(q_addr + h * (kRows * 128) + w * 32, 16, 1024);
-          const uint64_t bd = sdesc(k_addr + h * Sm::kHalfB + w * 32, 16, 1024);
-          mma_ss(tmem + (sb ? kColS1 : kColS0), ad, bd, id_s, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&s_full[sb]);
-        if constexpr (kFp8) tc_commit(kc_free);
+        // this KV tile is consumed once both PV products have run
+        if constexpr (kFp8)
+          tc_commit(vc_free);
+        else
+          tc_commit(&kv_empty[j % kStages]);
       }
       __syncwarp();
-      if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+      if (j + 1 < nkv[1]) issue_s(1, k_addr);
+      if (kFp8 && next && lane == 0) tc_commit(kc_free);  // K_{j+1} consumed
+      __syncwarp();
     }
-    if (ok && n_kv > 0) ok = issue_pv(n_kv - 1);
     // every MMA this thread issued must finish before TMEM is released
     if (lane == 0) tc_commit(done_bar);
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------- softmax
-    const int r = threadIdx.x;  // row = TMEM lane
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const int t_local = qt0 + r / G;
-    const bool row_ok = t_local < n;
-    const int32_t pos = row_ok ? L - n + t_local : p_max;
-    float m_ref = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      const int sb = j & 1;
-      if (!mbar_wait(&s_full[sb], (uint32_t)((j / 2) & 1), p.flags)) { ok = false; break; }
-      if (!mbar_wait(&facts_full[j % kFactsRing], (uint32_t)((j / kFactsRing) & 1), p.flags)) {
-        ok = false;
-        break;
-      }
-      const TileFacts tf = facts[j % kFactsRing];
-      tc_fence_after();
-      float s[kKeys];
+    const int x = warp >> 2;        // Q tile: 0 = A, 1 = B
+    const int wq = warp & 3;        // TMEM lane quadrant of this warp
+    if (x == 0 || hasB) {
+      const int r = wq * 32 + lane;  // row of the tile = TMEM lane
+      const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+      const uint32_t colS = col_s(x), colO = col_o(x);
+      const int t_local = q0[x] + r / G;
+      const bool row_ok = t_local < n;
+      const int32_t p_min = L - n + q0[x];
+      const int32_t pos = row_ok ? L - n + t_local : L - n + min(q0[x] + TQ, n) - 1;
+      float m_ref = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < nkv[x]; ++j) {
+        if (!mbar_wait(&s_full[x], (uint32_t)(j & 1), p.flags)) { ok = false; break; }
+        if (!mbar_wait(&facts_full[j % kFactsRing], (uint32_t)((j / kFactsRing) & 1), p.flags)) {
+          ok = false;
+          break;
+        }
+        const TileFacts tf = facts[j % kFactsRing];
+        tc_fence_after();
+        // mask: causal diagonal (which also covers keys past the end) and
+        // blocks of a rejected page; E4M3 K scales per 64-key block
+        const int32_t key0 = j * kKeys;
+        const bool diag = key0 + kKeys - 1 > p_min;
+        const float mul0 = kFp8 ? p.scale_log2 * tf.ks[0] : p.scale_log2;
+        const float mul1 = kFp8 ? p.scale_log2 * tf.ks[1] : p.scale_log2;
+        auto scaled = [&](float v, int c) -> float {
+          const bool keep = (!diag || key0 + c <= pos) && !((tf.bad >> (c >> 6)) & 1);
+          return keep ? v * (c < 64 ? mul0 : mul1) : -INFINITY;
+        };
+        // Tiles off the diagonal without a rejected page (nearly all) take a
+        // lean path: max of the raw scores, then one FMA + ex2 per element.
+        const bool plain = !diag && tf.bad == 0;
+        // pass 1: row max of the scaled, masked scores (64 columns per load)
+        float mt = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < kKeys; c += 32)
-        tmem_ld32(tmem + lane_base + (sb ? kColS1 : kColS0) + c, s + c);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[sb]);
-      // mask: causal diagonal (which also covers keys past the end) and
-      // blocks of a rejected page; E4M3 K scales per 64-key block
-      const int32_t key0 = j * kKeys;
-      const bool diag = key0 + kKeys - 1 > p_min;
-      const float mul0 = kFp8 ? p.scale_log2 * tf.ks[0] : p.scale_log2;
-      const float mul1 = kFp8 ? p.scale_log2 * tf.ks[1] : p.scale_log2;
-      float mt = -INFINITY;
+        for (int cb = 0; cb < kKeys; cb += 64) {
+          float sv[64];
+          tmem_ld32(tmem + lane_base + colS + cb, sv);
+          tmem_ld32(tmem + lane_base + colS + cb + 32, sv + 32);
+          tmem_wait_ld();
+          if (plain) {
+            float m = sv[0];
 #pragma unroll
-      for (int c = 0; c < kKeys; ++c) {
-        const int32_t key = key0 + c;
-        const bool keep = (!diag || key <= pos) && !((tf.bad >> (c >> 6)) & 1);
-        s[c] = keep ? s[c] * (c < 64 ? mul0 : mul1) : -INFINITY;
-        mt = fmaxf(mt, s[c]);
+            for (int i = 1; i < 64; ++i) m = fmaxf(m, sv[i]);
+            mt = fmaxf(mt, m * (cb < 64 ? mul0 : mul1));  // the multipliers are > 0
+          } else {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) mt = fmaxf(mt, scaled(sv[i], cb + i));
+          }
+        }
+        // The reference max is raised lazily (p <= 2^8) for bf16; for E4M3 at
+        // every increase, so that p * v_scale <= 2^15 fits the f16 P.
+        const bool need = mt > m_ref + (kFp8 ? 0.f : 8.f);  // true on the first visible tile
+        const float m_new = need ? mt : m_ref;
+        // S(j) done implies every earlier MMA is done, PV(j-1) included: O is
+        // stable and the P columns are free.
+        if (j >= 1 && __any_sync(0xffffffffu, need)) {
+          const float alpha = need ? fast_exp2(m_ref - m_new) : 1.f;
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {
+            float o[32];
+            tmem_ld32(tmem + lane_base + colO + c, o);
+            tmem_wait_ld();
+            uint32_t u[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(o[i] * alpha);
+            tmem_st16(tmem + lane_base + colO + c, u);
+            tmem_st16(tmem + lane_base + colO + c + 16, u + 16);
+          }
+          l *= alpha;
+        }
+        m_ref = m_new;
+        // a row with no visible key yet keeps m_ref = -inf: its p must be 0
+        const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+        const float pv0 = kFp8 ? tf.vs[0] : 1.f;  // E4M3 V scales ride on P
+        const float pv1 = kFp8 ? tf.vs[1] : 1.f;
+        // pass 2: P over S's own columns (16-bit pairs: P column c/2 lies in
+        // an S column already read)
+        float rs = 0.f;
+#pragma unroll
+        for (int cb = 0; cb < kKeys; cb += 64) {
+          float sv[64];
+          tmem_ld32(tmem + lane_base + colS + cb, sv);
+          tmem_ld32(tmem + lane_base + colS + cb + 32, sv + 32);
+          tmem_wait_ld();
+          const float mul = cb < 64 ? mul0 : mul1;
+          const float vsc = cb < 64 ? pv0 : pv1;
+          uint32_t pk[32];
+          // (two loops rather than a branch per element, which the compiler
+          // would turn into both paths under predicates)
+          if (plain) {
+#pragma unroll
+            for (int i = 0; i < 64; i += 2) {
+              const float p0 = fast_exp2(fmaf(sv[i], mul, -m_use));
+              const float p1 = fast_exp2(fmaf(sv[i + 1], mul, -m_use));
+              rs += p0 + p1;
+              if constexpr (kFp8)
+                pk[i / 2] = pack_f16(p0 * vsc, p1 * vsc);
+              else
+                pk[i / 2] = pack_bf16(p0, p1);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 64; i += 2) {
+              const float p0 = fast_exp2(scaled(sv[i], cb + i) - m_use);
+              const float p1 = fast_exp2(scaled(sv[i + 1], cb + i + 1) - m_use);
+              rs += p0 + p1;
+              if constexpr (kFp8)
+                pk[i / 2] = pack_f16(p0 * vsc, p1 * vsc);
+              else
+                pk[i / 2] = pack_bf16(p0, p1);
+            }
+          }
+          tmem_st16(tmem + lane_base + colS + cb / 2, pk);
+          tmem_st16(tmem + lane_base + colS + cb / 2 + 16, pk + 16);
+        }
+        l += rs;
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[x]);
       }
-      // The reference max is raised lazily (p <= 2^8) for bf16; for E4M3 at
-      // every increase, so that p * v_scale <= 2^15 fits the f16 P.
-      const bool need = mt > m_ref + (kFp8 ? 0.f : 8.f);  // also true on the first visible tile
-      // PV of the previous tile must be done before P is overwritten or O rescaled
-      if (j >= 1 && !mbar_wait(o_bar, (uint32_t)((j - 1) & 1), p.flags)) { ok = false; break; }
-      tc_fence_after();
-      const float m_new = need ? mt : m_ref;
-      if (j >= 1 && __any_sync(0xffffffffu, need)) {
-        const float alpha = need ? fast_exp2(m_ref - m_new) : 1.f;
+      // ------------------------------------------------------ epilogue
+      if (ok && nkv[x] > 0 &&
+          mbar_wait(&o_bar[x], (uint32_t)((nkv[x] - 1) & 1), p.flags)) {
+        tc_fence_after();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const int64_t qrow = (int64_t)q_begin + t_local;
+        const int h = g * G + (r % G);
+        __nv_bfloat16* dst = p.out + (qrow * p.num_q_heads + h) * D;
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
           float o[32];
-          tmem_ld32(tmem + lane_base + kColO + c, o);
+          tmem_ld32(tmem + lane_base + colO + c, o);
           tmem_wait_ld();
-          uint32_t u[32];
+          if (row_ok) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(o[i] * alpha);
-          tmem_st16(tmem + lane_base + kColO + c, u);
-          tmem_st16(tmem + lane_base + kColO + c + 16, u + 16);
-        }
-        l *= alpha;
-      }
-      m_ref = m_new;
-      // a row with no visible key yet keeps m_ref = -inf: its p must be 0
-      const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-      const float pv0 = kFp8 ? tf.vs[0] : 1.f;  // E4M3 V scales ride on P
-      const float pv1 = kFp8 ? tf.vs[1] : 1.f;
-      uint32_t pk[kKeys / 2];
-      float rs = 0.f;
-#pragma unroll
-      for (int c = 0; c < kKeys; c += 2) {
-        const float p0 = fast_exp2(s[c] - m_use);
-        const float p1 = fast_exp2(s[c + 1] - m_use);
-        rs += p0 + p1;
-        if constexpr (kFp8) {
-          const float vsc = c < 64 ? pv0 : pv1;
-          pk[c / 2] = pack_f16(p0 * vsc, p1 * vsc);
-        } else {
-          pk[c / 2] = pack_bf16(p0, p1);
-        }
-      }
-      l += rs;
-#pragma unroll
-      for (int c = 0; c < kKeys / 2; c += 16) tmem_st16(tmem + lane_base + kColP + c, pk + c);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
-    }
-    // -------------------------------------------------------- epilogue
-    if (ok && n_kv > 0 && mbar_wait(o_bar, (uint32_t)((n_kv - 1) & 1), p.flags)) {
-      tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const int64_t qrow = (int64_t)q_begin + t_local;
-      const int h = g * G + (r % G);
-      __nv_bfloat16* dst = p.out + (qrow * p.num_q_heads + h) * D;
-#pragma unroll
-      for (int c = 0; c < D; c += 32) {
-        float o[32];
-        tmem_ld32(tmem + lane_base + kColO + c, o);
-        tmem_wait_ld();
-        if (row_ok) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-            uint4 v;
-            v.x = pack_bf16(o[i] * inv, o[i + 1] * inv);
-            v.y = pack_bf16(o[i + 2] * inv, o[i + 3] * inv);
-            v.z = pack_bf16(o[i + 4] * inv, o[i + 5] * inv);
-            v.w = pack_bf16(o[i + 6] * inv, o[i + 7] * inv);
-            *reinterpret_cast<uint4*>(dst + c + i) = v;
+            for (int i = 0; i < 32; i += 8) {
+              uint4 v;
+              v.x = pack_bf16(o[i] * inv, o[i + 1] * inv);
+              v.y = pack_bf16(o[i + 2] * inv, o[i + 3] * inv);
+              v.z = pack_bf16(o[i + 4] * inv, o[i + 5] * inv);
+              v.w = pack_bf16(o[i + 6] * inv, o[i + 7] * inv);
+              *reinterpret_cast<uint4*>(dst + c + i) = v;
+            }
           }
         }
+        if (row_ok && p.lse)
+          p.lse[qrow * p.num_q_heads + h] =
+              l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
       }
-      if (row_ok && p.lse)
-        p.lse[qrow * p.num_q_heads + h] =
-            l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
   }
 
@@ -735,8 +806,8 @@ int prefill_entry(const pkv_cache* cache, const void* q, int32_t num_q_heads, in
   p.num_pages = cache->num_pages;
   p.page_size = cache->page_size;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
-  const int tq_tokens = pf::kRows / gqa_group;
-  const int q_tiles = (max_q_len + tq_tokens - 1) / tq_tokens;
+  const int pair_tokens = 2 * (pf::kRows / gqa_group);  // two Q tiles per CTA
+  const int q_tiles = (max_q_len + pair_tokens - 1) / pair_tokens;
   cudaError_t e;
   if (D == 128)
     e = fp8 ? pf::launch<128, true>(tq, tk, tv, p, q_tiles, stream)
