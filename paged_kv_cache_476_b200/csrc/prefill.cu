@@ -7,22 +7,27 @@
 // 0..p, out = softmax(scale * q K^T) V.
 //
 // Design (tensor-bound, B200-first):
-//  * One CTA per (128-row Q tile, kv head, chunk).  The 128 rows pack the G
-//    q heads of the kv head for 128/G consecutive query tokens (row = token *
-//    G + head), so every K/V tile staged in shared memory serves the whole
-//    GQA group.
-//  * Warp 4 (producer) loads the Q tile once with a 3-D TMA map over
+//  * One CTA per (pair of 128-row Q tiles A and B, kv head, chunk).  The 128
+//    rows of a tile pack the G q heads of the kv head for 128/G consecutive
+//    query tokens (row = token * G + head), so every K/V tile staged in
+//    shared memory serves the whole GQA group and both Q tiles.
+//  * CTAs take their items longest-first (most KV tiles first), so the short
+//    items fill the tail of the grid instead of the long ones.
+//  * Warp 8 (producer) loads the two Q tiles once with a 3-D TMA map over
 //    [token][head][d] and streams 128-key K/V tiles (one 128-token page or
 //    two 64-token pages, page-table indirected, 128-byte swizzled) into a
 //    two-stage mbarrier ring.
-//  * Warp 5 (one elected thread) issues tcgen05.mma: S = Q K^T (M=128,
-//    N=128, K=head_dim, both operands K-major from shared memory) into one
-//    of two TMEM buffers, then O += P V with P (bf16) read from TMEM and V as
-//    an MN-major operand.  tcgen05.commit signals completion on mbarriers.
-//  * Warps 0-3 (one TMEM lane = one row per thread) run the online softmax:
-//    load S from TMEM, mask the causal diagonal, keep a reference max that
-//    is raised only when a row's max grows by more than 2^8 (then O is
-//    rescaled in TMEM), write P to TMEM, and finally normalise O.
+//  * Warp 9 (one elected thread) issues tcgen05.mma: S = Q K^T (M=128,
+//    N=128, K=head_dim, both operands K-major from shared memory) into the
+//    tile's TMEM S buffer, then O += P V with P (16-bit) read from TMEM over
+//    S and V as an MN-major operand.  tcgen05.commit signals completion on
+//    mbarriers.  The two tiles alternate, so one tile's softmax runs under
+//    the other tile's products.
+//  * Warps 0-3 (tile A) and 4-7 (tile B), one TMEM lane = one row per
+//    thread, run the online softmax: load S from TMEM, mask the causal
+//    diagonal, keep a reference max that is raised only when a row's max
+//    grows by more than 2^8 (then O is rescaled in TMEM), write P to TMEM,
+//    and finally normalise O.
 //  * V rows past the sequence end (or of a rejected page) are zeroed in
 //    shared memory before their PV product: 0 * NaN would poison O.
 //  * E4M3 pools: two converter warps turn each landed E4M3 tile into a 16-bit
@@ -68,6 +73,8 @@ struct Params {
   int32_t max_pages;
   int32_t num_pages;
   int32_t page_size;
+  int32_t pair_slots;  // pairs of Q tiles per chunk the grid provides
+  int32_t lpt;         // 1: longest-first item order, 0: index order
   float scale_log2;
 };
 
@@ -267,6 +274,106 @@ __device__ __forceinline__ void convert_tile(uint32_t src, uint32_t dst, int t, 
   }
 }
 
+// ------------------------------------------------- longest-first CTA order
+// A work item is (chunk, pair of Q tiles); its cost is the number of KV tiles
+// its later tile visits, ceil((ctx + e) / 128) with ctx = L - n and e the end
+// of the pair inside the chunk, min(2 TQ (pair + 1), n): nondecreasing in the
+// pair index.  The hardware dispatches CTAs in index order onto whichever SM
+// frees first, so handing out items by descending cost is the greedy
+// longest-processing-time schedule.  Each CTA derives its item from its rank
+// with a warp-wide count: no plan buffer, no host knowledge of lengths.
+constexpr int kLptChunksPerLane = 4;
+constexpr int kLptMaxChunks = 32 * kLptChunksPerLane;  // more chunks: index order
+
+struct ChunkCost {
+  int32_t ctx, n, pairs;  // pairs: items of the chunk that exist in the grid
+};
+
+// Items of chunk `cc` whose cost is below k.
+__device__ __forceinline__ int32_t pairs_below(const ChunkCost& cc, int32_t k, int32_t pair_tokens) {
+  const int64_t lim = (int64_t)kKeys * (k - 1) - cc.ctx;  // cost < k  <=>  ctx + e <= lim
+  if (lim >= cc.n) return cc.pairs;
+  if (lim <= 0) return 0;
+  return min((int32_t)(lim / pair_tokens), cc.pairs);
+}
+
+// Sum over the warp's chunks of the items with cost >= k.
+__device__ __forceinline__ uint32_t items_at_least(const ChunkCost* cc, int32_t k,
+                                                   int32_t pair_tokens) {
+  uint32_t s = 0;
+#pragma unroll
+  for (int i = 0; i < kLptChunksPerLane; ++i)
+    s += (uint32_t)(cc[i].pairs - pairs_below(cc[i], k, pair_tokens));
+  return __reduce_add_sync(0xffffffffu, s);
+}
+
+// Warp 0: the item of rank `rank` in descending-cost order (ties by chunk
+// index, then pair index).  Returns false when the rank is past the last item.
+__device__ bool lpt_item(const Params& p, uint32_t rank, int32_t pair_tokens, int32_t* chunk_out,
+                         int32_t* pair_out) {
+  const int lane = threadIdx.x & 31;
+  ChunkCost cc[kLptChunksPerLane];
+  int32_t kmax = 0;
+#pragma unroll
+  for (int i = 0; i < kLptChunksPerLane; ++i) {
+    const int c = lane * kLptChunksPerLane + i;
+    cc[i].ctx = cc[i].n = cc[i].pairs = 0;
+    if (c < p.num_chunks) {
+      const int32_t n = max(__ldg(p.cu_q + c + 1) - __ldg(p.cu_q + c), 0);
+      const int32_t L = __ldg(p.seq_lens + c);
+      cc[i].n = n;
+      cc[i].ctx = (int32_t)max((int64_t)L - n, (int64_t)0);
+      cc[i].pairs = min((int32_t)(((int64_t)n + pair_tokens - 1) / pair_tokens), p.pair_slots);
+      kmax = max(kmax, (int32_t)(((int64_t)cc[i].ctx + n + kKeys - 1) / kKeys));
+    }
+  }
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  if (items_at_least(cc, 1, pair_tokens) <= rank) return false;
+  // largest k with more than `rank` items of cost >= k
+  int32_t lo = 1, hi = kmax + 1;
+  while (hi - lo > 1) {
+    const int32_t mid = lo + (hi - lo) / 2;
+    if (items_at_least(cc, mid, pair_tokens) > rank)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  uint32_t o = rank - items_at_least(cc, lo + 1, pair_tokens);  // offset among cost == lo
+  int32_t below[kLptChunksPerLane];
+  uint32_t eq[kLptChunksPerLane], mine = 0;
+#pragma unroll
+  for (int i = 0; i < kLptChunksPerLane; ++i) {
+    below[i] = pairs_below(cc[i], lo, pair_tokens);
+    eq[i] = (uint32_t)(pairs_below(cc[i], lo + 1, pair_tokens) - below[i]);
+    mine += eq[i];
+  }
+  uint32_t incl = mine;  // inclusive scan over lanes (chunks are lane-major)
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += v;
+  }
+  const uint32_t excl = incl - mine;
+  const uint32_t hit = __ballot_sync(0xffffffffu, excl <= o && o < incl);
+  const int owner = __ffs(hit) - 1;  // exists: the counts above add up past o
+  int32_t c_sel = 0, pr_sel = 0;
+  if (lane == owner) {
+    o -= excl;
+#pragma unroll
+    for (int i = 0; i < kLptChunksPerLane; ++i) {
+      if (o < eq[i]) {
+        c_sel = lane * kLptChunksPerLane + i;
+        pr_sel = below[i] + (int32_t)o;
+        break;
+      }
+      o -= eq[i];
+    }
+  }
+  *chunk_out = __shfl_sync(0xffffffffu, c_sel, owner);
+  *pair_out = __shfl_sync(0xffffffffu, pr_sel, owner);
+  return true;
+}
+
 template <int D, bool kFp8>
 __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,
@@ -299,31 +406,28 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
   const int lane = threadIdx.x & 31;
   const int G = p.group;
   const int TQ = kRows / G;  // query tokens per Q tile
-  const int chunk = blockIdx.z;
-  const int g = blockIdx.y;
-  const int qa0 = blockIdx.x * 2 * TQ;  // first token of tile A; tile B follows
+  int32_t* sched = reinterpret_cast<int32_t*>(tmem_base_smem + 1);  // chunk, pair, head
 
-  const int32_t q_begin = __ldg(p.cu_q + chunk);
-  const int32_t n = __ldg(p.cu_q + chunk + 1) - q_begin;
-  int32_t L = __ldg(p.seq_lens + chunk);
-  if (n <= 0 || qa0 >= n) return;  // uniform across the CTA
-  const int32_t cap = p.max_pages * p.page_size;
-  if (L > cap || n > L) {
-    if (threadIdx.x == 0) flag_error(p.flags, PKV_FLAG_BAD_LENGTH);
-    if (n > cap || L < n) return;  // nothing meaningful to compute
-    L = min(L, cap);
+  // Item choice (warp 0), barrier set-up (warp 1) and TMEM allocation (MMA
+  // warp) overlap; one barrier publishes all three.
+  if (warp == 0) {
+    const uint32_t lin = blockIdx.x;
+    int32_t c = -1, pr = 0, hd = 0;
+    if (p.lpt) {
+      hd = (int32_t)(lin % (uint32_t)p.num_kv_heads);
+      if (!lpt_item(p, lin / (uint32_t)p.num_kv_heads, 2 * TQ, &c, &pr)) c = -1;
+    } else {
+      pr = (int32_t)(lin % (uint32_t)p.pair_slots);
+      hd = (int32_t)((lin / (uint32_t)p.pair_slots) % (uint32_t)p.num_kv_heads);
+      c = (int32_t)(lin / ((uint32_t)p.pair_slots * (uint32_t)p.num_kv_heads));
+    }
+    if (lane == 0) {
+      sched[0] = c;
+      sched[1] = pr;
+      sched[2] = hd;
+    }
   }
-  const int q0[2] = {qa0, qa0 + TQ};
-  const bool hasB = q0[1] < n;
-  int nkv[2];
-#pragma unroll
-  for (int x = 0; x < 2; ++x) {
-    const int32_t pmax = L - n + min(q0[x] + TQ, n) - 1;  // largest query position
-    nkv[x] = (x == 0 || hasB) ? (pmax + kKeys) / kKeys : 0;
-  }
-  const int n_kv = max(nkv[0], nkv[1]);  // KV tiles the CTA visits
-
-  if (threadIdx.x == 0) {
+  if (warp == 1 && lane == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&kv_full[s], 1);
@@ -347,6 +451,38 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_base_smem;
+  const int chunk = sched[0];
+  const int g = sched[2];
+  const int qa0 = sched[1] * 2 * TQ;  // first token of tile A; tile B follows
+
+  // Decide, uniformly across the CTA, whether the item has work.
+  bool run = chunk >= 0 && chunk < p.num_chunks;
+  int32_t q_begin = 0, n = 0, L = 0;
+  if (run) {
+    q_begin = __ldg(p.cu_q + chunk);
+    n = __ldg(p.cu_q + chunk + 1) - q_begin;
+    L = __ldg(p.seq_lens + chunk);
+    run = n > 0 && qa0 < n;
+  }
+  const int32_t cap = p.max_pages * p.page_size;
+  if (run && (L > cap || n > L)) {
+    if (threadIdx.x == 0) flag_error(p.flags, PKV_FLAG_BAD_LENGTH);
+    if (n > cap || L < n) run = false;  // nothing meaningful to compute
+    L = min(L, cap);
+  }
+  if (!run) {
+    if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+    return;
+  }
+  const int q0[2] = {qa0, qa0 + TQ};
+  const bool hasB = q0[1] < n;
+  int nkv[2];
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    const int32_t pmax = L - n + min(q0[x] + TQ, n) - 1;  // largest query position
+    nkv[x] = (x == 0 || hasB) ? (pmax + kKeys) / kKeys : 0;
+  }
+  const int n_kv = max(nkv[0], nkv[1]);  // KV tiles the CTA visits
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
@@ -740,12 +876,12 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
 template <int D, bool kFp8>
 size_t smem_bytes() {
   return 1024 + Smem<D, kFp8>::kBytes + (16 + kFactsRing) * sizeof(uint64_t) +
-         kFactsRing * sizeof(TileFacts) + 16;
+         kFactsRing * sizeof(TileFacts) + 32;  // + TMEM base and the item
 }
 
 template <int D, bool kFp8>
 cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                   const Params& p, int q_tiles, cudaStream_t stream) {
+                   const Params& p, cudaStream_t stream) {
   const size_t smem = smem_bytes<D, kFp8>();
   static bool attr = false;
   if (!attr) {
@@ -754,8 +890,8 @@ cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  dim3 grid(q_tiles, p.num_kv_heads, p.num_chunks);
-  prefill_kernel<D, kFp8><<<grid, Smem<D, kFp8>::kThreads, smem, stream>>>(tq, tk, tv, p);
+  const unsigned blocks = (unsigned)p.pair_slots * (unsigned)p.num_kv_heads * (unsigned)p.num_chunks;
+  prefill_kernel<D, kFp8><<<blocks, Smem<D, kFp8>::kThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
@@ -807,14 +943,16 @@ int prefill_entry(const pkv_cache* cache, const void* q, int32_t num_q_heads, in
   p.page_size = cache->page_size;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   const int pair_tokens = 2 * (pf::kRows / gqa_group);  // two Q tiles per CTA
-  const int q_tiles = (max_q_len + pair_tokens - 1) / pair_tokens;
+  p.pair_slots = (max_q_len + pair_tokens - 1) / pair_tokens;
+  p.lpt = num_chunks <= pf::kLptMaxChunks ? 1 : 0;
+  if ((int64_t)p.pair_slots * p.num_kv_heads * num_chunks > INT32_MAX) return PKV_ERR_SHAPE;
   cudaError_t e;
   if (D == 128)
-    e = fp8 ? pf::launch<128, true>(tq, tk, tv, p, q_tiles, stream)
-            : pf::launch<128, false>(tq, tk, tv, p, q_tiles, stream);
+    e = fp8 ? pf::launch<128, true>(tq, tk, tv, p, stream)
+            : pf::launch<128, false>(tq, tk, tv, p, stream);
   else
-    e = fp8 ? pf::launch<64, true>(tq, tk, tv, p, q_tiles, stream)
-            : pf::launch<64, false>(tq, tk, tv, p, q_tiles, stream);
+    e = fp8 ? pf::launch<64, true>(tq, tk, tv, p, stream)
+            : pf::launch<64, false>(tq, tk, tv, p, stream);
   return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 

@@ -54,6 +54,24 @@ def test_prefill_matches_oracle(case):
     assert int(st.flags.item()) == 0
 
 
+@pytest.mark.parametrize("num_chunks", [128, 140])
+def test_prefill_many_chunks(num_chunks):
+    # up to 128 chunks the CTAs take items longest-first, beyond that in index
+    # order; both must cover every (chunk, Q-tile pair, kv head) exactly once
+    rng = np.random.default_rng(num_chunks)
+    ctx = [int(x) for x in rng.choice([0, 7, 150, 600], size=num_chunks)]
+    new = [int(x) for x in rng.choice([1, 5, 33, 64, 200], size=num_chunks)]
+    w = workloads.build("pfmany", 26, ctx, new, page_size=64, num_q_heads=8, num_kv_heads=2,
+                        head_dim=128, pool_slack=0.1, chunk_rows=range(num_chunks))
+    st = GpuState(w)
+    st.append_step()
+    out, lse = st.prefill()
+    torch.cuda.synchronize()
+    ref, ref_lse = _oracle_prefill(w)
+    compare(out, lse, ref, ref_lse)
+    assert int(st.flags.item()) == 0
+
+
 def test_prefill_row_equals_truncated_decode():
     # the last query of a chunk sees exactly what a decode step would see
     w = workloads.build("pfd", 22, [300, 50], [70, 9], page_size=64, num_q_heads=8,
