@@ -65,7 +65,8 @@ typedef enum {
   PKV_ERR_CUDA = -8,        /* a CUDA runtime call or kernel launch failed */
   PKV_ERR_ALIGN = -9,       /* a pointer that must be 16-byte aligned is not */
   PKV_ERR_UNSUPPORTED = -10, /* a valid combination this build does not implement */
-  PKV_ERR_SCRATCH_LIMIT = -11 /* request needs more than the static decode scratch */
+  PKV_ERR_SCRATCH_LIMIT = -11, /* request needs more than the static decode scratch */
+  PKV_ERR_NO_PAGES = -12     /* the free pages cannot cover a growth (paged_kv_runtime.h) */
 } pkv_status;
 
 typedef enum { PKV_KV_BF16 = 0, PKV_KV_FP8_E4M3 = 1 } pkv_kv_dtype;

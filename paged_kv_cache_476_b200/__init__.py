@@ -11,6 +11,7 @@ Entry points (same names as the C ABI):
     paged_decode_attention          split-KV decode, persistent and balanced
     paged_prefill_chunk_attention   causal prefill chunks on tcgen05
     paged_decode_workspace_bytes, paged_decode_plan, pkv_status_string
+    PageAllocator                   host page allocator + in-flight step planner
 """
 from __future__ import annotations
 
@@ -19,6 +20,7 @@ import math
 import os
 from typing import Optional
 
+import numpy as np
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -30,6 +32,7 @@ PKV_FLAG_BAD_PAGE = 0x1
 PKV_FLAG_BAD_LENGTH = 0x2
 PKV_FLAG_TIMEOUT = 0x4
 PKV_FLAG_BAD_SCALE = 0x8
+PKV_ERR_NO_PAGES = -12
 
 # Every symbol include/paged_kv.h declares.
 EXPORTED = (
@@ -41,6 +44,16 @@ EXPORTED = (
     "pkv_status_string",
     "pkv_abi_version",
     "paged_decode_attention_noalloc",
+    # include/paged_kv_runtime.h: host page allocator and step planner
+    "pkv_allocator_create",
+    "pkv_allocator_destroy",
+    "pkv_allocator_grow",
+    "pkv_allocator_release",
+    "pkv_allocator_seq_len",
+    "pkv_allocator_table",
+    "pkv_allocator_stats",
+    "pkv_allocator_free_pages",
+    "pkv_step_plan",
 )
 
 # Size of the library's static decode scratch (see paged_decode_attention_noalloc).
@@ -61,6 +74,21 @@ class PkvCache(ctypes.Structure):
         ("head_dim", ctypes.c_int32),
         ("kv_dtype", ctypes.c_int32),
         ("error_flags", ctypes.c_void_p),
+    ]
+
+
+class AllocStats(ctypes.Structure):
+    """Mirror of ``struct pkv_alloc_stats``."""
+
+    _fields_ = [
+        ("num_pages", ctypes.c_int32),
+        ("page_size", ctypes.c_int32),
+        ("max_seqs", ctypes.c_int32),
+        ("max_pages_per_seq", ctypes.c_int32),
+        ("pages_in_use", ctypes.c_int32),
+        ("peak_pages_in_use", ctypes.c_int32),
+        ("live_seqs", ctypes.c_int32),
+        ("tokens_cached", ctypes.c_int64),
     ]
 
 
@@ -94,6 +122,23 @@ def _load() -> ctypes.CDLL:
     lib.pkv_status_string.argtypes = [ctypes.c_int]
     lib.pkv_status_string.restype = ctypes.c_char_p
     lib.pkv_abi_version.restype = ctypes.c_int
+    ap = ctypes.c_void_p
+    pi = ctypes.POINTER(I32)
+    lib.pkv_allocator_create.argtypes = [I32, I32, I32, I32, pi, ctypes.POINTER(ap)]
+    lib.pkv_allocator_destroy.argtypes = [ap]
+    lib.pkv_allocator_destroy.restype = None
+    lib.pkv_allocator_grow.argtypes = [ap, I32, I32]
+    lib.pkv_allocator_release.argtypes = [ap, I32]
+    lib.pkv_allocator_seq_len.argtypes = [ap, I32, pi]
+    lib.pkv_allocator_table.argtypes = [ap]
+    lib.pkv_allocator_table.restype = pi
+    lib.pkv_allocator_stats.argtypes = [ap, ctypes.POINTER(AllocStats)]
+    lib.pkv_allocator_free_pages.argtypes = [ap, pi, I32, pi]
+    lib.pkv_step_plan.argtypes = [ap, pi, pi, I32, pi, pi, pi, pi]
+    for n in ("pkv_allocator_create", "pkv_allocator_grow", "pkv_allocator_release",
+              "pkv_allocator_seq_len", "pkv_allocator_stats", "pkv_allocator_free_pages",
+              "pkv_step_plan"):
+        getattr(lib, n).restype = ctypes.c_int
     return lib
 
 
@@ -303,3 +348,179 @@ def paged_decode_attention_noalloc(cache: PagedKVCache, q, page_table, seq_lens,
         _ptr(out), _ptr(lse), int(num_ctas), _stream(stream))
     _check("paged_decode_attention_noalloc", st)
     return out, lse
+
+
+# ----------------------------------------------------- host runtime (paged_kv_runtime.h)
+def _i32p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+class PageAllocator:
+    """The library's host page allocator (``pkv_allocator``) for one pool.
+
+    Free pages form a stack (``page_order[0]`` on top); growing a slot pops
+    pages in logical order, releasing pushes them back so the slot's first page
+    ends on top; growth is all-or-nothing.  ``table`` is a live numpy view of
+    the allocator's ``[max_seqs][max_pages_per_seq]`` page table.
+    """
+
+    def __init__(self, num_pages: int, page_size: int, max_seqs: int, max_pages_per_seq: int,
+                 page_order: Optional[np.ndarray] = None):
+        order = None
+        if page_order is not None:
+            order = np.ascontiguousarray(page_order, dtype=np.int32)
+            if order.shape != (num_pages,):
+                raise ValueError("page_order must have num_pages entries")
+        h = ctypes.c_void_p()
+        _check("pkv_allocator_create",
+               _lib.pkv_allocator_create(num_pages, page_size, max_seqs, max_pages_per_seq,
+                                         None if order is None else _i32p(order),
+                                         ctypes.byref(h)))
+        self._h = h
+        self._destroy = _lib.pkv_allocator_destroy  # usable during interpreter shutdown
+        self.num_pages, self.page_size = num_pages, page_size
+        self.max_seqs, self.max_pages_per_seq = max_seqs, max_pages_per_seq
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            self._destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        self.close()
+
+    def grow(self, slot: int, new_len: int) -> int:
+        """Grow ``slot`` to ``new_len`` tokens; returns the status (0 or PKV_ERR_NO_PAGES)."""
+        st = _lib.pkv_allocator_grow(self._h, slot, new_len)
+        if st not in (0, PKV_ERR_NO_PAGES):
+            _check("pkv_allocator_grow", st)
+        return st
+
+    def release(self, slot: int):
+        _check("pkv_allocator_release", _lib.pkv_allocator_release(self._h, slot))
+
+    def seq_len(self, slot: int) -> int:
+        v = ctypes.c_int32()
+        _check("pkv_allocator_seq_len", _lib.pkv_allocator_seq_len(self._h, slot, ctypes.byref(v)))
+        return v.value
+
+    @property
+    def table(self) -> np.ndarray:
+        p = _lib.pkv_allocator_table(self._h)
+        return np.ctypeslib.as_array(p, shape=(self.max_seqs, self.max_pages_per_seq))
+
+    def stats(self) -> AllocStats:
+        s = AllocStats()
+        _check("pkv_allocator_stats", _lib.pkv_allocator_stats(self._h, ctypes.byref(s)))
+        return s
+
+    def free_pages(self) -> np.ndarray:
+        """The free stack, top first."""
+        n = ctypes.c_int32()
+        out = np.empty(self.num_pages, dtype=np.int32)
+        _check("pkv_allocator_free_pages",
+               _lib.pkv_allocator_free_pages(self._h, _i32p(out), self.num_pages, ctypes.byref(n)))
+        return out[: n.value].copy()
+
+    def step_plan(self, slots, new_tokens):
+        """Plan one in-flight step (see ``pkv_step_plan``).
+
+        Returns ``(status, plan)``; ``plan`` is a dict of host int32 arrays
+        ``seq_lens_before [n]``, ``cu_new [n+1]``, ``seq_lens_after [n]`` and
+        ``page_table [n][max_pages_per_seq]``, or None on PKV_ERR_NO_PAGES.
+        """
+        slots = np.ascontiguousarray(slots, dtype=np.int32)
+        new = np.ascontiguousarray(new_tokens, dtype=np.int32)
+        n = len(slots)
+        if new.shape != (n,):
+            raise ValueError("slots and new_tokens must have the same length")
+        before = np.empty(n, np.int32)
+        cu = np.empty(n + 1, np.int32)
+        after = np.empty(n, np.int32)
+        table = np.empty((n, self.max_pages_per_seq), np.int32)
+        st = _lib.pkv_step_plan(self._h, _i32p(slots), _i32p(new), n, _i32p(before), _i32p(cu),
+                                _i32p(after), _i32p(table))
+        if st == PKV_ERR_NO_PAGES:
+            return st, None
+        _check("pkv_step_plan", st)
+        return 0, {"seq_lens_before": before, "cu_new": cu, "seq_lens_after": after,
+                   "page_table": table}
+
+
+class StepDriver:
+    """One in-flight step on the library: plan pages, stage, append, attend.
+
+    Rows of a step are ordered decode rows first (one new token each), then
+    prefill chunks.  ``pkv_step_plan`` writes the step's lengths, prefix sums
+    and page-table rows straight into one pinned host buffer, one
+    host-to-device copy moves it, and the step runs ``paged_kv_append`` over
+    all rows, ``paged_decode_attention`` over the decode rows and
+    ``paged_prefill_chunk_attention`` over the chunks, on one stream.
+    """
+
+    def __init__(self, cache: PagedKVCache, allocator: PageAllocator, max_rows: int,
+                 device="cuda"):
+        self.cache, self.alloc = cache, allocator
+        self.max_rows = int(max_rows)
+        mp = allocator.max_pages_per_seq
+        n = self.max_rows
+        words = 4 * n + 2 + n * mp
+        self._host = torch.empty(words, dtype=torch.int32, pin_memory=True)
+        self._dev = torch.empty(words, dtype=torch.int32, device=device)
+        self._slots = np.empty(n, np.int32)
+        self._new = np.empty(n, np.int32)
+        self._copied = None  # event: the staging buffer's last copy is done
+        self.device = device
+
+    def step(self, decode_slots, chunk_slots, chunk_lens, k_new, v_new, q_decode=None,
+             q_chunks=None, softmax_scale=None, stream=None):
+        """Run one step; returns ``(status, decode (out, lse) or None, chunks (out, lse) or None)``.
+
+        ``k_new``/``v_new``: bf16 ``[T, Hkv, D]`` on the device, the decode
+        rows' tokens first, then each chunk's tokens.  On PKV_ERR_NO_PAGES
+        nothing is launched and the allocator is unchanged.
+        """
+        nd, nc = len(decode_slots), len(chunk_slots)
+        n = nd + nc
+        if n == 0 or n > self.max_rows:
+            raise ValueError(f"a step needs 1..{self.max_rows} rows, got {n}")
+        mp = self.alloc.max_pages_per_seq
+        self._slots[:nd] = decode_slots
+        self._slots[nd:n] = chunk_slots
+        self._new[:nd] = 1
+        self._new[nd:n] = chunk_lens
+        if self._copied is not None:
+            self._copied.synchronize()  # the previous step's copy still reads the buffer
+        h = self._host.numpy()
+        before, cu = h[0:n], h[n:2 * n + 1]
+        after, table = h[2 * n + 1:3 * n + 1], h[3 * n + 1:3 * n + 1 + n * mp]
+        cu_q = h[3 * n + 1 + n * mp:3 * n + 1 + n * mp + nc + 1]
+        st = _lib.pkv_step_plan(self.alloc._h, _i32p(self._slots), _i32p(self._new), n,
+                                _i32p(before), _i32p(cu), _i32p(after), _i32p(table))
+        if st == PKV_ERR_NO_PAGES:
+            return st, None, None
+        _check("pkv_step_plan", st)
+        cu_q[:] = cu[nd:n + 1] - cu[nd]  # the chunks' own prefix sums
+        words = 3 * n + 2 + n * mp + nc
+        s = torch.cuda.current_stream() if stream is None else stream
+        with torch.cuda.stream(s):
+            d = self._dev[:words]
+            d.copy_(self._host[:words], non_blocking=True)
+            self._copied = torch.cuda.Event()
+            self._copied.record(s)
+            d_before, d_cu = d[0:n], d[n:2 * n + 1]
+            d_after = d[2 * n + 1:3 * n + 1]
+            d_table = d[3 * n + 1:3 * n + 1 + n * mp].view(n, mp)
+            d_cu_q = d[3 * n + 1 + n * mp:]
+            total = int(cu[n])
+            paged_kv_append(self.cache, d_table, d_before, d_cu, k_new, v_new,
+                            total_new_tokens=total, stream=s)
+            dec = chk = None
+            if nd:
+                dec = paged_decode_attention(self.cache, q_decode, d_table[:nd], d_after[:nd],
+                                             int(after[:nd].max()), softmax_scale, stream=s)
+            if nc:
+                chk = paged_prefill_chunk_attention(self.cache, q_chunks, d_cu_q, d_table[nd:],
+                                                    d_after[nd:], int(self._new[nd:n].max()),
+                                                    softmax_scale, stream=s)
+        return 0, dec, chk

@@ -2,7 +2,8 @@
 
 Usage: ``python paged_kv_cache_476_b200/build.py [--force]`` (run it as a
 file: importing the package first would load a possibly stale library).  Each ``.cu``
-under ``csrc/`` compiles to an object in ``_build/`` (in parallel), then the
+under ``csrc/`` compiles with nvcc and each host-only ``.cpp`` with g++ to an
+object in ``_build/`` (in parallel), then the
 objects link into ``paged_kv_cache_476_b200/libpagedkv.so`` with the CUDA
 runtime linked statically.  nvcc cross-compiles, so no GPU is needed.
 """
@@ -26,8 +27,12 @@ FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2", "-Xptxas",
          f"-I{os.path.join(ROOT, 'include')}", f"-I{CSRC}"]
 
 
+CXX = os.environ.get("CXX", "g++")
+CXXFLAGS = ["-O2", "-std=c++17", "-fPIC", "-Wall", f"-I{os.path.join(ROOT, 'include')}"]
+
+
 def _sources():
-    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
 
 
 def _headers():
@@ -43,9 +48,12 @@ def _stale(target, deps):
 
 
 def _compile(src, extra):
-    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+    obj = os.path.join(BUILD, os.path.splitext(os.path.basename(src))[0] + ".o")
     if _stale(obj, [src, *_headers()]) or extra.get("force"):
-        cmd = [NVCC, *ARCH, *FLAGS, *extra.get("flags", []), "-c", src, "-o", obj]
+        if src.endswith(".cpp"):  # host-only runtime code
+            cmd = [CXX, *CXXFLAGS, "-c", src, "-o", obj]
+        else:
+            cmd = [NVCC, *ARCH, *FLAGS, *extra.get("flags", []), "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed on {src}:\n{r.stdout}\n{r.stderr}")

@@ -127,6 +127,7 @@ const char* pkv_status_string(int status) {
     case PKV_ERR_UNSUPPORTED: return "this combination is not implemented";
     case PKV_ERR_SCRATCH_LIMIT:
       return "the request needs more decode scratch than the library's static 16 MiB array";
+    case PKV_ERR_NO_PAGES: return "the free pages cannot cover the growth request";
     default: return "unknown status";
   }
 }

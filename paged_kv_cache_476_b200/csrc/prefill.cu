@@ -15,8 +15,10 @@
 //    items fill the tail of the grid instead of the long ones.
 //  * Warp 8 (producer) loads the two Q tiles once with a 3-D TMA map over
 //    [token][head][d] and streams 128-key K/V tiles (one 128-token page or
-//    two 64-token pages, page-table indirected, 128-byte swizzled) into a
-//    two-stage mbarrier ring.
+//    two 64-token pages, page-table indirected, 128-byte swizzled) into
+//    two-slot K and V rings; a K slot frees as soon as both S products have
+//    read it, so the next K streams in a whole tile ahead, and the page
+//    lookup of the next tile runs before the slot wait.
 //  * Warp 9 (one elected thread) issues tcgen05.mma: S = Q K^T (M=128,
 //    N=128, K=head_dim, both operands K-major from shared memory) into the
 //    tile's TMEM S buffer, then O += P V with P (16-bit) read from TMEM over
@@ -152,6 +154,15 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// Store 8 consecutive 32-bit columns of this warp's 32 TMEM lanes.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+
 // Store 16 consecutive 32-bit columns of this warp's 32 TMEM lanes.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
   asm volatile(
@@ -161,6 +172,29 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
       "r"(r[15])
       : "memory");
+}
+
+// max(a, b, c) in one instruction (three-input form of sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// O row (this thread's TMEM lane, D fp32 columns from taddr) *= alpha.
+template <int D>
+__device__ __forceinline__ void rescale_o(uint32_t taddr, float alpha) {
+#pragma unroll
+  for (int c = 0; c < D; c += 32) {
+    float o[32];
+    tmem_ld32(taddr + c, o);
+    tmem_wait_ld();
+    uint32_t u[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(o[i] * alpha);
+    tmem_st16(taddr + c, u);
+    tmem_st16(taddr + c + 16, u + 16);
+  }
 }
 
 __device__ __forceinline__ void fence_async_smem() {
@@ -388,9 +422,13 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
   uint8_t* sconv = skv + kStages * Sm::kStageB;     // E4M3 only: 16-bit K, then V
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sm::kBytes);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;               // [kStages] TMA landed
-  uint64_t* kv_empty = kv_full + kStages;     // [kStages] stage may be refilled
-  uint64_t* s_full = kv_empty + kStages;      // [2] S of tile A / B computed
+  // K and V have rings of their own: K(j) is free once both S products of
+  // tile j ran, long before V(j) is, so K(j + 2) streams in early.
+  uint64_t* k_full = bars + 1;                // [kStages] TMA landed
+  uint64_t* k_empty = k_full + kStages;       // [kStages] slot may be refilled
+  uint64_t* v_full = k_empty + kStages;
+  uint64_t* v_empty = v_full + kStages;
+  uint64_t* s_full = v_empty + kStages;       // [2] S of tile A / B computed
   uint64_t* p_full = s_full + 2;              // [2] P of tile A / B written
   uint64_t* o_bar = p_full + 2;               // [2] PV of tile A / B done
   uint64_t* done_bar = o_bar + 2;
@@ -430,8 +468,10 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
   if (warp == 1 && lane == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], kFp8 ? 2 : 1);  // E4M3: released by the two converter warps
+      mbar_init(&k_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&k_empty[s], kFp8 ? 2 : 1);  // E4M3: released by the two converter warps
+      mbar_init(&v_empty[s], kFp8 ? 2 : 1);
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&s_full[x], 1);
@@ -500,29 +540,28 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
                       q_begin + q0[x], q_full);
       }
     }
-    const uint64_t pol = policy_evict_first();
-    for (int j = 0; j < n_kv; ++j) {
-      const int st = j % kStages;
-      if (j >= kStages) {
-        if (!mbar_wait(&kv_empty[st], (uint32_t)((j / kStages - 1) & 1), p.flags)) break;
-      }
-      if (lane == 0) {
-        uint8_t* kd = skv + st * Sm::kStageB;
-        uint8_t* vd = kd + Sm::kStageB / 2;
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      // Page lookup of tile j: page ids, E4M3 scales, rejected 64-key blocks.
+      struct Lookup {
         TileFacts tf;
-        tf.bad = 0;
-        uint32_t bytes = 0;
-        int32_t ys[2] = {0, 0};
-        bool live[2] = {false, false};
+        int32_t ys[2];  // first pool row of each 64-key block
+        int live;       // bit per 64-key block with data to load
+      };
+      auto lookup = [&](int j) -> Lookup {
+        Lookup lk;
+        lk.tf.bad = 0;
+        lk.live = 0;
         for (int sb = 0; sb < 2; ++sb) {
-          tf.ks[sb] = tf.vs[sb] = 1.f;
+          lk.tf.ks[sb] = lk.tf.vs[sb] = 1.f;
+          lk.ys[sb] = 0;
           const int32_t key0 = j * kKeys + sb * 64;
           if (key0 >= L) continue;
           const int32_t pj = key0 / p.page_size;
-          int32_t pid = __ldg(p.page_table + (int64_t)chunk * p.max_pages + pj);
+          const int32_t pid = __ldg(p.page_table + (int64_t)chunk * p.max_pages + pj);
           if (pid < 0 || pid >= p.num_pages) {
             flag_error(p.flags, PKV_FLAG_BAD_PAGE);
-            tf.bad |= 1 << sb;
+            lk.tf.bad |= 1 << sb;
             continue;
           }
           if constexpr (kFp8) {
@@ -530,37 +569,51 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
             const float vs = __ldg(p.v_scale + (int64_t)pid * p.num_kv_heads + g);
             if (!(ks > 0.f && ks <= 32768.f && vs > 0.f && vs <= 32768.f)) {
               flag_error(p.flags, PKV_FLAG_BAD_SCALE);
-              tf.bad |= 1 << sb;
+              lk.tf.bad |= 1 << sb;
               continue;
             }
-            tf.ks[sb] = ks;
-            tf.vs[sb] = vs;
+            lk.tf.ks[sb] = ks;
+            lk.tf.vs[sb] = vs;
           }
-          ys[sb] = (int32_t)(((int64_t)pid * p.num_kv_heads + g) * p.page_size +
-                             key0 % p.page_size);
-          live[sb] = true;
-          bytes += kFp8 ? 2u * 64u * D : 2u * Sm::kHalves * 64u * 128u;
+          lk.ys[sb] = (int32_t)(((int64_t)pid * p.num_kv_heads + g) * p.page_size +
+                                key0 % p.page_size);
+          lk.live |= 1 << sb;
         }
-        facts[j % kFactsRing] = tf;
-        mbar_arrive(&facts_full[j % kFactsRing]);
-        mbar_arrive_expect_tx(&kv_full[st], bytes);
+        return lk;
+      };
+      // bytes of one operand (K or V) per live 64-key block
+      constexpr uint32_t kBlockBytes = kFp8 ? 64u * D : Sm::kHalves * 64u * 128u;
+      // load one operand of a tile into its slot
+      auto load = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, const Lookup& lk) {
+        mbar_arrive_expect_tx(bar, (uint32_t)__popc(lk.live) * kBlockBytes);
         for (int sb = 0; sb < 2; ++sb) {
-          if (!live[sb]) continue;
+          if (!((lk.live >> sb) & 1)) continue;
           if constexpr (kFp8) {
-            tma_load_2d(kd + sb * 64 * D, &tmap_k, 0, ys[sb], &kv_full[st], pol);
-            tma_load_2d(vd + sb * 64 * D, &tmap_v, 0, ys[sb], &kv_full[st], pol);
+            tma_load_2d(dst + sb * 64 * D, map, 0, lk.ys[sb], bar, pol);
           } else {
 #pragma unroll
-            for (int h = 0; h < Sm::kHalves; ++h) {
-              tma_load_2d(kd + h * Sm::kHalfB + sb * 64 * 128, &tmap_k, h * 64, ys[sb],
-                          &kv_full[st], pol);
-              tma_load_2d(vd + h * Sm::kHalfB + sb * 64 * 128, &tmap_v, h * 64, ys[sb],
-                          &kv_full[st], pol);
-            }
+            for (int h = 0; h < Sm::kHalves; ++h)
+              tma_load_2d(dst + h * Sm::kHalfB + sb * 64 * 128, map, h * 64, lk.ys[sb], bar,
+                          pol);
           }
         }
+      };
+      Lookup cur = lookup(0);
+      for (int j = 0; j < n_kv; ++j) {
+        const int st = j % kStages;
+        const uint32_t ph = (uint32_t)((j / kStages - 1) & 1);
+        uint8_t* kd = skv + st * Sm::kStageB;
+        uint8_t* vd = kd + Sm::kStageB / 2;
+        // K(j) replaces K(j - 2), whose S products are done: every reader of
+        // the facts of tile j - 4 has finished too.
+        if (j >= kStages && !mbar_wait(&k_empty[st], ph, p.flags)) break;
+        facts[j % kFactsRing] = cur.tf;
+        mbar_arrive(&facts_full[j % kFactsRing]);
+        load(&tmap_k, kd, &k_full[st], cur);
+        if (j >= kStages && !mbar_wait(&v_empty[st], ph, p.flags)) break;
+        load(&tmap_v, vd, &v_full[st], cur);
+        if (j + 1 < n_kv) cur = lookup(j + 1);  // ahead of the next slot wait
       }
-      __syncwarp();
     }
   } else if (kFp8 && warp >= kConvWarp0) {
     // ------------------------------------------------- E4M3 -> 16-bit converters
@@ -568,7 +621,8 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
     const uint32_t kc = smem_u32(sconv), vc = kc + Sm::kTileB;
     for (int j = 0; j < n_kv; ++j) {
       const int st = j % kStages;
-      if (!mbar_wait(&kv_full[st], (uint32_t)((j / kStages) & 1), p.flags)) break;
+      const uint32_t par = (uint32_t)((j / kStages) & 1);
+      if (!mbar_wait(&k_full[st], par, p.flags)) break;
       const uint32_t k8 = smem_u32(skv + st * Sm::kStageB), v8 = k8 + Sm::kStageB / 2;
       const int bad = facts[j % kFactsRing].bad;
       const int32_t key0 = j * kKeys;
@@ -578,7 +632,11 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
       convert_tile<D, false>(k8, kc, t, zero_from, bad);  // bf16, like Q
       fence_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(kc_full);
+      if (lane == 0) {
+        mbar_arrive(kc_full);
+        mbar_arrive(&k_empty[st]);  // the E4M3 K slot may be refilled
+      }
+      if (!mbar_wait(&v_full[st], par, p.flags)) break;
       // V (rows that must not count are zeros: 0 * NaN would poison O)
       if (j >= 1 && !mbar_wait(vc_free, (uint32_t)((j - 1) & 1), p.flags)) break;
       convert_tile<D, true>(v8, vc, t, zero_from, bad);  // f16, like P
@@ -586,7 +644,7 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(vc_full);
-        mbar_arrive(&kv_empty[st]);  // the E4M3 stage may be refilled
+        mbar_arrive(&v_empty[st]);  // the E4M3 V slot may be refilled
       }
     }
   } else if (warp == kMmaWarp) {
@@ -604,7 +662,7 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
         return mbar_wait(kc_full, (uint32_t)(j & 1), p.flags);
       } else {
         *addr = smem_u32(skv + (j % kStages) * Sm::kStageB);
-        return mbar_wait(&kv_full[j % kStages], (uint32_t)((j / kStages) & 1), p.flags);
+        return mbar_wait(&k_full[j % kStages], (uint32_t)((j / kStages) & 1), p.flags);
       }
     };
     auto issue_s = [&](int x, uint32_t k_addr) {
@@ -631,6 +689,7 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
         return mbar_wait(vc_full, (uint32_t)(j & 1), p.flags);
       } else {
         const int st = j % kStages;
+        if (!mbar_wait(&v_full[st], (uint32_t)((j / kStages) & 1), p.flags)) return false;
         const int32_t key0 = j * kKeys;
         const int bad = facts[j % kFactsRing].bad;
         int zlo = kKeys;
@@ -675,7 +734,7 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
     if (ok) {
       issue_s(0, k_addr);
       if (hasB) issue_s(1, k_addr);
-      if (kFp8 && lane == 0) tc_commit(kc_free);  // K_0 is read by both S products
+      if (lane == 0) tc_commit(kFp8 ? kc_free : &k_empty[0]);  // K_0 is read by both S products
       __syncwarp();
     }
     for (int j = 0; j < n_kv && ok; ++j) {
@@ -686,16 +745,12 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
       if (next && !(ok = k_ready(j + 1, &k_addr))) break;
       if (j + 1 < nkv[0]) issue_s(0, k_addr);
       if (j < nkv[1] && !(ok = issue_pv(1, j, v_addr))) break;
-      if (lane == 0) {
-        // this KV tile is consumed once both PV products have run
-        if constexpr (kFp8)
-          tc_commit(vc_free);
-        else
-          tc_commit(&kv_empty[j % kStages]);
-      }
+      // V_j is consumed once both PV products have run, K_{j+1} once both
+      // S products have
+      if (lane == 0) tc_commit(kFp8 ? vc_free : &v_empty[j % kStages]);
       __syncwarp();
       if (j + 1 < nkv[1]) issue_s(1, k_addr);
-      if (kFp8 && next && lane == 0) tc_commit(kc_free);  // K_{j+1} consumed
+      if (next && lane == 0) tc_commit(kFp8 ? kc_free : &k_empty[(j + 1) % kStages]);
       __syncwarp();
     }
     // every MMA this thread issued must finish before TMEM is released
@@ -734,93 +789,87 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
           return keep ? v * (c < 64 ? mul0 : mul1) : -INFINITY;
         };
         // Tiles off the diagonal without a rejected page (nearly all) take a
-        // lean path: max of the raw scores, then one FMA + ex2 per element.
-        const bool plain = !diag && tf.bad == 0;
-        // pass 1: row max of the scaled, masked scores (64 columns per load)
-        float mt = -INFINITY;
-#pragma unroll
-        for (int cb = 0; cb < kKeys; cb += 64) {
-          float sv[64];
-          tmem_ld32(tmem + lane_base + colS + cb, sv);
-          tmem_ld32(tmem + lane_base + colS + cb + 32, sv + 32);
-          tmem_wait_ld();
-          if (plain) {
-            float m = sv[0];
-#pragma unroll
-            for (int i = 1; i < 64; ++i) m = fmaxf(m, sv[i]);
-            mt = fmaxf(mt, m * (cb < 64 ? mul0 : mul1));  // the multipliers are > 0
-          } else {
-#pragma unroll
-            for (int i = 0; i < 64; ++i) mt = fmaxf(mt, scaled(sv[i], cb + i));
-          }
-        }
-        // The reference max is raised lazily (p <= 2^8) for bf16; for E4M3 at
-        // every increase, so that p * v_scale <= 2^15 fits the f16 P.
-        const bool need = mt > m_ref + (kFp8 ? 0.f : 8.f);  // true on the first visible tile
-        const float m_new = need ? mt : m_ref;
-        // S(j) done implies every earlier MMA is done, PV(j-1) included: O is
-        // stable and the P columns are free.
-        if (j >= 1 && __any_sync(0xffffffffu, need)) {
-          const float alpha = need ? fast_exp2(m_ref - m_new) : 1.f;
-#pragma unroll
-          for (int c = 0; c < D; c += 32) {
-            float o[32];
-            tmem_ld32(tmem + lane_base + colO + c, o);
-            tmem_wait_ld();
-            uint32_t u[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(o[i] * alpha);
-            tmem_st16(tmem + lane_base + colO + c, u);
-            tmem_st16(tmem + lane_base + colO + c + 16, u + 16);
-          }
-          l *= alpha;
-        }
-        m_ref = m_new;
-        // a row with no visible key yet keeps m_ref = -inf: its p must be 0
-        const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-        const float pv0 = kFp8 ? tf.vs[0] : 1.f;  // E4M3 V scales ride on P
-        const float pv1 = kFp8 ? tf.vs[1] : 1.f;
-        // pass 2: P over S's own columns (16-bit pairs: P column c/2 lies in
-        // an S column already read)
+        // lean path: max of the raw scores, then one FMA + exp2 per element.
+        // (max(s) * mul = max(s * mul) needs mul > 0; other scales go the
+        // general way.)
+        const bool plain = !diag && tf.bad == 0 && mul0 > 0.f && mul1 > 0.f;
+        // Raise the reference max to the tile max mt when needed: lazily (p
+        // <= 2^8) for bf16; for E4M3 at every increase, so that p * v_scale
+        // <= 2^15 fits the f16 P.  Returns the max to subtract (0 while a row
+        // has seen no key, so that its p are 0).  O is rescaled by alpha
+        // after P is written (the registers of S are free by then): S(j) done
+        // implies every earlier MMA is done, PV(j-1) included, and PV(j)
+        // waits for this tile's P.
+        float alpha = 1.f;
+        auto set_max = [&](float mt) -> float {
+          const bool need = mt > m_ref + (kFp8 ? 0.f : 8.f);  // true on the first visible tile
+          const float m_new = need ? mt : m_ref;
+          if (j >= 1 && need) alpha = fast_exp2(m_ref - m_new);
+          m_ref = m_new;
+          return m_ref == -INFINITY ? 0.f : m_ref;
+        };
         float rs = 0.f;
+        {
+          // Two 64-column passes: the row max, then P.
+          float mt = -INFINITY;
 #pragma unroll
-        for (int cb = 0; cb < kKeys; cb += 64) {
-          float sv[64];
-          tmem_ld32(tmem + lane_base + colS + cb, sv);
-          tmem_ld32(tmem + lane_base + colS + cb + 32, sv + 32);
-          tmem_wait_ld();
-          const float mul = cb < 64 ? mul0 : mul1;
-          const float vsc = cb < 64 ? pv0 : pv1;
-          uint32_t pk[32];
-          // (two loops rather than a branch per element, which the compiler
-          // would turn into both paths under predicates)
-          if (plain) {
+          for (int cb = 0; cb < kKeys; cb += 64) {
+            float sv[64];
+            tmem_ld32(tmem + lane_base + colS + cb, sv);
+            tmem_ld32(tmem + lane_base + colS + cb + 32, sv + 32);
+            tmem_wait_ld();
+            if (plain) {
+              float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-            for (int i = 0; i < 64; i += 2) {
-              const float p0 = fast_exp2(fmaf(sv[i], mul, -m_use));
-              const float p1 = fast_exp2(fmaf(sv[i + 1], mul, -m_use));
-              rs += p0 + p1;
-              if constexpr (kFp8)
-                pk[i / 2] = pack_f16(p0 * vsc, p1 * vsc);
-              else
-                pk[i / 2] = pack_bf16(p0, p1);
-            }
-          } else {
+              for (int i = 0; i < 64; i += 4) {
+                m0 = fmax3(m0, sv[i], sv[i + 1]);
+                m1 = fmax3(m1, sv[i + 2], sv[i + 3]);
+              }
+              mt = fmaxf(mt, fmaxf(m0, m1) * (cb < 64 ? mul0 : mul1));
+            } else {
 #pragma unroll
-            for (int i = 0; i < 64; i += 2) {
-              const float p0 = fast_exp2(scaled(sv[i], cb + i) - m_use);
-              const float p1 = fast_exp2(scaled(sv[i + 1], cb + i + 1) - m_use);
-              rs += p0 + p1;
-              if constexpr (kFp8)
-                pk[i / 2] = pack_f16(p0 * vsc, p1 * vsc);
-              else
-                pk[i / 2] = pack_bf16(p0, p1);
+              for (int i = 0; i < 64; ++i) mt = fmaxf(mt, scaled(sv[i], cb + i));
             }
           }
-          tmem_st16(tmem + lane_base + colS + cb / 2, pk);
-          tmem_st16(tmem + lane_base + colS + cb / 2 + 16, pk + 16);
+          const float m_use = set_max(mt);
+#pragma unroll
+          for (int cb = 0; cb < kKeys; cb += 64) {
+            float sv[64];
+            tmem_ld32(tmem + lane_base + colS + cb, sv);
+            tmem_ld32(tmem + lane_base + colS + cb + 32, sv + 32);
+            tmem_wait_ld();
+            const float mul = cb < 64 ? mul0 : mul1;
+            const float vsc = kFp8 ? (cb < 64 ? tf.vs[0] : tf.vs[1]) : 1.f;  // E4M3 V scales ride on P
+            uint32_t pk[32];
+            // (two loops rather than a branch per element, which the compiler
+            // would turn into both paths under predicates)
+            if (plain) {
+              float r0 = 0.f, r1 = 0.f;
+#pragma unroll
+              for (int i = 0; i < 64; i += 2) {
+                const float p0 = fast_exp2(fmaf(sv[i], mul, -m_use));
+                const float p1 = fast_exp2(fmaf(sv[i + 1], mul, -m_use));
+                r0 += p0;
+                r1 += p1;
+                pk[i / 2] = kFp8 ? pack_f16(p0 * vsc, p1 * vsc) : pack_bf16(p0, p1);
+              }
+              rs += r0 + r1;
+            } else {
+#pragma unroll
+              for (int i = 0; i < 64; i += 2) {
+                const float p0 = fast_exp2(scaled(sv[i], cb + i) - m_use);
+                const float p1 = fast_exp2(scaled(sv[i + 1], cb + i + 1) - m_use);
+                rs += p0 + p1;
+                pk[i / 2] = kFp8 ? pack_f16(p0 * vsc, p1 * vsc) : pack_bf16(p0, p1);
+              }
+            }
+            // P column c/2 lies in an S column already read
+            tmem_st16(tmem + lane_base + colS + cb / 2, pk);
+            tmem_st16(tmem + lane_base + colS + cb / 2 + 16, pk + 16);
+          }
         }
-        l += rs;
+        if (__any_sync(0xffffffffu, alpha != 1.f)) rescale_o<D>(tmem + lane_base + colO, alpha);
+        l = l * alpha + rs;
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -863,8 +912,10 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
   __syncthreads();
   if (warp == kProducerWarp) {
     // no bulk copy may still be landing in shared memory when the CTA exits
-    for (int j = max(0, n_kv - kStages); j < n_kv; ++j)
-      mbar_wait(&kv_full[j % kStages], (uint32_t)((j / kStages) & 1), p.flags);
+    for (int j = max(0, n_kv - kStages); j < n_kv; ++j) {
+      mbar_wait(&k_full[j % kStages], (uint32_t)((j / kStages) & 1), p.flags);
+      mbar_wait(&v_full[j % kStages], (uint32_t)((j / kStages) & 1), p.flags);
+    }
   }
   if (warp == kMmaWarp) {
     mbar_wait(done_bar, 0, p.flags);
@@ -875,7 +926,7 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
 
 template <int D, bool kFp8>
 size_t smem_bytes() {
-  return 1024 + Smem<D, kFp8>::kBytes + (16 + kFactsRing) * sizeof(uint64_t) +
+  return 1024 + Smem<D, kFp8>::kBytes + (20 + kFactsRing) * sizeof(uint64_t) +
          kFactsRing * sizeof(TileFacts) + 32;  // + TMEM base and the item
 }
 

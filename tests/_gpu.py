@@ -117,16 +117,31 @@ class GpuState:
                 self.v_pool.view(torch.uint8).cpu().numpy().reshape(-1))
 
 
+def bf16_half_ulp(x):
+    """Half the bf16 spacing at |x| (8 significant bits): what rounding the exact
+    value to bf16 may cost at best."""
+    _, e = np.frexp(np.abs(x))  # |x| = m * 2^e, m in [0.5, 1)
+    return np.where(x == 0, 0.0, np.ldexp(1.0, e - 9))
+
+
 def compare(out, lse, ref_out, ref_lse, rows=None, max_abs=1e-2, mean_abs=1e-3, lse_abs=2e-3):
-    """bf16 output vs fp64 oracle: max-abs and mean-abs bounds; fp32 lse bound."""
+    """bf16 output vs fp64 oracle; fp32 lse bound.
+
+    Per element |out - ref| <= max_abs + half a bf16 ulp of ref: the bound
+    holds for the computation (P rounding, fp32 sums) and the output's own
+    rounding to bf16 comes on top (at |ref| >= 4 half an ulp alone is 2^-6 >
+    1e-2).  The mean of |out - ref| must stay <= mean_abs.
+    """
     o = out.float().cpu().numpy().astype(np.float64)
     r = ref_out
     if rows is not None:
         o, r = o[rows], r[rows]
     assert np.all(np.isfinite(o)), "non-finite output"
     err = np.abs(o - r)
-    info = f"max_abs={err.max():.3e} mean_abs={err.mean():.3e}"
-    assert err.max() <= max_abs, info
+    excess = err - (max_abs + bf16_half_ulp(r))
+    info = (f"max_abs={err.max():.3e} mean_abs={err.mean():.3e} "
+            f"worst excess over bound={excess.max():.3e}")
+    assert excess.max() <= 0, info
     assert err.mean() <= mean_abs, info
     if lse is not None and ref_lse is not None:
         l = lse.cpu().numpy().astype(np.float64)

@@ -11,7 +11,8 @@ import re
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "paged_kv.h")
+HEADERS = sorted(os.path.join(ROOT, "include", h) for h in os.listdir(os.path.join(ROOT, "include"))
+                 if h.endswith(".h"))
 
 
 @pytest.fixture(scope="module")
@@ -25,7 +26,7 @@ def pkv():
 
 
 def _declared_functions():
-    text = open(HEADER).read()
+    text = "\n".join(open(h).read() for h in HEADERS)
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(\w+)\s*\(", text, flags=re.M)))
 
@@ -41,13 +42,13 @@ def test_library_exports_every_declared_symbol(pkv):
     declared = _declared_functions()
     assert declared, "no declarations parsed"
     for name in declared:
-        assert hasattr(lib, name), f"{name} declared in paged_kv.h but not exported"
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
     assert set(declared) == set(pkv.EXPORTED)
 
 
 def test_status_strings_and_version(pkv):
     assert pkv.pkv_status_string(0) == "ok"
-    for s in range(-11, 0):
+    for s in range(-12, 0):
         assert pkv.pkv_status_string(s) != "unknown status"
     assert pkv.lib().pkv_abi_version() >> 16 == 1
 

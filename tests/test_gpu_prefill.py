@@ -72,6 +72,21 @@ def test_prefill_many_chunks(num_chunks):
     assert int(st.flags.item()) == 0
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_prefill_negative_scale(dtype):
+    # the row max of s * scale is not scale * max(s) when scale < 0
+    w = workloads.build("pfneg", 27, [300, 0], [200, 130], page_size=64, num_q_heads=8,
+                        num_kv_heads=2, head_dim=128, kv_dtype=dtype, pool_slack=0.2,
+                        chunk_rows=[0, 1], softmax_scale=-0.11)
+    st = GpuState(w)
+    st.append_step()
+    out, lse = st.prefill()
+    torch.cuda.synchronize()
+    ref, ref_lse = _oracle_prefill(w)
+    compare(out, lse, ref, ref_lse)
+    assert int(st.flags.item()) == 0
+
+
 def test_prefill_row_equals_truncated_decode():
     # the last query of a chunk sees exactly what a decode step would see
     w = workloads.build("pfd", 22, [300, 50], [70, 9], page_size=64, num_q_heads=8,
