@@ -289,77 +289,136 @@ def run_ours(args, rank, world, device, dist):
         if ev is not None:
             ev[3].record(stream)
 
-    launches_per_step = 1 + (1 if len(w.decode_rows) else 0) + (1 if has_pf else 0)
+    # append; decode_kernel + decode_merge_kernel; prefill_kernel
+    launches_per_step = 1 + (2 if len(w.decode_rows) else 0) + (1 if has_pf else 0)
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize()
     if int(st["flags"].item()) != 0:
         raise RuntimeError(f"device error flags {int(st['flags'].item()):#x}")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    # Eager steps with an event between kernels: the per-kernel times (and
+    # the decode kernel's duration for the roofline) come from here.
+    k_steps = max(1, min(args.steps, 300))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(k_steps)]
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(k_steps):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    eager_s = max_over_ranks(t0.elapsed_time(t1) / 1e3 / k_steps, dist, device)
+    dec_s = sum(e[1].elapsed_time(e[2]) for e in evs) / k_steps / 1e3
+    app_s = sum(e[0].elapsed_time(e[1]) for e in evs) / k_steps / 1e3
+    pf_s = sum(e[2].elapsed_time(e[3]) for e in evs) / k_steps / 1e3
+
+    # The timed steps: the step captured once into a CUDA graph and replayed,
+    # one graph launch per step instead of one launch per kernel (the PDL edge
+    # between the decode kernels is kept by capture).  Same kernels, same
+    # inputs, same work as the eager step.
+    graph = torch.cuda.CUDAGraph()
+    gstream = torch.cuda.Stream()
+    gstream.wait_stream(stream)
+    with torch.cuda.stream(gstream):
+        step()  # warm the caching allocator on the capture stream
+        gstream.synchronize()
+        with torch.cuda.graph(graph, stream=gstream):
+            step()
+    torch.cuda.synchronize()
+    for _ in range(max(3, args.warmup)):
+        graph.replay()
+    torch.cuda.synchronize()
+    if int(st["flags"].item()) != 0:
+        raise RuntimeError(f"device error flags {int(st['flags'].item()):#x}")
+    g0 = torch.cuda.Event(enable_timing=True)
+    g1 = torch.cuda.Event(enable_timing=True)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(device.index if device.index is not None else 0) as clk:
-        t0.record(stream)
-        for i in range(args.steps):
-            step(evs[i])
-        t1.record(stream)
+        g0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        g1.record(stream)
         torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    elapsed = t0.elapsed_time(t1) / 1e3  # seconds
-    dec_s = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps / 1e3
-    app_s = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps / 1e3
-    pf_s = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps / 1e3
-    elapsed = max_over_ranks(elapsed, dist, device)
+    elapsed = max_over_ranks(g0.elapsed_time(g1) / 1e3, dist, device)  # seconds
+    del graph
 
     # ---------------------------------------------------------------- e2e
     # Through the public API with host buffers: per step, H2D of the step's
     # inputs (q, new K/V, lengths, page table) from pinned memory and D2H of
-    # the attention output, all inside the timed region.
+    # the attention output, all inside the timed region.  Inputs and outputs
+    # move on streams of their own with two buffers each, so step i+1's inputs
+    # and step i-1's output cross PCIe while step i's kernels run.
     names = ("dec_q", "k_new", "v_new", "table", "ctx_lens", "dec_lens", "dec_table")
     offs, total = {}, 0
     for k in names:
         offs[k] = total
         total += (st[k].numel() * st[k].element_size() + 255) // 256 * 256
     h_buf = torch.empty(total, dtype=torch.uint8).pin_memory()
-    d_buf = torch.empty(total, dtype=torch.uint8, device=device)
-    d = {}
+    d_bufs = [torch.empty(total, dtype=torch.uint8, device=device) for _ in range(2)]
+    d = [{}, {}]
     for k in names:
         n = st[k].numel() * st[k].element_size()
         h_buf[offs[k]:offs[k] + n].copy_(st[k].contiguous().view(-1).view(torch.uint8).cpu())
-        d[k] = d_buf[offs[k]:offs[k] + n].view(st[k].dtype).view(st[k].shape)
-    h_out = torch.empty(st["dec_out"].shape, dtype=st["dec_out"].dtype).pin_memory()
+        for i in range(2):
+            d[i][k] = d_bufs[i][offs[k]:offs[k] + n].view(st[k].dtype).view(st[k].shape)
+    outs = [torch.empty_like(st["dec_out"]) for _ in range(2)]
+    h_outs = [torch.empty(st["dec_out"].shape, dtype=st["dec_out"].dtype).pin_memory()
+              for _ in range(2)]
+    h2d_stream = torch.cuda.Stream()  # inputs in
+    d2h_stream = torch.cuda.Stream()  # results out
+    h2d_done = [torch.cuda.Event() for _ in range(2)]
+    compute_done = [torch.cuda.Event() for _ in range(2)]
+    d2h_done = [torch.cuda.Event() for _ in range(2)]
     e_steps = max(1, min(args.steps, 200))
 
-    def e2e_step():
-        d_buf.copy_(h_buf, non_blocking=True)  # one H2D copy of every step input
-        pkv.paged_kv_append(cache, d["table"], d["ctx_lens"], st["cu_new"], d["k_new"],
-                            d["v_new"])
-        pkv.paged_decode_attention(cache, d["dec_q"], d["dec_table"], d["dec_lens"], st["dec_max"],
-                                   w.softmax_scale, out=st["dec_out"], lse=st["dec_lse"],
+    def e2e_step(i):
+        b = i & 1
+        with torch.cuda.stream(h2d_stream):
+            if i >= 2:
+                h2d_stream.wait_event(compute_done[b])  # step i-2 is done reading buffer b
+            d_bufs[b].copy_(h_buf, non_blocking=True)  # one H2D copy of every step input
+            h2d_done[b].record(h2d_stream)
+        stream.wait_event(h2d_done[b])
+        if i >= 2:
+            stream.wait_event(d2h_done[b])  # step i-2's output has left outs[b]
+        db = d[b]
+        pkv.paged_kv_append(cache, db["table"], db["ctx_lens"], st["cu_new"], db["k_new"],
+                            db["v_new"])
+        pkv.paged_decode_attention(cache, db["dec_q"], db["dec_table"], db["dec_lens"],
+                                   st["dec_max"], w.softmax_scale, out=outs[b], lse=st["dec_lse"],
                                    workspace=ws, num_ctas=args.num_ctas)
-        h_out.copy_(st["dec_out"], non_blocking=True)
+        compute_done[b].record(stream)
+        with torch.cuda.stream(d2h_stream):
+            d2h_stream.wait_event(compute_done[b])
+            h_outs[b].copy_(outs[b], non_blocking=True)  # D2H of the step's result
+            d2h_done[b].record(d2h_stream)
 
-    for _ in range(3):
-        e2e_step()
+    def e2e_run(n):
+        for i in range(n):
+            e2e_step(i)
+        stream.wait_stream(d2h_stream)
+
+    e2e_run(3)
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e_steps):
-        e2e_step()
+    h2d_stream.wait_event(e0)
+    e2e_run(e_steps)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_s = e0.elapsed_time(e1) / 1e3 / e_steps
     e2e_s = max_over_ranks(e2e_s, dist, device)
     h2d = sum(st[k].numel() * st[k].element_size() for k in names)
-    d2h = h_out.numel() * h_out.element_size()
+    d2h = h_outs[0].numel() * h_outs[0].element_size()
 
     flags = int(st["flags"].item())
     step_bytes = decode_bytes(w) + append_bytes(w)
@@ -410,7 +469,14 @@ def run_ours(args, rank, world, device, dist):
         },
         "e2e": {"value": round(whole_job_rate(step_bytes, world, e2e_s) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                "ms_per_step": round(e2e_s * 1e3, 5)},
+                "ms_per_step": round(e2e_s * 1e3, 5),
+                "mode": "eager API calls (append + decode) per step; H2D of step i+1 and "
+                        "D2H of step i-1 on their own streams, overlapping step i's kernels"},
+        "timing": "the step (append + decode [+ prefill]) captured once in a CUDA graph and "
+                  "replayed per step; kernels_ms from eager steps with events between kernels",
+        "eager": {"value": round(whole_job_rate(step_bytes, world, eager_s) / 1e9, 2),
+                  "unit": "GB/s", "ms_per_step": round(eager_s * 1e3, 5),
+                  "what": "the same step as separate launches"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
         "device_error_flags": flags,
