@@ -18,6 +18,8 @@ Functions and what they follow (pages on TensorRT-LLM):
                       split-KV decode formula; no counterpart on the pages)
 * ``e4m3_*`` / ``fp8_quantize``    E4M3 codec from the format definition
                       (yololab.net guide, "FP8 與極致量化")
+* ``int8_*``          symmetric INT8 codec (concept page, "關鍵機制"
+                      quantisation bullet: INT8 KV cache)
 
 Every function is pinned by ``tests/test_oracle_*.py`` against brute force,
 library special cases, closed forms and invariants.
@@ -38,6 +40,7 @@ _LIB = os.path.join(_BUILD, "liboracle.so")
 
 KV_BF16 = 0
 KV_E4M3 = 1
+KV_INT8 = 2
 
 _lib = None
 
@@ -81,6 +84,9 @@ def _declare(L):
     L.oracle_e4m3_encode_array.argtypes = [_P, _P, _I64]
     L.oracle_e4m3_decode_array.argtypes = [_P, _P, _I64]
     L.oracle_fp8_quantize_array.argtypes = [_P, _P, _P, _I64]
+    L.oracle_int8_encode.argtypes = [_F]
+    L.oracle_int8_encode.restype = ctypes.c_int8
+    L.oracle_int8_quantize_array.argtypes = [_P, _P, _P, _I64]
     cache = [_P, _P, _P, _P, _I, _I, _I, _I, _I]
     L.oracle_append.argtypes = cache + [_P, _I, _P, _P, _I, _P, _P]
     L.oracle_append.restype = _I
@@ -138,6 +144,21 @@ def fp8_quantize(x_bits, scale) -> np.ndarray:
     return out
 
 
+def int8_encode(y) -> np.ndarray:
+    """INT8 codes of fp32 values: nearest integer (ties to even) clamped to +-127, NaN -> 0."""
+    y = _c(y, np.float32).reshape(-1)
+    return np.array([lib().oracle_int8_encode(float(v)) for v in y], np.int8)
+
+
+def int8_quantize(x_bits, scale) -> np.ndarray:
+    """INT8 codes of bf16 values (given as uint16 bits) divided by fp32 scales."""
+    x_bits = _c(x_bits, np.uint16)
+    scale = _c(np.broadcast_to(scale, x_bits.shape), np.float32)
+    out = np.empty(x_bits.shape, np.int8)
+    lib().oracle_int8_quantize_array(_ptr(x_bits), _ptr(scale), _ptr(out), x_bits.size)
+    return out
+
+
 # ------------------------------------------------------------------- cache
 class Cache:
     """A host KV pool image: K and V byte pools ``[pages][Hkv][P][D]`` plus scales."""
@@ -149,8 +170,8 @@ class Cache:
         self.num_kv_heads = int(num_kv_heads)
         self.head_dim = int(head_dim)
         self.kv_dtype = kv_dtype
-        self.code = KV_E4M3 if kv_dtype == "e4m3" else KV_BF16
-        eb = 1 if self.code == KV_E4M3 else 2
+        self.code = {"bf16": KV_BF16, "e4m3": KV_E4M3, "int8": KV_INT8}[kv_dtype]
+        eb = 2 if self.code == KV_BF16 else 1
         nbytes = self.num_pages * self.num_kv_heads * self.page_size * self.head_dim * eb
         self.k_pool = _c(k_pool, np.uint8) if k_pool is not None else np.zeros(nbytes, np.uint8)
         self.v_pool = _c(v_pool, np.uint8) if v_pool is not None else np.zeros(nbytes, np.uint8)
@@ -251,12 +272,12 @@ def cache_for(w, seq_ids=None, include_new=True) -> Cache:
     ``Cache.append`` with the workload's page table; all other bytes keep the
     NaN sentinel.  ``include_new=False`` stores only the context tokens.
     """
-    from workloads import BF16_NAN_BITS, E4M3_NAN_CODE
+    from workloads import BF16_NAN_BITS, sentinel_byte
 
     seq_ids = range(w.batch) if seq_ids is None else list(seq_ids)
-    if w.kv_dtype == "e4m3":
-        k_pool = np.full(w.pool_bytes(), E4M3_NAN_CODE, np.uint8)
-        v_pool = np.full(w.pool_bytes(), E4M3_NAN_CODE, np.uint8)
+    if w.kv_dtype != "bf16":
+        k_pool = np.full(w.pool_bytes(), sentinel_byte(w.kv_dtype), np.uint8)
+        v_pool = np.full(w.pool_bytes(), sentinel_byte(w.kv_dtype), np.uint8)
         k_scale = np.ones((w.num_pages, w.num_kv_heads), np.float32)
         v_scale = np.ones((w.num_pages, w.num_kv_heads), np.float32)
     else:
@@ -267,7 +288,7 @@ def cache_for(w, seq_ids=None, include_new=True) -> Cache:
               k_pool, v_pool, k_scale, v_scale)
     for b in seq_ids:
         k, v = w.kv_seq(b)
-        if w.kv_dtype == "e4m3":
+        if w.kv_dtype != "bf16":
             pages, ks, vs = w.kv_scales_for(b, k, v)
             c.k_scale[pages] = ks
             c.v_scale[pages] = vs

@@ -37,6 +37,10 @@
  *  - FP8: E4M3 (bias 7, no infinities, 0x7F/0xFF NaN, max 448) with one fp32
  *    scale per (page, kv head) for K and one for V; stored code =
  *    e4m3_rne_satfinite(fp32(x) / scale); value = decode(code) * scale;
+ *  - INT8 (the concept page's INT8 KV-cache quantisation, "關鍵機制"
+ *    quantisation bullet): the same per-(page, kv head) scales; stored code =
+ *    round-half-even of the fp32 quotient clamped to [-127, 127] (-128 never
+ *    stored), NaN -> 0; value = code * scale;
  *  - a sequence of length 0 yields out = 0 and lse = -inf.
  */
 #include <math.h>
@@ -55,6 +59,7 @@
 
 #define KV_BF16 0
 #define KV_E4M3 1
+#define KV_INT8 2
 
 int oracle_num_threads(void) {
 #ifdef _OPENMP
@@ -150,6 +155,28 @@ uint8_t oracle_fp8_quantize(uint16_t x_bits, float scale) {
   return oracle_e4m3_encode(oracle_fp8_quotient(x_bits, scale));
 }
 
+/* ------------------------------------------------------------------ INT8 */
+/*
+ * Symmetric INT8: the nearest integer to y, ties to even, clamped to
+ * [-127, 127] (so -128 is never produced and +-inf give +-127); NaN gives 0.
+ */
+int8_t oracle_int8_encode(float y) {
+  if (isnan(y)) return 0;
+  double a = (double)y;
+  if (a > 127.0) a = 127.0;
+  if (a < -127.0) a = -127.0;
+  return (int8_t)nearbyint(a); /* default rounding: nearest, ties to even */
+}
+
+int8_t oracle_int8_quantize(uint16_t x_bits, float scale) {
+  return oracle_int8_encode(oracle_fp8_quotient(x_bits, scale));
+}
+
+void oracle_int8_quantize_array(const uint16_t* x_bits, const float* scale, int8_t* codes,
+                                int64_t n) {
+  for (int64_t i = 0; i < n; ++i) codes[i] = oracle_int8_quantize(x_bits[i], scale[i]);
+}
+
 /* Array helpers for exhaustive codec checks. */
 void oracle_e4m3_encode_array(const float* y, uint8_t* codes, int64_t n) {
   for (int64_t i = 0; i < n; ++i) codes[i] = oracle_e4m3_encode(y[i]);
@@ -168,7 +195,7 @@ void oracle_fp8_quantize_array(const uint16_t* x_bits, const float* scale, uint8
 typedef struct {
   uint8_t* k_pool;
   uint8_t* v_pool;
-  const float* k_scale; /* [num_pages][num_kv_heads], E4M3 only */
+  const float* k_scale; /* [num_pages][num_kv_heads], E4M3 and INT8 only */
   const float* v_scale;
   int kv_dtype;
   int num_pages;
@@ -177,7 +204,7 @@ typedef struct {
   int head_dim;
 } cache_t;
 
-static int elem_bytes(int kv_dtype) { return kv_dtype == KV_E4M3 ? 1 : 2; }
+static int elem_bytes(int kv_dtype) { return kv_dtype == KV_BF16 ? 2 : 1; }
 
 /* Byte offset of element (page, kv head, slot, d) in a pool. */
 static int64_t pool_offset(const cache_t* c, int64_t page, int g, int slot, int d) {
@@ -202,6 +229,8 @@ static double stored_value(const cache_t* c, const uint8_t* pool, const float* s
   int64_t off = pool_offset(c, page, g, slot, d);
   if (c->kv_dtype == KV_E4M3)
     return oracle_e4m3_decode(pool[off]) * (double)scale[page * c->num_kv_heads + g];
+  if (c->kv_dtype == KV_INT8)
+    return (double)(int8_t)pool[off] * (double)scale[page * c->num_kv_heads + g];
   uint16_t bits;
   memcpy(&bits, pool + off, 2);
   return bf16_value(bits);
@@ -209,8 +238,9 @@ static double stored_value(const cache_t* c, const uint8_t* pool, const float* s
 
 static int check_cache(const cache_t* c) {
   if (!c->k_pool || !c->v_pool) return ORC_ERR_ARG;
-  if (c->kv_dtype != KV_BF16 && c->kv_dtype != KV_E4M3) return ORC_ERR_ARG;
-  if (c->kv_dtype == KV_E4M3 && (!c->k_scale || !c->v_scale)) return ORC_ERR_ARG;
+  if (c->kv_dtype != KV_BF16 && c->kv_dtype != KV_E4M3 && c->kv_dtype != KV_INT8)
+    return ORC_ERR_ARG;
+  if (c->kv_dtype != KV_BF16 && (!c->k_scale || !c->v_scale)) return ORC_ERR_ARG;
   if (c->num_pages < 0 || c->page_size <= 0 || c->num_kv_heads <= 0 || c->head_dim <= 0)
     return ORC_ERR_ARG;
   return ORC_OK;
@@ -220,7 +250,8 @@ static int check_cache(const cache_t* c) {
 /*
  * Paged KV store.  New token j of sequence b sits at logical position
  * pos = seq_lens_before[b] + j; its page is page_table[b][pos / P] and its
- * slot pos % P.  bf16 stores the input bits; E4M3 stores the quantised code.
+ * slot pos % P.  bf16 stores the input bits; E4M3 and INT8 store the
+ * quantised code.
  * k_new/v_new: bf16 bits [total_new][num_kv_heads][head_dim], ordered by
  * sequence through cu_new [batch+1].
  */
@@ -251,6 +282,11 @@ int oracle_append(uint8_t* k_pool, uint8_t* v_pool, const float* k_scale, const 
             float vs = v_scale[page * num_kv_heads + g];
             k_pool[off] = oracle_fp8_quantize(k_new[src], ks);
             v_pool[off] = oracle_fp8_quantize(v_new[src], vs);
+          } else if (kv_dtype == KV_INT8) {
+            float ks = k_scale[page * num_kv_heads + g];
+            float vs = v_scale[page * num_kv_heads + g];
+            k_pool[off] = (uint8_t)oracle_int8_quantize(k_new[src], ks);
+            v_pool[off] = (uint8_t)oracle_int8_quantize(v_new[src], vs);
           } else {
             memcpy(k_pool + off, &k_new[src], 2);
             memcpy(v_pool + off, &v_new[src], 2);

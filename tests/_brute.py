@@ -33,6 +33,9 @@ def element(cache, pool, scales, page, g, slot, d) -> float:
     idx = ((page * H + g) * P + slot) * D + d
     if cache.kv_dtype == "e4m3":
         return e4m3_to_float(pool[idx]) * float(scales[page, g])
+    if cache.kv_dtype == "int8":  # two's-complement byte times the scale
+        code = int(pool[idx])
+        return float(code - 256 if code > 127 else code) * float(scales[page, g])
     lo, hi = int(pool[2 * idx]), int(pool[2 * idx + 1])
     return bf16_to_float(lo | (hi << 8))
 

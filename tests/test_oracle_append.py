@@ -71,7 +71,31 @@ def test_e4m3_append_matches_library_quantisation():
     assert np.all(vp[untouched] == workloads.E4M3_NAN_CODE)
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_int8_append_matches_library_rounding():
+    w = workloads.build("a", 7, [0, 17, 64], [1, 1, 65], page_size=16, num_q_heads=8,
+                        num_kv_heads=2, head_dim=32, kv_dtype="int8", pool_slack=0.2)
+    c = oracle.cache_for(w)
+    shape = (w.num_pages, w.num_kv_heads, w.page_size, w.head_dim)
+    kp = c.k_pool.view(np.int8).reshape(shape)
+    vp = c.v_pool.view(np.int8).reshape(shape)
+    P = w.page_size
+    for b in range(w.batch):
+        k, v = w.kv_seq(b)
+        t = np.arange(int(w.lens_after[b]))
+        pages = w.page_table[b, t // P]
+        for pool, src, sc in ((kp, k, c.k_scale), (vp, v, c.v_scale)):
+            s = sc[pages][:, :, None]  # [n, Hkv, 1]
+            y = (src.float().numpy() / s).astype(np.float32)  # IEEE fp32 quotient
+            ref = np.clip(np.rint(y), -127, 127).astype(np.int8)  # ties to even
+            assert np.array_equal(pool[pages, :, t % P, :], ref)
+            # absmax / 127 scales: the largest magnitude of each page lands on 127
+            assert np.abs(y).max() <= 127.0 * (1 + 2**-20)
+    untouched = ~_written_mask(w, lambda b: int(w.lens_after[b]))
+    assert np.all(c.k_pool.reshape(shape)[untouched] == workloads.INT8_UNOWNED)
+    assert np.all(c.v_pool.reshape(shape)[untouched] == workloads.INT8_UNOWNED)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3", "int8"])
 def test_context_then_new_equals_one_append(dtype):
     w = workloads.build("a", 5, [3, 8, 0], [1, 5, 9], page_size=4, num_q_heads=2,
                         num_kv_heads=1, head_dim=8, kv_dtype=dtype, pool_slack=0.5)

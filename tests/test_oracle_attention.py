@@ -50,6 +50,9 @@ def _contiguous_kv(w, c, b, n):
             vals = torch.from_numpy(pool.copy()).view(torch.float8_e4m3fn).to(torch.float64)
             vals = vals.numpy().reshape(shape)
             x = vals[pages, :, slots, :] * scale[pages][:, :, None].astype(np.float64)
+        elif w.kv_dtype == "int8":
+            vals = pool.view(np.int8).astype(np.float64).reshape(shape)
+            x = vals[pages, :, slots, :] * scale[pages][:, :, None].astype(np.float64)
         else:
             bits = pool.view(np.uint16).astype(np.uint32) << 16
             vals = bits.view(np.float32).astype(np.float64).reshape(shape)
@@ -71,7 +74,7 @@ def _sdpa(q, K, V, scale, mask=None):
 
 
 # ------------------------------------------------------------ brute force
-@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3", "int8"])
 def test_decode_matches_brute_force(dtype):
     w, c = _tiny(1, [0, 3, 4, 9], [1, 1, 1, 1], dtype=dtype)
     q = _q_bits((4, 4, 8), 11)
@@ -81,7 +84,7 @@ def test_decode_matches_brute_force(dtype):
     np.testing.assert_allclose(lse, bl, rtol=0, atol=1e-12)
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3", "int8"])
 def test_prefill_matches_brute_force(dtype):
     w, c = _tiny(2, [0, 5, 2], [3, 4, 6], dtype=dtype, chunk_rows=[0, 1, 2], Hq=2, Hkv=1)
     q = _q_bits((13, 2, 8), 12)
@@ -93,7 +96,7 @@ def test_prefill_matches_brute_force(dtype):
 
 
 # -------------------------------------------------- library special case
-@pytest.mark.parametrize("dtype,G", [("bf16", 4), ("bf16", 1), ("e4m3", 8)])
+@pytest.mark.parametrize("dtype,G", [("bf16", 4), ("bf16", 1), ("e4m3", 8), ("int8", 8)])
 def test_decode_matches_torch_sdpa(dtype, G):
     Hkv = 2
     w, c = _tiny(3, [5, 40, 63, 64, 100], [1] * 5, P=16, Hq=Hkv * G, Hkv=Hkv, D=32, dtype=dtype)
@@ -112,7 +115,7 @@ def test_decode_matches_torch_sdpa(dtype, G):
         np.testing.assert_allclose(lse[b], ref_lse, rtol=0, atol=1e-12)
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3", "int8"])
 def test_prefill_matches_torch_sdpa_bottom_right_causal(dtype):
     Hkv, G, D = 2, 2, 16
     w, c = _tiny(4, [0, 7, 30], [9, 16, 5], P=8, Hq=Hkv * G, Hkv=Hkv, D=D, dtype=dtype,
@@ -254,7 +257,7 @@ def test_gqa_equals_mha_with_duplicated_kv_heads():
     assert np.array_equal(og, om) and np.array_equal(lg, lm)
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3", "int8"])
 def test_chunk_rows_equal_truncated_decode(dtype):
     w, c = _tiny(23, [5, 0], [6, 1], P=4, dtype=dtype, chunk_rows=[0, 1])
     T = int(w.new_lens.sum())

@@ -100,3 +100,45 @@ def test_roundtrip_every_finite_code():
     codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
     vals = oracle.e4m3_decode(codes).astype(np.float32)
     assert np.array_equal(oracle.e4m3_encode(vals), codes)
+
+
+# ------------------------------------------------------------------- INT8
+# Symmetric INT8 KV codes (concept page, "關鍵機制" quantisation bullet):
+# nearest integer of the fp32 quotient, ties to even, clamped to +-127.
+GOLDEN_INT8 = os.path.join(os.path.dirname(__file__), "golden", "int8_points.txt")
+
+
+def test_int8_golden_points():
+    pts = []
+    for line in open(GOLDEN_INT8):
+        line = line.strip()
+        if line and not line.startswith("#"):
+            val, code, *_ = line.split()
+            pts.append((np.float32(float(val)), int(code)))
+    assert len(pts) >= 12
+    got = oracle.int8_encode(np.array([v for v, _ in pts], np.float32))
+    assert got.tolist() == [c for _, c in pts]
+
+
+@pytest.mark.parametrize("scale", [1.0, 0.37, 2.0**-4, 0.01])
+def test_int8_quantize_exhaustive_bf16_vs_numpy(scale):
+    # Library route: IEEE fp32 quotient, numpy's rint (round half to even),
+    # clip to the symmetric range.
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    x = (bits.astype(np.uint32) << 16).view(np.float32)
+    finite = np.isfinite(x)
+    bits, x = bits[finite], x[finite]
+    codes = oracle.int8_quantize(bits, np.float32(scale))
+    with np.errstate(over="ignore"):
+        y = (x / np.float32(scale)).astype(np.float32)
+    ref = np.clip(np.rint(y.astype(np.float64)), -127, 127).astype(np.int8)
+    assert np.array_equal(codes, ref)
+    assert codes.min() >= -127  # -128 never stored
+
+
+def test_int8_specials():
+    c = oracle.int8_encode(np.array([np.inf, -np.inf, np.nan], np.float32))
+    assert c.tolist() == [127, -127, 0]
+    # every code round-trips through its value
+    vals = np.arange(-127, 128, dtype=np.float32)
+    assert oracle.int8_encode(vals).tolist() == list(range(-127, 128))

@@ -45,6 +45,20 @@ import torch
 BF16_NAN_BITS = 0x7FC0
 E4M3_NAN_CODE = 0x7F
 E4M3_MAX = 448.0
+# INT8 pools: -128 is never stored (codes are clamped to +-127), so it marks
+# bytes no sequence owns.
+INT8_UNOWNED = 0x80
+INT8_MAX = 127.0
+
+
+def sentinel_byte(kv_dtype: str) -> int:
+    """Fill byte of unowned pool bytes of an 8-bit pool."""
+    return {"e4m3": E4M3_NAN_CODE, "int8": INT8_UNOWNED}[kv_dtype]
+
+
+def code_max(kv_dtype: str) -> float:
+    """Largest stored magnitude of an 8-bit format (the scale divisor)."""
+    return {"e4m3": E4M3_MAX, "int8": INT8_MAX}[kv_dtype]
 
 _STREAM_KV = 1
 _STREAM_QDEC = 2
@@ -76,7 +90,7 @@ class Workload:
     num_q_heads: int
     num_kv_heads: int
     head_dim: int
-    kv_dtype: str  # "bf16" or "e4m3"
+    kv_dtype: str  # "bf16", "e4m3" or "int8"
     ctx_lens: np.ndarray  # int32 [B], tokens already cached
     new_lens: np.ndarray  # int32 [B], tokens appended this step
     num_pages: int
@@ -104,7 +118,7 @@ class Workload:
 
     @property
     def elem_bytes(self) -> int:
-        return 1 if self.kv_dtype == "e4m3" else 2
+        return 2 if self.kv_dtype == "bf16" else 1
 
     def cu_new(self) -> np.ndarray:
         return np.concatenate([[0], np.cumsum(self.new_lens)]).astype(np.int32)
@@ -158,7 +172,8 @@ class Workload:
 
     # ------------------------------------------------------ FP8 scale policy
     def kv_scales_for(self, b: int, k: torch.Tensor = None, v: torch.Tensor = None):
-        """Per-(page, kv head) scales of sequence ``b``: absmax/448 in fp32.
+        """Per-(page, kv head) scales of sequence ``b``: absmax/448 (E4M3) or
+        absmax/127 (INT8) in fp32.
 
         The absmax runs over every element the page will hold after this
         step's append, so no stored value saturates.  Returns
@@ -175,8 +190,8 @@ class Workload:
             lo, hi = j * P, min((j + 1) * P, n)
             ka = k[lo:hi].float().abs().amax(dim=(0, 2)).numpy().astype(np.float32)
             va = v[lo:hi].float().abs().amax(dim=(0, 2)).numpy().astype(np.float32)
-            ks[j] = ka / np.float32(E4M3_MAX)
-            vs[j] = va / np.float32(E4M3_MAX)
+            ks[j] = ka / np.float32(code_max(self.kv_dtype))
+            vs[j] = va / np.float32(code_max(self.kv_dtype))
         tiny = np.float32(2.0**-126)
         return pages, np.maximum(ks, tiny), np.maximum(vs, tiny)
 
@@ -336,6 +351,6 @@ def config(n: int, seed: Optional[int] = None) -> Workload:
 
 def empty_pool(w: Workload) -> np.ndarray:
     """Host pool image (uint8 view) filled with the NaN sentinel of its dtype."""
-    if w.kv_dtype == "e4m3":
-        return np.full(w.pool_bytes(), E4M3_NAN_CODE, dtype=np.uint8)
+    if w.kv_dtype != "bf16":
+        return np.full(w.pool_bytes(), sentinel_byte(w.kv_dtype), dtype=np.uint8)
     return np.full(w.pool_bytes() // 2, BF16_NAN_BITS, dtype=np.uint16).view(np.uint8)
