@@ -8,7 +8,7 @@ U[128,4096], page size 64, 32 q / 8 kv heads, head_dim 128, bf16).  Inputs are
 seeded synthetic data resident in HBM; the KV pool (~0.55 GB) exceeds the
 126 MB L2, so no flush is needed between steps.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..5]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..6]
     python bench.py --impl reference ...   # the CPU oracle on the host cores
 
 Prints ONE JSON line (rank 0).  ``value`` is whole-job achieved HBM GB/s of
@@ -115,7 +115,7 @@ def decode_bytes(w, rows=None) -> int:
     P = w.page_size
     kv = int(la.sum()) * w.num_kv_heads * w.head_dim * 2 * w.elem_bytes
     pages = int(((la + P - 1) // P).sum())
-    scales = pages * w.num_kv_heads * 2 * 4 if w.kv_dtype == "e4m3" else 0
+    scales = pages * w.num_kv_heads * 2 * 4 if w.kv_dtype != "bf16" else 0
     qo = 2 * len(rows) * w.num_q_heads * w.head_dim * 2
     return kv + scales + qo + pages * 4
 
@@ -200,9 +200,10 @@ def setup_device_state(w, device):
     import workloads
 
     shape = w.pool_shape()
-    if w.kv_dtype == "e4m3":
-        k_pool = torch.full(shape, workloads.E4M3_NAN_CODE, dtype=torch.uint8, device=device)
-        v_pool = torch.full(shape, workloads.E4M3_NAN_CODE, dtype=torch.uint8, device=device)
+    if w.kv_dtype != "bf16":
+        fill = workloads.sentinel_byte(w.kv_dtype)
+        k_pool = torch.full(shape, fill, dtype=torch.uint8, device=device)
+        v_pool = torch.full(shape, fill, dtype=torch.uint8, device=device)
         k_scale = torch.ones((w.num_pages, w.num_kv_heads), dtype=torch.float32, device=device)
         v_scale = torch.ones_like(k_scale)
     else:
@@ -218,7 +219,7 @@ def setup_device_state(w, device):
     for b in range(w.batch):
         k, v = w.kv_seq(b)
         c = int(w.ctx_lens[b])
-        if w.kv_dtype == "e4m3":
+        if w.kv_dtype != "bf16":
             pages, ks, vs = w.kv_scales_for(b, k, v)
             idx = torch.from_numpy(pages.astype(np.int64)).to(device)
             k_scale[idx] = torch.from_numpy(ks).to(device)
@@ -437,7 +438,7 @@ def run_ours(args, rank, world, device, dist):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16" if w.kv_dtype == "bf16" else "e4m3-kv/bf16-q",
+        "dtype": "bf16" if w.kv_dtype == "bf16" else f"{w.kv_dtype}-kv/bf16-q",
         "data": "synthetic (seeded N(0,1) bf16 K/V/Q, permuted pages, NaN sentinels)",
         "tokens_per_s": round(whole_job_rate(len(w.decode_rows), world, step_s), 1),
         "config": {

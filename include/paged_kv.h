@@ -69,7 +69,7 @@ typedef enum {
   PKV_ERR_NO_PAGES = -12     /* the free pages cannot cover a growth (paged_kv_runtime.h) */
 } pkv_status;
 
-typedef enum { PKV_KV_BF16 = 0, PKV_KV_FP8_E4M3 = 1 } pkv_kv_dtype;
+typedef enum { PKV_KV_BF16 = 0, PKV_KV_FP8_E4M3 = 1, PKV_KV_INT8 = 2 } pkv_kv_dtype;
 
 /* Device-side error bits OR-ed into pkv_cache.error_flags. */
 #define PKV_FLAG_BAD_PAGE 0x1    /* a page-table entry outside [0, num_pages) */

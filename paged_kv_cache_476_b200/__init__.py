@@ -28,6 +28,8 @@ LIB_PATH = os.path.join(_PKG, "libpagedkv.so")
 
 PKV_KV_BF16 = 0
 PKV_KV_FP8_E4M3 = 1
+PKV_KV_INT8 = 2
+_KV_CODES = {"bf16": PKV_KV_BF16, "e4m3": PKV_KV_FP8_E4M3, "int8": PKV_KV_INT8}
 PKV_FLAG_BAD_PAGE = 0x1
 PKV_FLAG_BAD_LENGTH = 0x2
 PKV_FLAG_TIMEOUT = 0x4
@@ -189,24 +191,26 @@ def _stream(stream) -> ctypes.c_void_p:
 class PagedKVCache:
     """Caller-owned paged KV pool: K and V ``[num_pages, Hkv, page_size, head_dim]``.
 
-    ``kv_dtype`` is ``"bf16"`` (torch.bfloat16 pools) or ``"e4m3"`` (uint8 or
-    float8_e4m3fn pools plus fp32 ``k_scale``/``v_scale`` ``[num_pages, Hkv]``).
+    ``kv_dtype`` is ``"bf16"`` (torch.bfloat16 pools), ``"e4m3"`` (uint8 or
+    float8_e4m3fn pools) or ``"int8"`` (int8 or uint8 pools); the one-byte
+    formats take fp32 ``k_scale``/``v_scale`` ``[num_pages, Hkv]``.
     ``error_flags`` is an optional int32 device scalar that kernels OR
     ``PKV_FLAG_*`` bits into.
     """
 
     def __init__(self, k_pool, v_pool, kv_dtype="bf16", k_scale=None, v_scale=None,
                  error_flags=None):
-        if kv_dtype not in ("bf16", "e4m3"):
-            raise ValueError("kv_dtype must be 'bf16' or 'e4m3'")
-        dt = torch.bfloat16 if kv_dtype == "bf16" else (torch.uint8, torch.float8_e4m3fn)
+        if kv_dtype not in _KV_CODES:
+            raise ValueError("kv_dtype must be 'bf16', 'e4m3' or 'int8'")
+        dt = {"bf16": torch.bfloat16, "e4m3": (torch.uint8, torch.float8_e4m3fn),
+              "int8": (torch.int8, torch.uint8)}[kv_dtype]
         _dev("k_pool", k_pool, dt, 4)
         _dev("v_pool", v_pool, dt, 4)
         if k_pool.shape != v_pool.shape:
             raise ValueError("k_pool and v_pool shapes differ")
-        if kv_dtype == "e4m3":
+        if kv_dtype != "bf16":
             if k_scale is None or v_scale is None:
-                raise ValueError("E4M3 pools need k_scale and v_scale")
+                raise ValueError("one-byte pools need k_scale and v_scale")
             _dev("k_scale", k_scale, torch.float32, 2)
             _dev("v_scale", v_scale, torch.float32, 2)
         if error_flags is not None:
@@ -220,7 +224,7 @@ class PagedKVCache:
                            None if k_scale is None else k_scale.data_ptr(),
                            None if v_scale is None else v_scale.data_ptr(),
                            self.num_pages, self.page_size, self.num_kv_heads, self.head_dim,
-                           PKV_KV_FP8_E4M3 if kv_dtype == "e4m3" else PKV_KV_BF16,
+                           _KV_CODES[kv_dtype],
                            None if error_flags is None else error_flags.data_ptr())
 
     @property

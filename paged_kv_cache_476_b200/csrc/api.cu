@@ -34,8 +34,10 @@ int check_cache(const pkv_cache* c) {
   if (c->num_pages < 1 || c->num_kv_heads < 1) return PKV_ERR_SHAPE;
   if (c->page_size != 64 && c->page_size != 128) return PKV_ERR_PAGE_SIZE;
   if (c->head_dim != 64 && c->head_dim != 128) return PKV_ERR_HEAD_DIM;
-  if (c->kv_dtype != PKV_KV_BF16 && c->kv_dtype != PKV_KV_FP8_E4M3) return PKV_ERR_DTYPE;
-  if (c->kv_dtype == PKV_KV_FP8_E4M3 && (!c->k_scale || !c->v_scale)) return PKV_ERR_DTYPE;
+  if (c->kv_dtype != PKV_KV_BF16 && c->kv_dtype != PKV_KV_FP8_E4M3 &&
+      c->kv_dtype != PKV_KV_INT8)
+    return PKV_ERR_DTYPE;
+  if (c->kv_dtype != PKV_KV_BF16 && (!c->k_scale || !c->v_scale)) return PKV_ERR_DTYPE;
   // pool rows (pages * heads * page_size) index a TMA tensor: keep them in int32
   const long long rows = (long long)c->num_pages * c->num_kv_heads * c->page_size;
   if (rows >= INT_MAX) return PKV_ERR_SHAPE;
@@ -87,14 +89,14 @@ int encode_pool_map(CUtensorMap* map, void* base, bool fp8, int64_t rows, int ro
   return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_CUDA;
 }
 
-static int decode_ctas_per_sm(int head_dim, bool fp8, int group, int* out) {
+static int decode_ctas_per_sm(int head_dim, int fmt, int group, int* out) {
   // cached per variant: the occupancy of a kernel does not change at run time
-  static int cache[2][2][4] = {};
+  static int cache[2][3][4] = {};
   const int gi = group == 1 ? 0 : group == 2 ? 1 : group == 4 ? 2 : 3;
-  int& slot = cache[head_dim == 128][fp8][gi];
+  int& slot = cache[head_dim == 128][fmt][gi];
   if (slot == 0) {
     int n = 0;
-    if (decode_occupancy(head_dim, fp8, group, &n) != cudaSuccess || n < 1) return PKV_ERR_CUDA;
+    if (decode_occupancy(head_dim, fmt, group, &n) != cudaSuccess || n < 1) return PKV_ERR_CUDA;
     slot = n;
   }
   *out = slot;
@@ -162,8 +164,7 @@ int paged_kv_append(const pkv_cache* cache, const int32_t* page_table, int32_t m
   p.page_size = cache->page_size;
   p.num_kv_heads = cache->num_kv_heads;
   p.head_dim = cache->head_dim;
-  cudaError_t e = launch_append(p, cache->kv_dtype == PKV_KV_FP8_E4M3, sms,
-                                static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_append(p, cache->kv_dtype, sms, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
@@ -225,10 +226,11 @@ int paged_decode_attention(const pkv_cache* cache, const void* q, int32_t num_q_
   if (need == 0) return PKV_ERR_CUDA;
   if (!workspace || !aligned16(workspace) || workspace_bytes < need) return PKV_ERR_WORKSPACE;
 
-  const bool fp8 = cache->kv_dtype == PKV_KV_FP8_E4M3;
+  const int fmt = cache->kv_dtype;
+  const bool fp8 = k8(fmt);  // one-byte codes (E4M3 or INT8)
   int sms = 0, per_sm = 0;
   if ((st = device_sms(&sms))) return st;
-  if ((st = decode_ctas_per_sm(cache->head_dim, fp8, gqa_group, &per_sm))) return st;
+  if ((st = decode_ctas_per_sm(cache->head_dim, fmt, gqa_group, &per_sm))) return st;
   if (per_sm > kMaxDecodeCtasPerSm) per_sm = kMaxDecodeCtasPerSm;
   int32_t ctas = 0;
   if ((st = paged_decode_plan(batch, cache->num_kv_heads, max_seq_len, sms, num_ctas, per_sm,
@@ -277,7 +279,7 @@ int paged_decode_attention(const pkv_cache* cache, const void* q, int32_t num_q_
   p.num_pages = cache->num_pages;
   p.page_size = cache->page_size;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
-  cudaError_t e = decode_run(D, fp8, tk, tv, p, ctas, static_cast<cudaStream_t>(stream));
+  cudaError_t e = decode_run(D, fmt, tk, tv, p, ctas, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 

@@ -8,7 +8,9 @@
 // loads are coalesced over [token][kv head][d]; each warp writes whole
 // 16-byte chunks of a contiguous page row.  bf16 pools receive the bits;
 // E4M3 pools receive e4m3_rne_satfinite(x / scale) computed with an IEEE
-// fp32 division and the hardware satfinite conversion.
+// fp32 division and the hardware satfinite conversion; INT8 pools receive the
+// nearest integer (ties to even) of the same quotient clamped to +-127, NaN
+// stored as 0 (concept page, "關鍵機制", INT8 KV-cache quantisation).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -28,7 +30,14 @@ __device__ __forceinline__ int owner_of(const int32_t* cu_new, int batch, int to
   return lo;
 }
 
-template <bool kFp8>
+// Symmetric INT8 code of a quotient: round to nearest even, clamp to +-127.
+__device__ __forceinline__ uint32_t int8_code(float y) {
+  if (y != y) return 0u;
+  const int q = __float2int_rn(fminf(fmaxf(y, -127.f), 127.f));
+  return static_cast<uint32_t>(q) & 0xffu;
+}
+
+template <int kFmt>
 __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
   const int vecs_per_row = p.head_dim / 8;                 // 16-byte vectors per (token, head)
   const int64_t per_token = (int64_t)p.num_kv_heads * vecs_per_row;
@@ -60,7 +69,7 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
     const int64_t dst_elem =
         (((int64_t)page * p.num_kv_heads + g) * p.page_size + slot) * p.head_dim + vec * 8;
     uint8_t* pool = is_v ? p.v_pool : p.k_pool;
-    if constexpr (!kFp8) {
+    if constexpr (!k8(kFmt)) {
       *reinterpret_cast<uint4*>(pool + dst_elem * 2) = src;
     } else {
       const float s = __ldg((is_v ? p.v_scale : p.k_scale) + (int64_t)page * p.num_kv_heads + g);
@@ -74,7 +83,11 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
         float2 f = __bfloat1622float2(x[k]);
         f.x = __fdiv_rn(f.x, s);
         f.y = __fdiv_rn(f.y, s);
-        const uint16_t two = __nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
+        uint16_t two;
+        if constexpr (kFmt == PKV_KV_INT8)
+          two = static_cast<uint16_t>(int8_code(f.x) | (int8_code(f.y) << 8));
+        else
+          two = __nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
         if (k & 1)
           w[k >> 1] |= static_cast<uint32_t>(two) << 16;
         else
@@ -85,17 +98,19 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
   }
 }
 
-cudaError_t launch_append(const AppendParams& p, bool fp8, int num_sms, cudaStream_t stream) {
+cudaError_t launch_append(const AppendParams& p, int fmt, int num_sms, cudaStream_t stream) {
   const int64_t vectors = 2LL * p.total_new * p.num_kv_heads * (p.head_dim / 8);
   if (vectors == 0) return cudaSuccess;
   const int threads = 256;
   int64_t blocks = (vectors + threads - 1) / threads;
   const int64_t cap = (int64_t)num_sms * 8;
   if (blocks > cap) blocks = cap;
-  if (fp8)
-    append_kernel<true><<<(unsigned)blocks, threads, 0, stream>>>(p);
+  if (fmt == PKV_KV_INT8)
+    append_kernel<PKV_KV_INT8><<<(unsigned)blocks, threads, 0, stream>>>(p);
+  else if (fmt == PKV_KV_FP8_E4M3)
+    append_kernel<PKV_KV_FP8_E4M3><<<(unsigned)blocks, threads, 0, stream>>>(p);
   else
-    append_kernel<false><<<(unsigned)blocks, threads, 0, stream>>>(p);
+    append_kernel<PKV_KV_BF16><<<(unsigned)blocks, threads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

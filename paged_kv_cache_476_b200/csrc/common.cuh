@@ -188,6 +188,27 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t codes) {
   return out;
 }
 
+// Two INT8 codes (low byte = element 0) to an f16x2, exactly.  Flipping the
+// sign bit of a two's-complement byte q gives the unsigned byte q + 128; put
+// under the f16 exponent of 1024 (bits 0x64xx) it reads 1024 + q + 128, and
+// subtracting 1152 leaves q (every integer up to 2048 is an f16).
+__device__ __forceinline__ uint32_t s8x2_to_f16x2(uint16_t codes) {
+  const uint32_t u = (uint32_t)codes ^ 0x8080u;
+  uint32_t v = __byte_perm(u, 0x6464u, 0x4140);  // bytes: u0, 0x64, u1, 0x64
+  const uint32_t bias = 0x64806480u;             // f16x2 {1152, 1152}
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(v) : "r"(v), "r"(bias));
+  return v;
+}
+
+// Two 8-bit KV codes of format kFmt to an f16x2 (exact for both formats).
+template <int kFmt>
+__device__ __forceinline__ uint32_t kv8x2_to_f16x2(uint16_t codes) {
+  if constexpr (kFmt == PKV_KV_INT8)
+    return s8x2_to_f16x2(codes);
+  else
+    return e4m3x2_to_f16x2(codes);
+}
+
 // 2^x on the MUFU unit (flush-to-zero for tiny results).
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;

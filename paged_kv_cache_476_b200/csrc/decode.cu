@@ -68,9 +68,9 @@ struct FlushDesc {
   int32_t b, g, slot, seg_base, nseg, whole, final;
 };
 
-template <int D, bool kFp8>
+template <int D, int kFmt>
 struct Layout {
-  static constexpr int kEB = kFp8 ? 1 : 2;
+  static constexpr int kEB = k8(kFmt) ? 1 : 2;
   static constexpr int kRowB = D * kEB;                        // bytes of a token row
   static constexpr int kBoxRowB = kRowB >= 128 ? 128 : kRowB;  // TMA box inner bytes
   static constexpr int kNumBox = kRowB / kBoxRowB;             // boxes per tile row
@@ -88,16 +88,16 @@ struct SmemPlan {
 
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
-template <int D, bool kFp8, int kStages>
+template <int D, int kFmt, int kStages>
 __host__ __device__ inline SmemPlan smem_plan(int G) {
-  using Ly = Layout<D, kFp8>;
+  using Ly = Layout<D, kFmt>;
   SmemPlan s;
   uint32_t o = kStages * Ly::kStageB;
   s.q = o;
   o += kStages * align_up(G * D * 2, 128);
   o = align_up(o, 1024);
   s.conv = o;
-  if (kFp8) o += kConsumerWarps * Ly::kConvB;
+  if (k8(kFmt)) o += kConsumerWarps * Ly::kConvB;
   s.red_o = o;
   o += kConsumerWarps * G * D * 4;
   s.red_m = o;
@@ -144,17 +144,17 @@ __device__ __forceinline__ int32_t clamp_len(const DecodeParams& p, int32_t len,
   return len;
 }
 
-template <int D, bool kFp8, int kStages>
+template <int D, int kFmt, int kStages>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
-  using Ly = Layout<D, kFp8>;
+  using Ly = Layout<D, kFmt>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte align the dynamic window (the swizzle pattern needs it).
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int G = p.group;
-  const SmemPlan sp = smem_plan<D, kFp8, kStages>(G);
+  const SmemPlan sp = smem_plan<D, kFmt, kStages>(G);
   const uint32_t kQStride = align_up(G * D * 2, 128);
   uint8_t* tiles = smem;
   uint8_t* qbuf = smem + sp.q;
@@ -333,13 +333,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int j = t / tiles_per_page;
       const int sub = t - j * tiles_per_page;
       const int pages_b = (len + p.page_size - 1) / p.page_size;
-      const int key = kFp8 ? b * Hkv + g : b;
+      const int key = k8(kFmt) ? b * Hkv + g : b;
       if (cache_key != key || j < cache_j0 || j >= cache_j0 + 32) {
         cache_key = key;
         cache_j0 = j;
         const int jj = j + lane;
         my_pid = jj < pages_b ? __ldg(p.page_table + (int64_t)b * p.max_pages + jj) : 0;
-        if constexpr (kFp8) {
+        if constexpr (k8(kFmt)) {
           if (jj < pages_b && my_pid >= 0 && my_pid < p.num_pages) {
             my_ks = __ldg(p.k_scale + (int64_t)my_pid * Hkv + g);
             my_vs = __ldg(p.v_scale + (int64_t)my_pid * Hkv + g);
@@ -348,12 +348,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       int pid = __shfl_sync(0xffffffffu, my_pid, j - cache_j0);
       float ks = 1.f, vs = 1.f;
-      if constexpr (kFp8) {
+      if constexpr (k8(kFmt)) {
         ks = __shfl_sync(0xffffffffu, my_ks, j - cache_j0);
         vs = __shfl_sync(0xffffffffu, my_vs, j - cache_j0);
       }
       bool bad = pid < 0 || pid >= p.num_pages;
-      if constexpr (kFp8) {
+      if constexpr (k8(kFmt)) {
         if (!bad && !(ks > 0.f && ks <= 32768.f && vs > 0.f && vs <= 32768.f)) {
           bad = true;
           if (lane == 0) flag_error(p.flags, PKV_FLAG_BAD_SCALE);
@@ -463,15 +463,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     // bookkeeping is read from the (still unreleased) stage at hand-off
     const int t_flags = info[stage].flags;
     const int t_valid = info[stage].valid;
-    const float t_ks = kFp8 ? info[stage].ks : 1.f;
-    const float t_vs = kFp8 ? info[stage].vs : 1.f;
+    const float t_ks = k8(kFmt) ? info[stage].ks : 1.f;
+    const float t_vs = k8(kFmt) ? info[stage].vs : 1.f;
     const uint8_t* qs = qbuf + stage * kQStride;
     if (t_flags & kSegFirst) {
       m_run = -INFINITY;
       l_part = 0.f;
 #pragma unroll
       for (int m = 0; m < D / 16; ++m) ot[m][0] = ot[m][1] = ot[m][2] = ot[m][3] = 0.f;
-      if constexpr (!kFp8) {
+      if constexpr (!k8(kFmt)) {
 #pragma unroll
         for (int kk = 0; kk < KS; ++kk) {
           const uint32_t* qrow = reinterpret_cast<const uint32_t*>(qs + gid * D * 2);
@@ -519,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint32_t vbase = kbase + Ly::kTileB;
       // ---- S = Q K^T over my 16 tokens (two n-tiles of 8) ----
       float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      if constexpr (!kFp8) {
+      if constexpr (!k8(kFmt)) {
         // two independent accumulation chains per n-tile (even / odd k-steps)
         float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
@@ -544,18 +544,18 @@ __global__ void __launch_bounds__(kThreads, 2)
           const int chunk = 2 * kp + (mat & 1);
           uint32_t r0, r1, r2, r3;
           ldsm_x4(tile_addr<Ly::kBoxRowB, kTile>(kbase, row, chunk), r0, r1, r2, r3);
-          mma_f16(s[0], qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, e4m3x2_to_f16x2(r0 & 0xffff),
-                  e4m3x2_to_f16x2(r0 >> 16));
+          mma_f16(s[0], qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, kv8x2_to_f16x2<kFmt>(r0 & 0xffff),
+                  kv8x2_to_f16x2<kFmt>(r0 >> 16));
           mma_f16(s[0], qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u,
-                  e4m3x2_to_f16x2(r1 & 0xffff), e4m3x2_to_f16x2(r1 >> 16));
-          mma_f16(s[1], qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, e4m3x2_to_f16x2(r2 & 0xffff),
-                  e4m3x2_to_f16x2(r2 >> 16));
+                  kv8x2_to_f16x2<kFmt>(r1 & 0xffff), kv8x2_to_f16x2<kFmt>(r1 >> 16));
+          mma_f16(s[1], qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, kv8x2_to_f16x2<kFmt>(r2 & 0xffff),
+                  kv8x2_to_f16x2<kFmt>(r2 >> 16));
           mma_f16(s[1], qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u,
-                  e4m3x2_to_f16x2(r3 & 0xffff), e4m3x2_to_f16x2(r3 >> 16));
+                  kv8x2_to_f16x2<kFmt>(r3 & 0xffff), kv8x2_to_f16x2<kFmt>(r3 >> 16));
         }
       }
       // ---- online softmax on row gid (log2 domain) ----
-      const float mul = kFp8 ? qk_mul * t_ks : qk_mul;
+      const float mul = k8(kFmt) ? qk_mul * t_ks : qk_mul;
       float x[4];
 #pragma unroll
       for (int n = 0; n < 2; ++n)
@@ -586,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       // ---- O^T += V^T P^T over my 16 tokens (P^T comes straight from S) ----
       uint32_t pa0, pa2;
-      if constexpr (!kFp8) {
+      if constexpr (!k8(kFmt)) {
         pa0 = pack_bf16(pr[0], pr[1]);
         pa2 = pack_bf16(pr[2], pr[3]);
       } else {
@@ -602,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 2)
               (2 * tid4 + 9 < valid ? 0xffff0000u : 0u);
       }
       uint32_t vsrc;
-      if constexpr (!kFp8) {
+      if constexpr (!k8(kFmt)) {
         vsrc = vbase;
       } else {
         // E4M3 -> f16 copy of my 16 V rows into my conversion tile, laid out
@@ -621,14 +621,14 @@ __global__ void __launch_bounds__(kThreads, 2)
                        : "=r"(raw.x), "=r"(raw.y), "=r"(raw.z), "=r"(raw.w)
                        : "r"(src));
           uint4 h0, h1;
-          h0.x = e4m3x2_to_f16x2(raw.x & 0xffff);
-          h0.y = e4m3x2_to_f16x2(raw.x >> 16);
-          h0.z = e4m3x2_to_f16x2(raw.y & 0xffff);
-          h0.w = e4m3x2_to_f16x2(raw.y >> 16);
-          h1.x = e4m3x2_to_f16x2(raw.z & 0xffff);
-          h1.y = e4m3x2_to_f16x2(raw.z >> 16);
-          h1.z = e4m3x2_to_f16x2(raw.w & 0xffff);
-          h1.w = e4m3x2_to_f16x2(raw.w >> 16);
+          h0.x = kv8x2_to_f16x2<kFmt>(raw.x & 0xffff);
+          h0.y = kv8x2_to_f16x2<kFmt>(raw.x >> 16);
+          h0.z = kv8x2_to_f16x2<kFmt>(raw.y & 0xffff);
+          h0.w = kv8x2_to_f16x2<kFmt>(raw.y >> 16);
+          h1.x = kv8x2_to_f16x2<kFmt>(raw.z & 0xffff);
+          h1.y = kv8x2_to_f16x2<kFmt>(raw.z >> 16);
+          h1.z = kv8x2_to_f16x2<kFmt>(raw.w & 0xffff);
+          h1.w = kv8x2_to_f16x2<kFmt>(raw.w >> 16);
           const uint32_t d0 = tile_addr<128, 16>(cbase, r, 2 * ch);
           const uint32_t d1 = tile_addr<128, 16>(cbase, r, 2 * ch + 1);
           asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(d0), "r"(h0.x),
@@ -647,7 +647,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         // (8-15, 2m), (8-15, 2m+1), transposed on load
         const int chunk = 2 * m + (mat & 1);
         uint32_t a0, a1, a2, a3;
-        if constexpr (!kFp8) {
+        if constexpr (!k8(kFmt)) {
           const int row = 16 * warp + mrow + (mat >> 1) * 8;
           ldsm_x4_t(tile_addr<Ly::kBoxRowB, kTile>(vsrc, row, chunk), a0, a1, a2, a3);
         } else {
@@ -658,7 +658,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         a1 &= vm0;
         a2 &= vm1;
         a3 &= vm1;
-        if constexpr (!kFp8)
+        if constexpr (!k8(kFmt))
           mma_bf16(ot[m], a0, a1, a2, a3, pa0, pa2);
         else
           mma_f16(ot[m], a0, a1, a2, a3, pa0, pa2);
@@ -809,28 +809,28 @@ cudaError_t merge_launch(const DecodeParams& p, cudaStream_t stream) {
 }
 
 // ------------------------------------------------------------- host side
-template <int D, bool kFp8, int kStages>
+template <int D, int kFmt, int kStages>
 size_t decode_smem_bytes(int G) {
-  return 1024 + smem_plan<D, kFp8, kStages>(G).total;  // + alignment slack
+  return 1024 + smem_plan<D, kFmt, kStages>(G).total;  // + alignment slack
 }
 
-template <int D, bool kFp8, int kStages>
+template <int D, int kFmt, int kStages>
 cudaError_t decode_prepare(int G, int* ctas_per_sm) {
-  auto k = decode_kernel<D, kFp8, kStages>;
-  const size_t smem = decode_smem_bytes<D, kFp8, kStages>(G);
+  auto k = decode_kernel<D, kFmt, kStages>;
+  const size_t smem = decode_smem_bytes<D, kFmt, kStages>(G);
   // The attribute belongs to the instantiation, which serves every group
   // size: allow the largest footprint once, not the one of this call.
-  const size_t most = decode_smem_bytes<D, kFp8, kStages>(kMaxGroup);
+  const size_t most = decode_smem_bytes<D, kFmt, kStages>(kMaxGroup);
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most);
   if (e != cudaSuccess) return e;
   return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, k, kThreads, smem);
 }
 
-template <int D, bool kFp8, int kStages>
+template <int D, int kFmt, int kStages>
 cudaError_t decode_launch(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                           int num_ctas, cudaStream_t stream) {
-  const size_t smem = decode_smem_bytes<D, kFp8, kStages>(p.group);
-  decode_kernel<D, kFp8, kStages><<<num_ctas, kThreads, smem, stream>>>(tk, tv, p);
+  const size_t smem = decode_smem_bytes<D, kFmt, kStages>(p.group);
+  decode_kernel<D, kFmt, kStages><<<num_ctas, kThreads, smem, stream>>>(tk, tv, p);
   return cudaGetLastError();
 }
 
@@ -838,48 +838,66 @@ cudaError_t decode_launch(const CUtensorMap& tk, const CUtensorMap& tv, const De
 // memory per SM, 1 KB of it reserved per CTA).
 constexpr size_t kSmemPerCtaFor2 = 113 * 1024;
 
-template <int D, bool kFp8>
+template <int D, int kFmt>
 int pick_stages(int G) {
-  if (decode_smem_bytes<D, kFp8, 4>(G) <= kSmemPerCtaFor2) return 4;
-  if (decode_smem_bytes<D, kFp8, 3>(G) <= kSmemPerCtaFor2) return 3;
+  if (decode_smem_bytes<D, kFmt, 4>(G) <= kSmemPerCtaFor2) return 4;
+  if (decode_smem_bytes<D, kFmt, 3>(G) <= kSmemPerCtaFor2) return 3;
   return 2;
 }
 
-template <int D, bool kFp8>
+template <int D, int kFmt>
 cudaError_t occupancy_for(int G, int* n) {
-  switch (pick_stages<D, kFp8>(G)) {
-    case 4: return decode_prepare<D, kFp8, 4>(G, n);
-    case 3: return decode_prepare<D, kFp8, 3>(G, n);
-    default: return decode_prepare<D, kFp8, 2>(G, n);
+  switch (pick_stages<D, kFmt>(G)) {
+    case 4: return decode_prepare<D, kFmt, 4>(G, n);
+    case 3: return decode_prepare<D, kFmt, 3>(G, n);
+    default: return decode_prepare<D, kFmt, 2>(G, n);
   }
 }
 
-template <int D, bool kFp8>
+template <int D, int kFmt>
 cudaError_t run_for(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                     int num_ctas, cudaStream_t stream) {
   cudaError_t e;
-  switch (pick_stages<D, kFp8>(p.group)) {
-    case 4: e = decode_launch<D, kFp8, 4>(tk, tv, p, num_ctas, stream); break;
-    case 3: e = decode_launch<D, kFp8, 3>(tk, tv, p, num_ctas, stream); break;
-    default: e = decode_launch<D, kFp8, 2>(tk, tv, p, num_ctas, stream); break;
+  switch (pick_stages<D, kFmt>(p.group)) {
+    case 4: e = decode_launch<D, kFmt, 4>(tk, tv, p, num_ctas, stream); break;
+    case 3: e = decode_launch<D, kFmt, 3>(tk, tv, p, num_ctas, stream); break;
+    default: e = decode_launch<D, kFmt, 2>(tk, tv, p, num_ctas, stream); break;
   }
   if (e != cudaSuccess) return e;
   return merge_launch<D>(p, stream);
 }
 
-cudaError_t decode_occupancy(int head_dim, bool fp8, int group, int* ctas_per_sm) {
-  if (!fp8 && head_dim == 128) return occupancy_for<128, false>(group, ctas_per_sm);
-  if (!fp8 && head_dim == 64) return occupancy_for<64, false>(group, ctas_per_sm);
-  if (fp8 && head_dim == 128) return occupancy_for<128, true>(group, ctas_per_sm);
-  return occupancy_for<64, true>(group, ctas_per_sm);
+// Each (head_dim, format) pair is its own instantiation (and its own
+// shared-memory attribute); E4M3 and INT8 share a layout, not a kernel.
+cudaError_t decode_occupancy(int head_dim, int fmt, int group, int* ctas_per_sm) {
+  const bool d128 = head_dim == 128;
+  switch (fmt) {
+    case PKV_KV_INT8:
+      return d128 ? occupancy_for<128, PKV_KV_INT8>(group, ctas_per_sm)
+                  : occupancy_for<64, PKV_KV_INT8>(group, ctas_per_sm);
+    case PKV_KV_FP8_E4M3:
+      return d128 ? occupancy_for<128, PKV_KV_FP8_E4M3>(group, ctas_per_sm)
+                  : occupancy_for<64, PKV_KV_FP8_E4M3>(group, ctas_per_sm);
+    default:
+      return d128 ? occupancy_for<128, PKV_KV_BF16>(group, ctas_per_sm)
+                  : occupancy_for<64, PKV_KV_BF16>(group, ctas_per_sm);
+  }
 }
 
-cudaError_t decode_run(int head_dim, bool fp8, const CUtensorMap& tk, const CUtensorMap& tv,
+cudaError_t decode_run(int head_dim, int fmt, const CUtensorMap& tk, const CUtensorMap& tv,
                        const DecodeParams& p, int num_ctas, cudaStream_t stream) {
-  if (!fp8 && head_dim == 128) return run_for<128, false>(tk, tv, p, num_ctas, stream);
-  if (!fp8 && head_dim == 64) return run_for<64, false>(tk, tv, p, num_ctas, stream);
-  if (fp8 && head_dim == 128) return run_for<128, true>(tk, tv, p, num_ctas, stream);
-  return run_for<64, true>(tk, tv, p, num_ctas, stream);
+  const bool d128 = head_dim == 128;
+  switch (fmt) {
+    case PKV_KV_INT8:
+      return d128 ? run_for<128, PKV_KV_INT8>(tk, tv, p, num_ctas, stream)
+                  : run_for<64, PKV_KV_INT8>(tk, tv, p, num_ctas, stream);
+    case PKV_KV_FP8_E4M3:
+      return d128 ? run_for<128, PKV_KV_FP8_E4M3>(tk, tv, p, num_ctas, stream)
+                  : run_for<64, PKV_KV_FP8_E4M3>(tk, tv, p, num_ctas, stream);
+    default:
+      return d128 ? run_for<128, PKV_KV_BF16>(tk, tv, p, num_ctas, stream)
+                  : run_for<64, PKV_KV_BF16>(tk, tv, p, num_ctas, stream);
+  }
 }
 
 }  // namespace pkv

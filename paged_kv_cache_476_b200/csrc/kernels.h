@@ -10,6 +10,9 @@
 
 namespace pkv {
 
+// KV formats of the pools (pkv_kv_dtype): is the stored code one byte?
+__host__ __device__ constexpr bool k8(int fmt) { return fmt != PKV_KV_BF16; }
+
 struct AppendParams {
   uint8_t* k_pool;
   uint8_t* v_pool;
@@ -52,9 +55,10 @@ struct DecodeParams {
   float scale_log2;  // softmax_scale * log2(e)
 };
 
-cudaError_t launch_append(const AppendParams& p, bool fp8, int num_sms, cudaStream_t stream);
-cudaError_t decode_occupancy(int head_dim, bool fp8, int group, int* ctas_per_sm);
-cudaError_t decode_run(int head_dim, bool fp8, const CUtensorMap& tk, const CUtensorMap& tv,
+// fmt: the pool's pkv_kv_dtype
+cudaError_t launch_append(const AppendParams& p, int fmt, int num_sms, cudaStream_t stream);
+cudaError_t decode_occupancy(int head_dim, int fmt, int group, int* ctas_per_sm);
+cudaError_t decode_run(int head_dim, int fmt, const CUtensorMap& tk, const CUtensorMap& tv,
                        const DecodeParams& p, int num_ctas, cudaStream_t stream);
 
 int check_cache(const pkv_cache* c);

@@ -32,9 +32,9 @@
 //    and finally normalise O.
 //  * V rows past the sequence end (or of a rejected page) are zeroed in
 //    shared memory before their PV product: 0 * NaN would poison O.
-//  * E4M3 pools: two converter warps turn each landed E4M3 tile into a 16-bit
-//    tile (exact) laid out as TMA lays out bf16 tiles: K as bf16 (Q's type),
-//    V as f16.  The per-(page, head) K scales multiply the scores of their
+//  * E4M3 and INT8 pools: two converter warps turn each landed tile of
+//    one-byte codes into a 16-bit tile (exact) laid out as TMA lays out bf16
+//    tiles: K as bf16 (Q's type), V as f16.  The per-(page, head) K scales multiply the scores of their
 //    64-key block; the V scales ride on P, kept in f16 (11-bit mantissa) so
 //    that PV is an f16 x f16 product.
 //  * Every wait is bounded; TMEM is freed on every exit path.
@@ -154,15 +154,6 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// Store 8 consecutive 32-bit columns of this warp's 32 TMEM lanes.
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
-          taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-      : "memory");
-}
-
 // Store 16 consecutive 32-bit columns of this warp's 32 TMEM lanes.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
   asm volatile(
@@ -224,17 +215,17 @@ __host__ __device__ constexpr uint32_t idesc_f16kind(int M, int N, int b_mn_majo
          | ((uint32_t)(M >> 4) << 24);       // M / 16
 }
 
-template <int D, bool kFp8>
+template <int D, int kFmt>
 struct Smem {
   static constexpr int kHalves = D / 64;            // 128-byte column boxes per bf16 row
   static constexpr int kQB = kRows * D * 2;         // one Q tile
   static constexpr int kTileB = kKeys * D * 2;      // bf16 K (or V) tile
   static constexpr int kHalfB = kKeys * 128;        // one 64-column half of a bf16 tile
   static constexpr int kTile8B = kKeys * D;         // E4M3 K (or V) tile as it lands
-  static constexpr int kStageB = kFp8 ? 2 * kTile8B : 2 * kTileB;
-  static constexpr int kConvB = kFp8 ? 2 * kTileB : 0;  // converted K, then V
+  static constexpr int kStageB = k8(kFmt) ? 2 * kTile8B : 2 * kTileB;
+  static constexpr int kConvB = k8(kFmt) ? 2 * kTileB : 0;  // converted K, then V
   static constexpr int kBytes = 2 * kQB + kStages * kStageB + kConvB;
-  static constexpr int kThreads = kFp8 ? 384 : 320;  // + two converter warps
+  static constexpr int kThreads = k8(kFmt) ? 384 : 320;  // + two converter warps
 };
 
 // Per-KV-tile facts the producer passes on: rejected 64-key blocks and the
@@ -266,7 +257,7 @@ __device__ __forceinline__ uint32_t e4m3_chunk(uint32_t base, int r, int c) {
 // E4M3 tile -> bf16 or f16 tile (both exact: every E4M3 value is an f16 and a
 // bf16), rows in `zero_mask` (bit per 64-row block) or at/after `zero_from`
 // written as zeros.  64 threads share the work.
-template <int D, bool kToF16>
+template <int D, int kFmt, bool kToF16>
 __device__ __forceinline__ void convert_tile(uint32_t src, uint32_t dst, int t, int zero_from,
                                              int zero_mask) {
   constexpr int kChunks = kKeys * D / 16;  // 16-byte E4M3 chunks
@@ -285,8 +276,8 @@ __device__ __forceinline__ void convert_tile(uint32_t src, uint32_t dst, int t, 
                    : "r"(e4m3_chunk<D>(src, r, c)));
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const uint32_t h01 = e4m3x2_to_f16x2(w[k] & 0xffff);
-        const uint32_t h23 = e4m3x2_to_f16x2(w[k] >> 16);
+        const uint32_t h01 = kv8x2_to_f16x2<kFmt>(w[k] & 0xffff);
+        const uint32_t h23 = kv8x2_to_f16x2<kFmt>(w[k] >> 16);
         if constexpr (kToF16) {
           o[2 * k] = h01;
           o[2 * k + 1] = h23;
@@ -408,12 +399,12 @@ __device__ bool lpt_item(const Params& p, uint32_t rank, int32_t pair_tokens, in
   return true;
 }
 
-template <int D, bool kFp8>
-__global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
+template <int D, int kFmt>
+__global__ void __launch_bounds__(Smem<D, kFmt>::kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,
                    const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v, const Params p) {
-  using Sm = Smem<D, kFp8>;
+  using Sm = Smem<D, kFmt>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -470,8 +461,8 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
-      mbar_init(&k_empty[s], kFp8 ? 2 : 1);  // E4M3: released by the two converter warps
-      mbar_init(&v_empty[s], kFp8 ? 2 : 1);
+      mbar_init(&k_empty[s], k8(kFmt) ? 2 : 1);  // E4M3: released by the two converter warps
+      mbar_init(&v_empty[s], k8(kFmt) ? 2 : 1);
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&s_full[x], 1);
@@ -564,7 +555,7 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
             lk.tf.bad |= 1 << sb;
             continue;
           }
-          if constexpr (kFp8) {
+          if constexpr (k8(kFmt)) {
             const float ks = __ldg(p.k_scale + (int64_t)pid * p.num_kv_heads + g);
             const float vs = __ldg(p.v_scale + (int64_t)pid * p.num_kv_heads + g);
             if (!(ks > 0.f && ks <= 32768.f && vs > 0.f && vs <= 32768.f)) {
@@ -582,13 +573,13 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
         return lk;
       };
       // bytes of one operand (K or V) per live 64-key block
-      constexpr uint32_t kBlockBytes = kFp8 ? 64u * D : Sm::kHalves * 64u * 128u;
+      constexpr uint32_t kBlockBytes = k8(kFmt) ? 64u * D : Sm::kHalves * 64u * 128u;
       // load one operand of a tile into its slot
       auto load = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, const Lookup& lk) {
         mbar_arrive_expect_tx(bar, (uint32_t)__popc(lk.live) * kBlockBytes);
         for (int sb = 0; sb < 2; ++sb) {
           if (!((lk.live >> sb) & 1)) continue;
-          if constexpr (kFp8) {
+          if constexpr (k8(kFmt)) {
             tma_load_2d(dst + sb * 64 * D, map, 0, lk.ys[sb], bar, pol);
           } else {
 #pragma unroll
@@ -615,7 +606,7 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
         if (j + 1 < n_kv) cur = lookup(j + 1);  // ahead of the next slot wait
       }
     }
-  } else if (kFp8 && warp >= kConvWarp0) {
+  } else if (k8(kFmt) && warp >= kConvWarp0) {
     // ------------------------------------------------- E4M3 -> 16-bit converters
     const int t = threadIdx.x - kConvWarp0 * 32;  // 0..63
     const uint32_t kc = smem_u32(sconv), vc = kc + Sm::kTileB;
@@ -623,13 +614,14 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
       const int st = j % kStages;
       const uint32_t par = (uint32_t)((j / kStages) & 1);
       if (!mbar_wait(&k_full[st], par, p.flags)) break;
-      const uint32_t k8 = smem_u32(skv + st * Sm::kStageB), v8 = k8 + Sm::kStageB / 2;
+      const uint32_t k_codes = smem_u32(skv + st * Sm::kStageB);
+      const uint32_t v_codes = k_codes + Sm::kStageB / 2;
       const int bad = facts[j % kFactsRing].bad;
       const int32_t key0 = j * kKeys;
       const int zero_from = key0 + kKeys > L ? max(0, L - key0) : kKeys;
       // K (rows that must not count are masked in the scores; keep them finite)
       if (j >= 1 && !mbar_wait(kc_free, (uint32_t)((j - 1) & 1), p.flags)) break;
-      convert_tile<D, false>(k8, kc, t, zero_from, bad);  // bf16, like Q
+      convert_tile<D, kFmt, false>(k_codes, kc, t, zero_from, bad);  // bf16, like Q
       fence_async_smem();
       __syncwarp();
       if (lane == 0) {
@@ -639,7 +631,7 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
       if (!mbar_wait(&v_full[st], par, p.flags)) break;
       // V (rows that must not count are zeros: 0 * NaN would poison O)
       if (j >= 1 && !mbar_wait(vc_free, (uint32_t)((j - 1) & 1), p.flags)) break;
-      convert_tile<D, true>(v8, vc, t, zero_from, bad);  // f16, like P
+      convert_tile<D, kFmt, true>(v_codes, vc, t, zero_from, bad);  // f16, like P
       fence_async_smem();
       __syncwarp();
       if (lane == 0) {
@@ -653,11 +645,11 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
     // tensor core always has the other tile's work while a softmax runs.
     const uint32_t id_s = idesc_f16kind(kRows, kKeys, 0, true);
     // E4M3: P (scaled by the V scales) and V are f16 for the PV product
-    const uint32_t id_o = idesc_f16kind(kRows, D, 1, !kFp8);
+    const uint32_t id_o = idesc_f16kind(kRows, D, 1, !k8(kFmt));
     const uint32_t q_addr = smem_u32(sq);
     bool ok = mbar_wait(q_full, 0, p.flags);
     auto k_ready = [&](int j, uint32_t* addr) -> bool {
-      if constexpr (kFp8) {
+      if constexpr (k8(kFmt)) {
         *addr = smem_u32(sconv);
         return mbar_wait(kc_full, (uint32_t)(j & 1), p.flags);
       } else {
@@ -684,7 +676,7 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
     // V of tile j, made safe for the PV product (rows past the end or of a
     // rejected page zeroed); returns false on a timeout
     auto v_ready = [&](int j, uint32_t* addr) -> bool {
-      if constexpr (kFp8) {
+      if constexpr (k8(kFmt)) {
         *addr = smem_u32(sconv) + Sm::kTileB;
         return mbar_wait(vc_full, (uint32_t)(j & 1), p.flags);
       } else {
@@ -734,7 +726,7 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
     if (ok) {
       issue_s(0, k_addr);
       if (hasB) issue_s(1, k_addr);
-      if (lane == 0) tc_commit(kFp8 ? kc_free : &k_empty[0]);  // K_0 is read by both S products
+      if (lane == 0) tc_commit(k8(kFmt) ? kc_free : &k_empty[0]);  // K_0 is read by both S products
       __syncwarp();
     }
     for (int j = 0; j < n_kv && ok; ++j) {
@@ -747,10 +739,10 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
       if (j < nkv[1] && !(ok = issue_pv(1, j, v_addr))) break;
       // V_j is consumed once both PV products have run, K_{j+1} once both
       // S products have
-      if (lane == 0) tc_commit(kFp8 ? vc_free : &v_empty[j % kStages]);
+      if (lane == 0) tc_commit(k8(kFmt) ? vc_free : &v_empty[j % kStages]);
       __syncwarp();
       if (j + 1 < nkv[1]) issue_s(1, k_addr);
-      if (next && lane == 0) tc_commit(kFp8 ? kc_free : &k_empty[(j + 1) % kStages]);
+      if (next && lane == 0) tc_commit(k8(kFmt) ? kc_free : &k_empty[(j + 1) % kStages]);
       __syncwarp();
     }
     // every MMA this thread issued must finish before TMEM is released
@@ -782,8 +774,8 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
         // blocks of a rejected page; E4M3 K scales per 64-key block
         const int32_t key0 = j * kKeys;
         const bool diag = key0 + kKeys - 1 > p_min;
-        const float mul0 = kFp8 ? p.scale_log2 * tf.ks[0] : p.scale_log2;
-        const float mul1 = kFp8 ? p.scale_log2 * tf.ks[1] : p.scale_log2;
+        const float mul0 = k8(kFmt) ? p.scale_log2 * tf.ks[0] : p.scale_log2;
+        const float mul1 = k8(kFmt) ? p.scale_log2 * tf.ks[1] : p.scale_log2;
         auto scaled = [&](float v, int c) -> float {
           const bool keep = (!diag || key0 + c <= pos) && !((tf.bad >> (c >> 6)) & 1);
           return keep ? v * (c < 64 ? mul0 : mul1) : -INFINITY;
@@ -802,7 +794,7 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
         // waits for this tile's P.
         float alpha = 1.f;
         auto set_max = [&](float mt) -> float {
-          const bool need = mt > m_ref + (kFp8 ? 0.f : 8.f);  // true on the first visible tile
+          const bool need = mt > m_ref + (k8(kFmt) ? 0.f : 8.f);  // true on the first visible tile
           const float m_new = need ? mt : m_ref;
           if (j >= 1 && need) alpha = fast_exp2(m_ref - m_new);
           m_ref = m_new;
@@ -839,7 +831,7 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
             tmem_ld32(tmem + lane_base + colS + cb + 32, sv + 32);
             tmem_wait_ld();
             const float mul = cb < 64 ? mul0 : mul1;
-            const float vsc = kFp8 ? (cb < 64 ? tf.vs[0] : tf.vs[1]) : 1.f;  // E4M3 V scales ride on P
+            const float vsc = k8(kFmt) ? (cb < 64 ? tf.vs[0] : tf.vs[1]) : 1.f;  // E4M3 V scales ride on P
             uint32_t pk[32];
             // (two loops rather than a branch per element, which the compiler
             // would turn into both paths under predicates)
@@ -851,7 +843,7 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
                 const float p1 = fast_exp2(fmaf(sv[i + 1], mul, -m_use));
                 r0 += p0;
                 r1 += p1;
-                pk[i / 2] = kFp8 ? pack_f16(p0 * vsc, p1 * vsc) : pack_bf16(p0, p1);
+                pk[i / 2] = k8(kFmt) ? pack_f16(p0 * vsc, p1 * vsc) : pack_bf16(p0, p1);
               }
               rs += r0 + r1;
             } else {
@@ -860,7 +852,7 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
                 const float p0 = fast_exp2(scaled(sv[i], cb + i) - m_use);
                 const float p1 = fast_exp2(scaled(sv[i + 1], cb + i + 1) - m_use);
                 rs += p0 + p1;
-                pk[i / 2] = kFp8 ? pack_f16(p0 * vsc, p1 * vsc) : pack_bf16(p0, p1);
+                pk[i / 2] = k8(kFmt) ? pack_f16(p0 * vsc, p1 * vsc) : pack_bf16(p0, p1);
               }
             }
             // P column c/2 lies in an S column already read
@@ -924,25 +916,25 @@ __global__ void __launch_bounds__(Smem<D, kFp8>::kThreads, 1)
   }
 }
 
-template <int D, bool kFp8>
+template <int D, int kFmt>
 size_t smem_bytes() {
-  return 1024 + Smem<D, kFp8>::kBytes + (20 + kFactsRing) * sizeof(uint64_t) +
+  return 1024 + Smem<D, kFmt>::kBytes + (20 + kFactsRing) * sizeof(uint64_t) +
          kFactsRing * sizeof(TileFacts) + 32;  // + TMEM base and the item
 }
 
-template <int D, bool kFp8>
+template <int D, int kFmt>
 cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const Params& p, cudaStream_t stream) {
-  const size_t smem = smem_bytes<D, kFp8>();
+  const size_t smem = smem_bytes<D, kFmt>();
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, kFp8>,
+    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, kFmt>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
   const unsigned blocks = (unsigned)p.pair_slots * (unsigned)p.num_kv_heads * (unsigned)p.num_chunks;
-  prefill_kernel<D, kFp8><<<blocks, Smem<D, kFp8>::kThreads, smem, stream>>>(tq, tk, tv, p);
+  prefill_kernel<D, kFmt><<<blocks, Smem<D, kFmt>::kThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
@@ -967,7 +959,8 @@ int prefill_entry(const pkv_cache* cache, const void* q, int32_t num_q_heads, in
   if (!q || !cu_q_lens || !page_table || !seq_lens || !out) return PKV_ERR_NULL;
   if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(out) & 15))
     return PKV_ERR_ALIGN;
-  const bool fp8 = cache->kv_dtype == PKV_KV_FP8_E4M3;
+  const int fmt = cache->kv_dtype;
+  const bool fp8 = k8(fmt);  // one-byte codes
   const int D = cache->head_dim;
   CUtensorMap tq, tk, tv;
   if ((st = encode_q_map(&tq, q, total_q, num_q_heads, D, gqa_group))) return st;
@@ -999,11 +992,13 @@ int prefill_entry(const pkv_cache* cache, const void* q, int32_t num_q_heads, in
   if ((int64_t)p.pair_slots * p.num_kv_heads * num_chunks > INT32_MAX) return PKV_ERR_SHAPE;
   cudaError_t e;
   if (D == 128)
-    e = fp8 ? pf::launch<128, true>(tq, tk, tv, p, stream)
-            : pf::launch<128, false>(tq, tk, tv, p, stream);
+    e = fmt == PKV_KV_INT8       ? pf::launch<128, PKV_KV_INT8>(tq, tk, tv, p, stream)
+        : fmt == PKV_KV_FP8_E4M3 ? pf::launch<128, PKV_KV_FP8_E4M3>(tq, tk, tv, p, stream)
+                                 : pf::launch<128, PKV_KV_BF16>(tq, tk, tv, p, stream);
   else
-    e = fp8 ? pf::launch<64, true>(tq, tk, tv, p, stream)
-            : pf::launch<64, false>(tq, tk, tv, p, stream);
+    e = fmt == PKV_KV_INT8       ? pf::launch<64, PKV_KV_INT8>(tq, tk, tv, p, stream)
+        : fmt == PKV_KV_FP8_E4M3 ? pf::launch<64, PKV_KV_FP8_E4M3>(tq, tk, tv, p, stream)
+                                 : pf::launch<64, PKV_KV_BF16>(tq, tk, tv, p, stream);
   return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 

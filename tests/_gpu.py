@@ -10,8 +10,9 @@ import workloads
 
 def sentinel_pool(w, device):
     shape = w.pool_shape()
-    if w.kv_dtype == "e4m3":
-        return torch.full(shape, workloads.E4M3_NAN_CODE, dtype=torch.uint8, device=device)
+    if w.kv_dtype != "bf16":
+        return torch.full(shape, workloads.sentinel_byte(w.kv_dtype), dtype=torch.uint8,
+                          device=device)
     return torch.full(shape, workloads.BF16_NAN_BITS, dtype=torch.int16,
                       device=device).view(torch.bfloat16)
 
@@ -29,7 +30,7 @@ class GpuState:
         self.v_pool = sentinel_pool(w, device)
         self.flags = torch.zeros(1, dtype=torch.int32, device=device)
         self.k_scale = self.v_scale = None
-        if w.kv_dtype == "e4m3":
+        if w.kv_dtype != "bf16":
             self.k_scale = torch.ones((w.num_pages, w.num_kv_heads), dtype=torch.float32,
                                       device=device)
             self.v_scale = torch.ones_like(self.k_scale)
@@ -55,7 +56,7 @@ class GpuState:
         for b in rows:
             k, v = w.kv_seq(b)
             c = int(w.ctx_lens[b])
-            if w.kv_dtype == "e4m3":
+            if w.kv_dtype != "bf16":
                 pages, k_s, v_s = w.kv_scales_for(b, k, v)
                 idx = torch.from_numpy(pages.astype(np.int64)).to(self.device)
                 self.k_scale[idx] = torch.from_numpy(k_s).to(self.device)

@@ -1,7 +1,7 @@
 """Parity of the CUDA append and decode kernels with the oracle (needs a GPU).
 
 Append: the device pool must equal the oracle's own pool byte for byte (bf16
-bits, E4M3 codes, and every untouched sentinel byte).  Decode: bf16 output
+bits, E4M3 or INT8 codes, and every untouched sentinel byte).  Decode: bf16 output
 within max-abs 1e-2 and mean-abs 1e-3 of the fp64 oracle; lse within 2e-3.
 Inputs are the seeded synthetic workloads (shapes of the five benchmark
 configurations plus ragged edge cases).
@@ -33,7 +33,7 @@ def _check_pool(st, w):
 
 
 # ------------------------------------------------------------------ append
-@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3", "int8"])
 @pytest.mark.parametrize("P,D", [(64, 64), (64, 128), (128, 128), (128, 64)])
 def test_append_is_bit_exact(dtype, P, D):
     w = workloads.build("append", 7, [0, 1, 63, 64, 127, 200, 5], [1, 1, 1, 65, 2, 129, 300],
@@ -71,6 +71,27 @@ def test_append_e4m3_saturates_like_the_oracle():
     k, v = st.pool_bytes()
     assert np.array_equal(k, c.k_pool) and np.array_equal(v, c.v_pool)
     assert (k == 0x7E).any() and (k == 0xFE).any()
+
+
+def test_append_int8_clamps_like_the_oracle():
+    # scales far below absmax/127: most codes clamp to +-127 (never -128)
+    w = workloads.build("sat8", 8, [10, 70], [3, 1], page_size=64, num_q_heads=2,
+                        num_kv_heads=1, head_dim=128, kv_dtype="int8", pool_slack=0.5)
+    st = GpuState(w)
+    st.k_scale.fill_(2.0**-9)
+    st.v_scale.fill_(0.013)
+    st.append_step()
+    torch.cuda.synchronize()
+    c = oracle.cache_for(w, include_new=False)
+    c.k_scale[:] = 2.0**-9
+    c.v_scale[:] = 0.013
+    k_new, v_new = w.new_kv()
+    c.append(w.page_table, w.ctx_lens, w.cu_new(), oracle.bf16_bits(k_new),
+             oracle.bf16_bits(v_new))
+    k, v = st.pool_bytes()
+    assert np.array_equal(k, c.k_pool) and np.array_equal(v, c.v_pool)
+    new_k = k.view(np.int8)
+    assert (new_k == 127).any() and (new_k == -127).any()
 
 
 def test_append_bad_page_is_skipped_and_flagged():
@@ -112,6 +133,9 @@ CASES = [
     ("e4m3", 64, 128, 8, 8, [0, 1, 63, 64, 300, 1500, 4095]),
     ("e4m3", 128, 128, 2, 4, [0, 129, 1000, 2047]),
     ("e4m3", 64, 64, 2, 2, [3, 64, 65, 400]),
+    ("int8", 64, 128, 8, 8, [0, 1, 63, 64, 300, 1500, 4095]),
+    ("int8", 128, 128, 2, 4, [0, 129, 1000, 2047]),
+    ("int8", 64, 64, 2, 1, [3, 64, 65, 400]),
 ]
 
 
@@ -201,6 +225,19 @@ def test_config_long_context_decode_sampled():
 
 def test_config_70b_fp8_decode_full():
     w = workloads.llama70b_fp8_decode()
+    st = GpuState(w)
+    st.append_step()
+    torch.cuda.synchronize()
+    _check_pool(st, w)
+    out, lse = st.decode()
+    torch.cuda.synchronize()
+    ref, ref_lse = _oracle_decode(w)
+    compare(out, lse, ref, ref_lse)
+    assert int(st.flags.item()) == 0
+
+
+def test_config_70b_int8_decode_full():
+    w = workloads.llama70b_int8_decode()
     st = GpuState(w)
     st.append_step()
     torch.cuda.synchronize()

@@ -2,8 +2,8 @@
 
 Causal chunk attention (query i of a chunk with n queries over L tokens sees
 keys 0..L-n+i): bf16 output within max-abs 1e-2 and mean-abs 1e-3 of the
-fp64 oracle, lse within 2e-3.  Cases cover bf16 and E4M3 pools (the oracle
-attends over its own bit-identical E4M3 pool), GQA groups 1..8, head_dim
+fp64 oracle, lse within 2e-3.  Cases cover bf16, E4M3 and INT8 pools (the
+oracle attends over its own bit-identical pool of codes), GQA groups 1..8, head_dim
 64/128, page sizes 64/128, chunks without context, chunks shorter than a Q
 tile, ragged tails and the in-flight mixed-batch configuration.
 """
@@ -37,6 +37,9 @@ CASES = [
     ("e4m3", 128, 128, 1, 8, [5, 0, 300], [17, 1, 129]),
     ("e4m3", 64, 64, 2, 2, [63, 64, 0], [65, 1, 300]),
     ("e4m3", 128, 64, 2, 1, [1000], [200]),
+    ("int8", 64, 128, 2, 4, [0, 100, 700], [512, 33, 130]),
+    ("int8", 128, 128, 1, 8, [5, 0, 300], [17, 1, 129]),
+    ("int8", 64, 64, 2, 2, [63, 64, 0], [65, 1, 300]),
 ]
 
 
@@ -72,7 +75,7 @@ def test_prefill_many_chunks(num_chunks):
     assert int(st.flags.item()) == 0
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3", "int8"])
 def test_prefill_negative_scale(dtype):
     # the row max of s * scale is not scale * max(s) when scale < 0
     w = workloads.build("pfneg", 27, [300, 0], [200, 130], page_size=64, num_q_heads=8,

@@ -323,6 +323,15 @@ def llama70b_fp8_decode(seed: int = 3) -> Workload:
                  kv_dtype="e4m3", rng=rng)
 
 
+def llama70b_int8_decode(seed: int = 3) -> Workload:
+    """The 70B-shaped decode batch of ``llama70b_fp8_decode`` with INT8 K/V pools."""
+    rng = np.random.default_rng(seed)
+    ctx = np.clip(np.rint(np.exp(rng.normal(math.log(1024.0), 0.8, size=256))), 1, 8191)
+    return build("llama3_70b_int8_decode_b256_p64_gqa8_d128", seed, ctx.astype(np.int64),
+                 [1] * 256, page_size=64, num_q_heads=64, num_kv_heads=8, head_dim=128,
+                 kv_dtype="int8", rng=rng)
+
+
 def mixed_inflight(seed: int = 4) -> Workload:
     """32 decode seqs U[256,4096] + 4 prefill chunks of 512 over context U[0,2048]."""
     rng = np.random.default_rng(seed)
@@ -341,6 +350,7 @@ CONFIGS = {
     3: long_context_decode,
     4: llama70b_fp8_decode,
     5: mixed_inflight,
+    6: llama70b_int8_decode,
 }
 
 
