@@ -226,6 +226,26 @@ int paged_decode_attention_noalloc(const pkv_cache* cache, const void* q, int32_
                                    int32_t batch, int32_t max_seq_len, float softmax_scale,
                                    void* out, float* lse, int32_t num_ctas, void* stream);
 
+/*
+ * Combine attention results over disjoint key ranges (sequence parallelism).
+ * Part r attended over its own keys of each row -- e.g. one GPU's pages of a
+ * long sequence, via paged_decode_attention with that GPU's slice of the page
+ * table -- and gave the normalised output out_r and its lse_r.  The result
+ * over all keys is
+ *   lse = log sum_r exp(lse_r),   out = sum_r exp(lse_r - lse) out_r,
+ * the split-KV reduction (concept page, "執行時執行模型": attention over the
+ * sequence's pages; splitting them across devices is this library's reading).
+ * A part with lse_r = -inf (no key) has weight 0; a row whose parts are all
+ * empty becomes 0 with lse -inf.
+ *   parts      bf16 [num_parts][rows][head_dim], 16-byte aligned
+ *   lse_parts  fp32 [num_parts][rows]
+ *   out        bf16 [rows][head_dim], 16-byte aligned; lse fp32 [rows] or NULL
+ * rows = batch * num_q_heads.  head_dim in {64, 128}; num_parts >= 1.
+ */
+int paged_attention_combine(const void* parts, const float* lse_parts, int32_t num_parts,
+                            int32_t rows, int32_t head_dim, void* out, float* lse,
+                            void* stream);
+
 /* Human-readable name of a pkv_status value (static storage). */
 const char* pkv_status_string(int status);
 

@@ -46,6 +46,7 @@ EXPORTED = (
     "pkv_status_string",
     "pkv_abi_version",
     "paged_decode_attention_noalloc",
+    "paged_attention_combine",
     # include/paged_kv_runtime.h: host page allocator and step planner
     "pkv_allocator_create",
     "pkv_allocator_destroy",
@@ -121,6 +122,8 @@ def _load() -> ctypes.CDLL:
     lib.paged_decode_attention_noalloc.argtypes = [cp, P, I32, I32, P, I32, P, I32, I32, F, P, P,
                                                    I32, P]
     lib.paged_decode_attention_noalloc.restype = ctypes.c_int
+    lib.paged_attention_combine.argtypes = [P, P, I32, I32, I32, P, P, P]
+    lib.paged_attention_combine.restype = ctypes.c_int
     lib.pkv_status_string.argtypes = [ctypes.c_int]
     lib.pkv_status_string.restype = ctypes.c_char_p
     lib.pkv_abi_version.restype = ctypes.c_int
@@ -351,6 +354,27 @@ def paged_decode_attention_noalloc(cache: PagedKVCache, q, page_table, seq_lens,
         page_table.shape[1], _ptr(seq_lens), B, int(max_seq_len), float(softmax_scale),
         _ptr(out), _ptr(lse), int(num_ctas), _stream(stream))
     _check("paged_decode_attention_noalloc", st)
+    return out, lse
+
+
+def paged_attention_combine(parts, lse_parts, out=None, lse=None, stream=None):
+    """Merge attention over disjoint key ranges.
+
+    ``parts`` bf16 ``[R, B, Hq, D]`` (normalised outputs of each part),
+    ``lse_parts`` fp32 ``[R, B, Hq]``.  Returns ``(out [B, Hq, D], lse [B, Hq])``.
+    """
+    _dev("parts", parts, torch.bfloat16, 4)
+    _dev("lse_parts", lse_parts, torch.float32, 3)
+    R, B, Hq, D = parts.shape
+    if tuple(lse_parts.shape) != (R, B, Hq):
+        raise ValueError("lse_parts must be [R, B, Hq]")
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=parts.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=parts.device)
+    _check("paged_attention_combine",
+           _lib.paged_attention_combine(_ptr(parts), _ptr(lse_parts), R, B * Hq, D, _ptr(out),
+                                        _ptr(lse), _stream(stream)))
     return out, lse
 
 

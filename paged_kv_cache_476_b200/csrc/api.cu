@@ -283,6 +283,20 @@ int paged_decode_attention(const pkv_cache* cache, const void* q, int32_t num_q_
   return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
+int paged_attention_combine(const void* parts, const float* lse_parts, int32_t num_parts,
+                            int32_t rows, int32_t head_dim, void* out, float* lse,
+                            void* stream) {
+  if (num_parts < 1 || rows < 0) return PKV_ERR_SHAPE;
+  if (head_dim != 64 && head_dim != 128) return PKV_ERR_HEAD_DIM;
+  if (rows == 0) return PKV_OK;
+  if (!parts || !lse_parts || !out) return PKV_ERR_NULL;
+  if (!aligned16(parts) || !aligned16(out)) return PKV_ERR_ALIGN;
+  if ((int64_t)num_parts * rows * head_dim >= INT64_C(1) << 40) return PKV_ERR_SHAPE;
+  cudaError_t e = launch_combine(parts, lse_parts, num_parts, rows, head_dim, out, lse,
+                                 static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
 int paged_prefill_chunk_attention(const pkv_cache* cache, const void* q, int32_t num_q_heads,
                                   int32_t gqa_group, const int32_t* cu_q_lens,
                                   const int32_t* page_table, int32_t max_pages_per_seq,

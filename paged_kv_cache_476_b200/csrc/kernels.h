@@ -61,6 +61,9 @@ cudaError_t decode_occupancy(int head_dim, int fmt, int group, int* ctas_per_sm)
 cudaError_t decode_run(int head_dim, int fmt, const CUtensorMap& tk, const CUtensorMap& tv,
                        const DecodeParams& p, int num_ctas, cudaStream_t stream);
 
+cudaError_t launch_combine(const void* parts, const float* lse_parts, int num_parts, int rows,
+                           int head_dim, void* out, float* lse, cudaStream_t stream);
+
 int check_cache(const pkv_cache* c);
 int check_group(const pkv_cache* c, int32_t num_q_heads, int32_t gqa_group);
 int encode_pool_map(CUtensorMap* map, void* base, bool fp8, int64_t rows, int row_elems,
