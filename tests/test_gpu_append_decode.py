@@ -259,3 +259,26 @@ def test_config_mixed_decode_part():
     torch.cuda.synchronize()
     ref, ref_lse = _oracle_decode(w)
     compare(out, lse, ref, ref_lse)
+
+
+def test_workspace_reused_across_batch_shapes():
+    # one workspace, zeroed once, serves calls with other shapes after it:
+    # the granule counter sits at a fixed offset and every call leaves it zero
+    import paged_kv_cache_476_b200 as pkv
+
+    big = workloads.build("wsA", 15, [3000, 9000, 40, 2500] * 8, [1] * 32, page_size=64,
+                          num_q_heads=32, num_kv_heads=8, head_dim=128, pool_slack=0.1)
+    small = workloads.build("wsB", 16, [700, 5, 1500], [1] * 3, page_size=64,
+                            num_q_heads=16, num_kv_heads=2, head_dim=128, pool_slack=0.2)
+    need = max(pkv.paged_decode_workspace_bytes(32, 32, 8, 128, 9001),
+               pkv.paged_decode_workspace_bytes(3, 16, 2, 128, 1501))
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for w in (big, small, big, small):
+        st = GpuState(w)
+        st.append_step()
+        q, table, lens, max_len = st.decode_inputs()
+        out, lse = pkv.paged_decode_attention(st.cache, q, table, lens, max_len, w.softmax_scale,
+                                              workspace=ws)
+        torch.cuda.synchronize()
+        ref, ref_lse = _oracle_decode(w)
+        compare(out, lse, ref, ref_lse)
