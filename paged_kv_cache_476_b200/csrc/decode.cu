@@ -77,13 +77,12 @@ struct Layout {
   static constexpr int kBoxB = kTile * kBoxRowB;
   static constexpr int kTileB = kNumBox * kBoxB;  // one K (or V) tile
   static constexpr int kStageB = 2 * kTileB;
-  static constexpr int kConvB = 16 * D * 2;  // per-warp f16 V tile (E4M3 only)
 };
 
 // Shared-memory carve-up; the Q slices and the reduction buffers are sized
 // by the GQA group so that two CTAs fit on one SM.
 struct SmemPlan {
-  uint32_t q, conv, red_o, red_m, red_l, bars, info, misc, total;
+  uint32_t q, red_o, red_m, red_l, bars, info, misc, total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
@@ -96,8 +95,6 @@ __host__ __device__ inline SmemPlan smem_plan(int G) {
   s.q = o;
   o += kStages * align_up(G * D * 2, 128);
   o = align_up(o, 1024);
-  s.conv = o;
-  if (k8(kFmt)) o += kConsumerWarps * Ly::kConvB;
   s.red_o = o;
   o += kConsumerWarps * G * D * 4;
   s.red_m = o;
@@ -158,7 +155,6 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t kQStride = align_up(G * D * 2, 128);
   uint8_t* tiles = smem;
   uint8_t* qbuf = smem + sp.q;
-  uint8_t* conv = smem + sp.conv;
   float* red_o = reinterpret_cast<float*>(smem + sp.red_o);
   float* red_m = reinterpret_cast<float*>(smem + sp.red_m);
   float* red_l = reinterpret_cast<float*>(smem + sp.red_l);
@@ -574,15 +570,18 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int e = 0; e < 4; ++e) pr[e] = fast_exp2(x[e] - m_new);
       l_part = l_part * alpha + (pr[0] + pr[1]) + (pr[2] + pr[3]);
       m_run = m_new;
-      // alpha belongs to head gid; O^T columns are heads 2*tid4 and 2*tid4+1
-      const float a_lo = __shfl_sync(0xffffffffu, alpha, 8 * tid4);
-      const float a_hi = __shfl_sync(0xffffffffu, alpha, 8 * tid4 + 4);
+      // alpha belongs to head gid; O^T columns are heads 2*tid4 and 2*tid4+1.
+      // Once the running max settles (most tiles), no row's alpha moves.
+      if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        const float a_lo = __shfl_sync(0xffffffffu, alpha, 8 * tid4);
+        const float a_hi = __shfl_sync(0xffffffffu, alpha, 8 * tid4 + 4);
 #pragma unroll
-      for (int m = 0; m < D / 16; ++m) {
-        ot[m][0] *= a_lo;
-        ot[m][1] *= a_hi;
-        ot[m][2] *= a_lo;
-        ot[m][3] *= a_hi;
+        for (int m = 0; m < D / 16; ++m) {
+          ot[m][0] *= a_lo;
+          ot[m][1] *= a_hi;
+          ot[m][2] *= a_lo;
+          ot[m][3] *= a_hi;
+        }
       }
       // ---- O^T += V^T P^T over my 16 tokens (P^T comes straight from S) ----
       uint32_t pa0, pa2;
@@ -601,67 +600,45 @@ __global__ void __launch_bounds__(kThreads, 2)
         vm1 = (2 * tid4 + 8 < valid ? 0x0000ffffu : 0u) |
               (2 * tid4 + 9 < valid ? 0xffff0000u : 0u);
       }
-      uint32_t vsrc;
       if constexpr (!k8(kFmt)) {
-        vsrc = vbase;
-      } else {
-        // E4M3 -> f16 copy of my 16 V rows into my conversion tile, laid out
-        // like a bf16 tile (256-byte rows as two 128-byte swizzled boxes).
-        uint8_t* cv = conv + warp * Ly::kConvB;
-        const uint32_t cbase = smem_u32(cv);
-        constexpr int kChunks = 16 * D / 16;  // 16-byte E4M3 chunks of my rows
 #pragma unroll
-        for (int k = 0; k < kChunks / 32; ++k) {
-          const int ci = lane + 32 * k;
-          const int r = ci / (D / 16);
-          const int ch = ci % (D / 16);
-          uint4 raw;
-          const uint32_t src = tile_addr<Ly::kBoxRowB, kTile>(vbase, 16 * warp + r, ch);
-          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(raw.x), "=r"(raw.y), "=r"(raw.z), "=r"(raw.w)
-                       : "r"(src));
-          uint4 h0, h1;
-          h0.x = kv8x2_to_f16x2<kFmt>(raw.x & 0xffff);
-          h0.y = kv8x2_to_f16x2<kFmt>(raw.x >> 16);
-          h0.z = kv8x2_to_f16x2<kFmt>(raw.y & 0xffff);
-          h0.w = kv8x2_to_f16x2<kFmt>(raw.y >> 16);
-          h1.x = kv8x2_to_f16x2<kFmt>(raw.z & 0xffff);
-          h1.y = kv8x2_to_f16x2<kFmt>(raw.z >> 16);
-          h1.z = kv8x2_to_f16x2<kFmt>(raw.w & 0xffff);
-          h1.w = kv8x2_to_f16x2<kFmt>(raw.w >> 16);
-          const uint32_t d0 = tile_addr<128, 16>(cbase, r, 2 * ch);
-          const uint32_t d1 = tile_addr<128, 16>(cbase, r, 2 * ch + 1);
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(d0), "r"(h0.x),
-                       "r"(h0.y), "r"(h0.z), "r"(h0.w)
-                       : "memory");
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(d1), "r"(h1.x),
-                       "r"(h1.y), "r"(h1.z), "r"(h1.w)
-                       : "memory");
-        }
-        __syncwarp();
-        vsrc = cbase;
-      }
-#pragma unroll
-      for (int m = 0; m < D / 16; ++m) {
-        // A = V^T rows d 16m..16m+15: matrices (tokens 0-7, chunk 2m), (0-7, 2m+1),
-        // (8-15, 2m), (8-15, 2m+1), transposed on load
-        const int chunk = 2 * m + (mat & 1);
-        uint32_t a0, a1, a2, a3;
-        if constexpr (!k8(kFmt)) {
+        for (int m = 0; m < D / 16; ++m) {
+          // A = V^T rows d 16m..16m+15: matrices (tokens 0-7, chunk 2m), (0-7, 2m+1),
+          // (8-15, 2m), (8-15, 2m+1), transposed on load
+          const int chunk = 2 * m + (mat & 1);
           const int row = 16 * warp + mrow + (mat >> 1) * 8;
-          ldsm_x4_t(tile_addr<Ly::kBoxRowB, kTile>(vsrc, row, chunk), a0, a1, a2, a3);
-        } else {
-          const int row = mrow + (mat >> 1) * 8;
-          ldsm_x4_t(tile_addr<128, 16>(vsrc, row, chunk), a0, a1, a2, a3);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(tile_addr<Ly::kBoxRowB, kTile>(vbase, row, chunk), a0, a1, a2, a3);
+          mma_bf16(ot[m], a0 & vm0, a1 & vm0, a2 & vm1, a3 & vm1, pa0, pa2);
         }
-        a0 &= vm0;
-        a1 &= vm0;
-        a2 &= vm1;
-        a3 &= vm1;
-        if constexpr (!k8(kFmt))
-          mma_bf16(ot[m], a0, a1, a2, a3, pa0, pa2);
-        else
-          mma_f16(ot[m], a0, a1, a2, a3, pa0, pa2);
+      } else {
+        // One-byte V codes straight from the landed tile.  A transposed load
+        // of 16-bit elements (byte pairs d, d+1) gives each thread, per 8x8
+        // matrix, codes of tokens (2*tid4, 2*tid4+1) x bytes (2*gid, 2*gid+1)
+        // of a 16-byte chunk; two exact conversions and a swap of 16-bit
+        // halves make the A fragment of V^T with row gid = d 16m + 2*gid and
+        // row gid+8 = d 16m + 2*gid + 1 (the snapshot below undoes the order).
+        auto v_rows = [&](uint32_t codes, uint32_t& even_d, uint32_t& odd_d) {
+          const uint32_t t0 = kv8x2_to_f16x2<kFmt>(codes & 0xffff);  // token 2*tid4
+          const uint32_t t1 = kv8x2_to_f16x2<kFmt>(codes >> 16);     // token 2*tid4+1
+          even_d = __byte_perm(t0, t1, 0x5410);
+          odd_d = __byte_perm(t0, t1, 0x7632);
+        };
+#pragma unroll
+        for (int m = 0; m < D / 16; m += 2) {
+          // matrices: (tokens 0-7, chunk m), (8-15, m), (0-7, m+1), (8-15, m+1)
+          const int row = 16 * warp + mrow + (mat & 1) * 8;
+          const int chunk = m + (mat >> 1);
+          uint32_t r0, r1, r2, r3;
+          ldsm_x4_t(tile_addr<Ly::kBoxRowB, kTile>(vbase, row, chunk), r0, r1, r2, r3);
+          uint32_t a0, a1, a2, a3;
+          v_rows(r0, a0, a1);
+          v_rows(r1, a2, a3);
+          mma_f16(ot[m], a0 & vm0, a1 & vm0, a2 & vm1, a3 & vm1, pa0, pa2);
+          v_rows(r2, a0, a1);
+          v_rows(r3, a2, a3);
+          mma_f16(ot[m + 1], a0 & vm0, a1 & vm0, a2 & vm1, a3 & vm1, pa0, pa2);
+        }
       }
     }
     if (t_flags & kSegLast) {
@@ -679,16 +656,20 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int h0 = 2 * tid4, h1 = 2 * tid4 + 1;
       float* r0 = red_o + (warp * G + h0) * D;
       float* r1 = red_o + (warp * G + h1) * D;
+      // fragment rows gid and gid+8 of d-tile m hold d 16m + gid and +8
+      // (bf16), or 16m + 2*gid and +1 (one-byte codes, see the PV product)
+      const int d_step = k8(kFmt) ? 1 : 8;
+      const int d_lane = k8(kFmt) ? 2 * gid : gid;
 #pragma unroll
       for (int m = 0; m < D / 16; ++m) {
-        const int d = 16 * m + gid;
+        const int d = 16 * m + d_lane;
         if (h0 < G) {
           r0[d] = ot[m][0];
-          r0[d + 8] = ot[m][2];
+          r0[d + d_step] = ot[m][2];
         }
         if (h1 < G) {
           r1[d] = ot[m][1];
-          r1[d + 8] = ot[m][3];
+          r1[d + d_step] = ot[m][3];
         }
       }
     }
