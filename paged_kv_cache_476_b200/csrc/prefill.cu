@@ -314,12 +314,15 @@ struct ChunkCost {
   int32_t ctx, n, pairs;  // pairs: items of the chunk that exist in the grid
 };
 
-// Items of chunk `cc` whose cost is below k.
+// Items of chunk `cc` whose cost is below k.  Straight-line: the warp runs
+// it for every chunk slot at every step of the search, and branches there
+// split the lanes.
 __device__ __forceinline__ int32_t pairs_below(const ChunkCost& cc, int32_t k, int32_t pair_tokens) {
   const int64_t lim = (int64_t)kKeys * (k - 1) - cc.ctx;  // cost < k  <=>  ctx + e <= lim
-  if (lim >= cc.n) return cc.pairs;
-  if (lim <= 0) return 0;
-  return min((int32_t)(lim / pair_tokens), cc.pairs);
+  // clamped to [0, n] (n < 2^31), so that a 32-bit division serves
+  const uint32_t v = (uint32_t)max(min(lim, (int64_t)cc.n), (int64_t)0);
+  const int32_t q = min((int32_t)(v / (uint32_t)pair_tokens), cc.pairs);
+  return lim >= cc.n ? cc.pairs : q;
 }
 
 // Sum over the warp's chunks of the items with cost >= k.
@@ -348,7 +351,7 @@ __device__ bool lpt_item(const Params& p, uint32_t rank, int32_t pair_tokens, in
       const int32_t L = __ldg(p.seq_lens + c);
       cc[i].n = n;
       cc[i].ctx = (int32_t)max((int64_t)L - n, (int64_t)0);
-      cc[i].pairs = min((int32_t)(((int64_t)n + pair_tokens - 1) / pair_tokens), p.pair_slots);
+      cc[i].pairs = min((int32_t)(((uint32_t)n + pair_tokens - 1) / (uint32_t)pair_tokens), p.pair_slots);
       kmax = max(kmax, (int32_t)(((int64_t)cc[i].ctx + n + kKeys - 1) / kKeys));
     }
   }
