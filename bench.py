@@ -349,6 +349,43 @@ def run_ours(args, rank, world, device, dist):
     elapsed = max_over_ranks(g0.elapsed_time(g1) / 1e3, dist, device)  # seconds
     del graph
 
+    # The same decode step with the append fused into the decode launch
+    # (paged_decode_attention_append), graph-replayed the same way: decode
+    # configurations only, where every sequence appends one token.
+    fused_s = None
+    one_each = (not has_pf and len(w.decode_rows) == w.batch
+                and bool((np.asarray(w.new_lens) == 1).all()))
+    if one_each:
+        def fused_step():
+            pkv.paged_decode_attention_append(cache, st["dec_q"], st["dec_table"], st["dec_lens"],
+                                              st["dec_max"], st["k_new"], st["v_new"],
+                                              w.softmax_scale, out=st["dec_out"],
+                                              lse=st["dec_lse"], workspace=ws,
+                                              num_ctas=args.num_ctas)
+
+        fgraph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(gstream):
+            fused_step()
+            gstream.synchronize()
+            with torch.cuda.graph(fgraph, stream=gstream):
+                fused_step()
+        torch.cuda.synchronize()
+        for _ in range(max(3, args.warmup)):
+            fgraph.replay()
+        f_steps = max(1, min(args.steps, 500))
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        g0.record(stream)
+        for _ in range(f_steps):
+            fgraph.replay()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        fused_s = max_over_ranks(g0.elapsed_time(g1) / 1e3 / f_steps, dist, device)
+        del fgraph
+        if int(st["flags"].item()) != 0:
+            raise RuntimeError(f"device error flags {int(st['flags'].item()):#x}")
+
     # ---------------------------------------------------------------- e2e
     # Through the public API with host buffers: per step, H2D of the step's
     # inputs (q, new K/V, lengths, page table) from pinned memory and D2H of
@@ -478,6 +515,11 @@ def run_ours(args, rank, world, device, dist):
         "eager": {"value": round(whole_job_rate(step_bytes, world, eager_s) / 1e9, 2),
                   "unit": "GB/s", "ms_per_step": round(eager_s * 1e3, 5),
                   "what": "the same step as separate launches"},
+        "fused": None if fused_s is None else {
+            "value": round(whole_job_rate(step_bytes, world, fused_s) / 1e9, 2), "unit": "GB/s",
+            "ms_per_step": round(fused_s * 1e3, 5),
+            "what": "the same step with the append fused into the decode launch "
+                    "(paged_decode_attention_append), graph-replayed"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
         "device_error_flags": flags,

@@ -168,6 +168,37 @@ int paged_decode_attention(const pkv_cache* cache, const void* q, int32_t num_q_
                            void* stream);
 
 /*
+ * Decode step with the append fused in: one launch stores each sequence's
+ * new token and attends over all its tokens, the new one included.  Same
+ * arguments and result as paged_decode_attention, plus the new tokens:
+ *   k_new, v_new  bf16 [batch][num_kv_heads][head_dim], 16-byte aligned; row b
+ *                 is sequence b's new token, stored at position
+ *                 seq_lens[b] - 1 (seq_lens counts it)
+ * The pools end up holding exactly the bytes of
+ *   paged_kv_append(cache, page_table, max_pages_per_seq,
+ *                   seq_lens_before = seq_lens - 1, cu_new = 0, 1, ..., batch, ...)
+ * (bf16 bits; E4M3 or INT8 codes of x / scale with the page's scales), and out
+ * and lse are those of paged_decode_attention on that cache.  The token is
+ * stored by the CTA that reads the tile holding it, which then orders the
+ * stores before its own tile loads; the new K/V therefore make one trip
+ * through L2 instead of a separate kernel's.  Rows with seq_lens[b] = 0 store
+ * nothing.  A row whose length exceeds max_pages_per_seq * page_size, or
+ * whose page id is invalid, stores nothing and sets the error flag, as the
+ * decode does.  Source: concept page "PagedAttention 及 KV 快取管理" (each
+ * step appends the token's K/V to the sequence's pages, then attention reads
+ * them) and "編譯期圖最佳化" (the paged operations fused into the engine).
+ * Errors: PKV_ERR_NULL for a missing k_new / v_new, PKV_ERR_ALIGN for a
+ * misaligned one, then every check of paged_decode_attention.
+ */
+int paged_decode_attention_append(const pkv_cache* cache, const void* q, int32_t num_q_heads,
+                                  int32_t gqa_group, const int32_t* page_table,
+                                  int32_t max_pages_per_seq, const int32_t* seq_lens,
+                                  int32_t batch, int32_t max_seq_len, float softmax_scale,
+                                  const void* k_new, const void* v_new, void* out, float* lse,
+                                  void* workspace, size_t workspace_bytes, int32_t num_ctas,
+                                  void* stream);
+
+/*
  * Causal prefill-chunk attention over the paged cache.  Chunk c owns the
  * queries [cu_q_lens[c], cu_q_lens[c+1]) of the packed q and has seq_lens[c]
  * tokens cached AFTER its append (its own new tokens included).  Query i of a

@@ -47,6 +47,7 @@ EXPORTED = (
     "pkv_abi_version",
     "paged_decode_attention_noalloc",
     "paged_attention_combine",
+    "paged_decode_attention_append",
     # include/paged_kv_runtime.h: host page allocator and step planner
     "pkv_allocator_create",
     "pkv_allocator_destroy",
@@ -116,6 +117,9 @@ def _load() -> ctypes.CDLL:
     lib.paged_decode_attention.argtypes = [cp, P, I32, I32, P, I32, P, I32, I32, F, P, P, P, SZ,
                                            I32, P]
     lib.paged_decode_attention.restype = ctypes.c_int
+    lib.paged_decode_attention_append.argtypes = [cp, P, I32, I32, P, I32, P, I32, I32, F, P, P,
+                                                  P, P, P, SZ, I32, P]
+    lib.paged_decode_attention_append.restype = ctypes.c_int
     lib.paged_prefill_chunk_attention.argtypes = [cp, P, I32, I32, P, P, I32, P, I32, I32, I32,
                                                   F, P, P, P]
     lib.paged_prefill_chunk_attention.restype = ctypes.c_int
@@ -300,6 +304,43 @@ def paged_decode_attention(cache: PagedKVCache, q, page_table, seq_lens, max_seq
         page_table.shape[1], _ptr(seq_lens), B, int(max_seq_len), float(softmax_scale),
         _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), int(num_ctas), _stream(stream))
     _check("paged_decode_attention", st)
+    return out, lse
+
+
+def paged_decode_attention_append(cache: PagedKVCache, q, page_table, seq_lens, max_seq_len: int,
+                                  k_new, v_new, softmax_scale: Optional[float] = None, out=None,
+                                  lse=None, workspace=None, num_ctas: int = 0,
+                                  want_lse: bool = True, stream=None):
+    """A decode step with the append fused in.
+
+    ``k_new``/``v_new`` bf16 ``[B, Hkv, D]`` hold each sequence's new token,
+    stored at position ``seq_lens[b] - 1`` (``seq_lens`` counts it) by the
+    same launch that then attends over all ``seq_lens[b]`` tokens.  Equal to
+    ``paged_kv_append`` of one token per sequence followed by
+    ``paged_decode_attention``.  Returns ``(out, lse)`` like the latter.
+    """
+    _dev("q", q, torch.bfloat16, 3)
+    _dev("page_table", page_table, torch.int32, 2)
+    _dev("seq_lens", seq_lens, torch.int32, 1)
+    _dev("k_new", k_new, torch.bfloat16, 3)
+    _dev("v_new", v_new, torch.bfloat16, 3)
+    B, Hq, D = q.shape
+    if tuple(k_new.shape) != (B, cache.num_kv_heads, D) or k_new.shape != v_new.shape:
+        raise ValueError("k_new and v_new must be [batch, num_kv_heads, head_dim]")
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = decode_workspace(cache, B, Hq, max_seq_len, num_ctas)
+    st = _lib.paged_decode_attention_append(
+        ctypes.byref(cache.c_struct), _ptr(q), Hq, Hq // cache.num_kv_heads, _ptr(page_table),
+        page_table.shape[1], _ptr(seq_lens), B, int(max_seq_len), float(softmax_scale),
+        _ptr(k_new), _ptr(v_new), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+        int(num_ctas), _stream(stream))
+    _check("paged_decode_attention_append", st)
     return out, lse
 
 

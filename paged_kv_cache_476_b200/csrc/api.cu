@@ -112,7 +112,7 @@ using namespace pkv;
 
 extern "C" {
 
-int pkv_abi_version(void) { return (1 << 16) | 0; }
+int pkv_abi_version(void) { return (1 << 16) | 1; }
 
 const char* pkv_status_string(int status) {
   switch (status) {
@@ -206,12 +206,14 @@ size_t paged_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t 
   return (bytes + 255) & ~size_t(255);
 }
 
-int paged_decode_attention(const pkv_cache* cache, const void* q, int32_t num_q_heads,
-                           int32_t gqa_group, const int32_t* page_table,
-                           int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
-                           int32_t max_seq_len, float softmax_scale, void* out, float* lse,
-                           void* workspace, size_t workspace_bytes, int32_t num_ctas,
-                           void* stream) {
+// Decode, with the fused append of one new token per sequence when k_new
+// and v_new are given (both null otherwise).
+static int decode_entry(const pkv_cache* cache, const void* q, int32_t num_q_heads,
+                        int32_t gqa_group, const int32_t* page_table, int32_t max_pages_per_seq,
+                        const int32_t* seq_lens, int32_t batch, int32_t max_seq_len,
+                        float softmax_scale, const void* k_new, const void* v_new, void* out,
+                        float* lse, void* workspace, size_t workspace_bytes, int32_t num_ctas,
+                        void* stream) {
   int st = check_cache(cache);
   if (st) return st;
   if ((st = check_group(cache, num_q_heads, gqa_group))) return st;
@@ -259,7 +261,7 @@ int paged_decode_attention(const pkv_cache* cache, const void* q, int32_t num_q_
   off = (off + 15) & ~size_t(15);
   int2* unit_info = reinterpret_cast<int2*>(ws + off);
 
-  DecodeParams p;
+  DecodeParams p{};
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.page_table = page_table;
   p.seq_lens = seq_lens;
@@ -271,6 +273,12 @@ int paged_decode_attention(const pkv_cache* cache, const void* q, int32_t num_q_
   p.part_ml = part_ml;
   p.unit_info = unit_info;
   p.flags = cache->error_flags;
+  if (k_new) {
+    p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+    p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+    p.k_pool = static_cast<uint8_t*>(cache->k_pool);
+    p.v_pool = static_cast<uint8_t*>(cache->v_pool);
+  }
   p.batch = batch;
   p.num_q_heads = num_q_heads;
   p.num_kv_heads = cache->num_kv_heads;
@@ -281,6 +289,31 @@ int paged_decode_attention(const pkv_cache* cache, const void* q, int32_t num_q_
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   cudaError_t e = decode_run(D, fmt, tk, tv, p, ctas, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+int paged_decode_attention(const pkv_cache* cache, const void* q, int32_t num_q_heads,
+                           int32_t gqa_group, const int32_t* page_table,
+                           int32_t max_pages_per_seq, const int32_t* seq_lens, int32_t batch,
+                           int32_t max_seq_len, float softmax_scale, void* out, float* lse,
+                           void* workspace, size_t workspace_bytes, int32_t num_ctas,
+                           void* stream) {
+  return decode_entry(cache, q, num_q_heads, gqa_group, page_table, max_pages_per_seq, seq_lens,
+                      batch, max_seq_len, softmax_scale, nullptr, nullptr, out, lse, workspace,
+                      workspace_bytes, num_ctas, stream);
+}
+
+int paged_decode_attention_append(const pkv_cache* cache, const void* q, int32_t num_q_heads,
+                                  int32_t gqa_group, const int32_t* page_table,
+                                  int32_t max_pages_per_seq, const int32_t* seq_lens,
+                                  int32_t batch, int32_t max_seq_len, float softmax_scale,
+                                  const void* k_new, const void* v_new, void* out, float* lse,
+                                  void* workspace, size_t workspace_bytes, int32_t num_ctas,
+                                  void* stream) {
+  if (batch > 0 && (!k_new || !v_new)) return PKV_ERR_NULL;
+  if (batch > 0 && (!aligned16(k_new) || !aligned16(v_new))) return PKV_ERR_ALIGN;
+  return decode_entry(cache, q, num_q_heads, gqa_group, page_table, max_pages_per_seq, seq_lens,
+                      batch, max_seq_len, softmax_scale, k_new, v_new, out, lse, workspace,
+                      workspace_bytes, num_ctas, stream);
 }
 
 int paged_attention_combine(const void* parts, const float* lse_parts, int32_t num_parts,

@@ -30,13 +30,6 @@ __device__ __forceinline__ int owner_of(const int32_t* cu_new, int batch, int to
   return lo;
 }
 
-// Symmetric INT8 code of a quotient: round to nearest even, clamp to +-127.
-__device__ __forceinline__ uint32_t int8_code(float y) {
-  if (y != y) return 0u;
-  const int q = __float2int_rn(fminf(fmaxf(y, -127.f), 127.f));
-  return static_cast<uint32_t>(q) & 0xffu;
-}
-
 template <int kFmt>
 __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
   const int vecs_per_row = p.head_dim / 8;                 // 16-byte vectors per (token, head)
@@ -80,14 +73,7 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
       uint32_t w[2];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        float2 f = __bfloat1622float2(x[k]);
-        f.x = __fdiv_rn(f.x, s);
-        f.y = __fdiv_rn(f.y, s);
-        uint16_t two;
-        if constexpr (kFmt == PKV_KV_INT8)
-          two = static_cast<uint16_t>(int8_code(f.x) | (int8_code(f.y) << 8));
-        else
-          two = __nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
+        const uint16_t two = encode8x2<kFmt>(x[k], s);
         if (k & 1)
           w[k >> 1] |= static_cast<uint32_t>(two) << 16;
         else

@@ -200,6 +200,29 @@ __device__ __forceinline__ uint32_t s8x2_to_f16x2(uint16_t codes) {
   return v;
 }
 
+// Symmetric INT8 code of a quotient: round to nearest even, clamp to +-127,
+// NaN stored as 0.
+__device__ __forceinline__ uint32_t int8_code(float y) {
+  if (y != y) return 0u;
+  const int q = __float2int_rn(fminf(fmaxf(y, -127.f), 127.f));
+  return static_cast<uint32_t>(q) & 0xffu;
+}
+
+// Codes of pool format kFmt for two bf16 values and their (page, head) scale
+// (low byte = first value): the IEEE fp32 quotient x / scale, then E4M3 with
+// round-to-nearest-even and satfinite, or the INT8 code above.  Every writer
+// of one-byte pools goes through here, so all write the same bytes.
+template <int kFmt>
+__device__ __forceinline__ uint16_t encode8x2(__nv_bfloat162 x, float scale) {
+  float2 f = __bfloat1622float2(x);
+  f.x = __fdiv_rn(f.x, scale);
+  f.y = __fdiv_rn(f.y, scale);
+  if constexpr (kFmt == PKV_KV_INT8)
+    return static_cast<uint16_t>(int8_code(f.x) | (int8_code(f.y) << 8));
+  else
+    return static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3));
+}
+
 // Two 8-bit KV codes of format kFmt to an f16x2 (exact for both formats).
 template <int kFmt>
 __device__ __forceinline__ uint32_t kv8x2_to_f16x2(uint16_t codes) {

@@ -141,6 +141,33 @@ __device__ __forceinline__ int32_t clamp_len(const DecodeParams& p, int32_t len,
   return len;
 }
 
+// Fused append: the producer warp writes sequence b's newest token (K and V
+// of kv head g, from k_new/v_new [B][Hkv][D]) into pool row (pid, g, slot):
+// the bytes paged_kv_append writes for it (bf16 bits, or the one-byte codes
+// of the quotient by the page's scale).  Four values per lane.
+template <int D, int kFmt>
+__device__ __forceinline__ void append_newest(const DecodeParams& p, int b, int g, int pid,
+                                              int slot, float ks, float vs, int lane) {
+  const int64_t src = ((int64_t)b * p.num_kv_heads + g) * D;
+  const int64_t dst = (((int64_t)pid * p.num_kv_heads + g) * p.page_size + slot) * D;
+  for (int e = lane * 4; e < D; e += 128) {
+    const uint2 kx = *reinterpret_cast<const uint2*>(p.k_new + src + e);
+    const uint2 vx = *reinterpret_cast<const uint2*>(p.v_new + src + e);
+    if constexpr (!k8(kFmt)) {
+      *reinterpret_cast<uint2*>(p.k_pool + (dst + e) * 2) = kx;
+      *reinterpret_cast<uint2*>(p.v_pool + (dst + e) * 2) = vx;
+    } else {
+      auto codes = [](uint2 x, float s) -> uint32_t {
+        const uint32_t lo = encode8x2<kFmt>(*reinterpret_cast<const __nv_bfloat162*>(&x.x), s);
+        const uint32_t hi = encode8x2<kFmt>(*reinterpret_cast<const __nv_bfloat162*>(&x.y), s);
+        return lo | (hi << 16);
+      };
+      *reinterpret_cast<uint32_t*>(p.k_pool + dst + e) = codes(kx, ks);
+      *reinterpret_cast<uint32_t*>(p.v_pool + dst + e) = codes(vx, vs);
+    }
+  }
+}
+
 template <int D, int kFmt, int kStages>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
@@ -343,6 +370,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
       int pid = __shfl_sync(0xffffffffu, my_pid, j - cache_j0);
+      const bool page_ok = pid >= 0 && pid < p.num_pages;
       float ks = 1.f, vs = 1.f;
       if constexpr (k8(kFmt)) {
         ks = __shfl_sync(0xffffffffu, my_ks, j - cache_j0);
@@ -359,6 +387,16 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (lane == 0) flag_error(p.flags, PKV_FLAG_BAD_PAGE);
       }
       if (bad) pid = 0;
+      // Fused append: this CTA is the one that reads the tile holding the
+      // sequence's newest token (position len - 1), so it stores the token
+      // first (as paged_kv_append would: whenever the page id is valid) and
+      // orders those generic-proxy stores before its own bulk-tensor loads.
+      if (p.k_new && t == ntile - 1 && page_ok && __ldg(p.seq_lens + b) == len) {
+        append_newest<D, kFmt>(p, b, g, __shfl_sync(0xffffffffu, my_pid, j - cache_j0),
+                               (len - 1) % p.page_size, ks, vs, lane);
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __syncwarp();
+      }
       const bool first = (i == 0) || (t == 0);
       if (first) seg_first_t = t;
       const bool last = (i == n_tiles - 1) || (t == ntile - 1);

@@ -45,6 +45,12 @@ struct DecodeParams {
   float2* part_ml;     // [U + C][G]
   int2* unit_info;     // [U]: (first partial slot, number of segments)
   int32_t* flags;
+  // Fused append (all null otherwise): one new token per sequence, at
+  // position seq_lens[b] - 1, written into the pools before it is read.
+  const __nv_bfloat16* k_new;  // [B][Hkv][D]
+  const __nv_bfloat16* v_new;
+  uint8_t* k_pool;
+  uint8_t* v_pool;
   int32_t batch;
   int32_t num_q_heads;
   int32_t num_kv_heads;
