@@ -20,6 +20,9 @@ Functions and what they follow (pages on TensorRT-LLM):
                       (yololab.net guide, "FP8 與極致量化")
 * ``int8_*``          symmetric INT8 codec (concept page, "關鍵機制"
                       quantisation bullet: INT8 KV cache)
+* ``e2m1_*`` / ``nvfp4_*``   FP4 (E2M1) codec with E4M3 block scales per 16
+                      values (solosoft post: FP4 quantisation needs
+                      Blackwell; the block layout is a reading)
 
 Every function is pinned by ``tests/test_oracle_*.py`` against brute force,
 library special cases, closed forms and invariants.
@@ -87,6 +90,14 @@ def _declare(L):
     L.oracle_int8_encode.argtypes = [_F]
     L.oracle_int8_encode.restype = ctypes.c_int8
     L.oracle_int8_quantize_array.argtypes = [_P, _P, _P, _I64]
+    L.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
+    L.oracle_e2m1_decode.restype = _D
+    L.oracle_e2m1_encode.argtypes = [_F]
+    L.oracle_e2m1_encode.restype = ctypes.c_uint8
+    L.oracle_e2m1_encode_array.argtypes = [_P, _P, _I64]
+    L.oracle_nvfp4_quantize_row.argtypes = [_P, _I64, _F, _P, _P]
+    L.oracle_nvfp4_value.argtypes = [_P, _P, _F, _I64]
+    L.oracle_nvfp4_value.restype = _D
     cache = [_P, _P, _P, _P, _I, _I, _I, _I, _I]
     L.oracle_append.argtypes = cache + [_P, _I, _P, _P, _I, _P, _P]
     L.oracle_append.restype = _I
@@ -156,6 +167,51 @@ def int8_quantize(x_bits, scale) -> np.ndarray:
     scale = _c(np.broadcast_to(scale, x_bits.shape), np.float32)
     out = np.empty(x_bits.shape, np.int8)
     lib().oracle_int8_quantize_array(_ptr(x_bits), _ptr(scale), _ptr(out), x_bits.size)
+    return out
+
+
+def e2m1_decode(codes) -> np.ndarray:
+    """Values of E2M1 codes (low 4 bits), fp64."""
+    return np.array([lib().oracle_e2m1_decode(int(c) & 0xF) for c in np.ravel(codes)],
+                    np.float64).reshape(np.shape(codes))
+
+
+def e2m1_encode(y) -> np.ndarray:
+    """E2M1 codes of fp32 values: nearest, ties to even, saturating at +-6, NaN -> 0."""
+    y = _c(y, np.float32)
+    out = np.empty(y.shape, np.uint8)
+    lib().oracle_e2m1_encode_array(_ptr(y), _ptr(out), y.size)
+    return out
+
+
+def nvfp4_quantize(x_bits, scale):
+    """NVFP4 codes of bf16 rows (uint16 bits ``[rows, n]``, n a multiple of 16)
+    with one fp32 scale per row: ``(packed uint8 [rows, n/2], block scales
+    uint8 [rows, n/16])``, the even element in the low nibble."""
+    x_bits = _c(np.atleast_2d(x_bits), np.uint16)
+    rows, n = x_bits.shape
+    if n % 16:
+        raise ValueError("row length must be a multiple of 16")
+    scale = _c(np.broadcast_to(scale, (rows,)), np.float32)
+    packed = np.empty((rows, n // 2), np.uint8)
+    blocks = np.empty((rows, n // 16), np.uint8)
+    for r in range(rows):
+        lib().oracle_nvfp4_quantize_row(_ptr(x_bits[r]), n, float(scale[r]), _ptr(packed[r]),
+                                        _ptr(blocks[r]))
+    return packed, blocks
+
+
+def nvfp4_dequantize(packed, blocks, scale) -> np.ndarray:
+    """Stored values (fp64 ``[rows, n]``) of rows quantised by ``nvfp4_quantize``."""
+    packed = _c(np.atleast_2d(packed), np.uint8)
+    blocks = _c(np.atleast_2d(blocks), np.uint8)
+    rows, n = packed.shape[0], packed.shape[1] * 2
+    scale = _c(np.broadcast_to(scale, (rows,)), np.float32)
+    out = np.empty((rows, n), np.float64)
+    for r in range(rows):
+        for i in range(n):
+            out[r, i] = lib().oracle_nvfp4_value(_ptr(packed[r]), _ptr(blocks[r]),
+                                                 float(scale[r]), i)
     return out
 
 

@@ -41,6 +41,9 @@
  *    quantisation bullet): the same per-(page, kv head) scales; stored code =
  *    round-half-even of the fp32 quotient clamped to [-127, 127] (-128 never
  *    stored), NaN -> 0; value = code * scale;
+ *  - NVFP4 (the pages: FP4 quantisation needs Blackwell; codec only so far):
+ *    E2M1 codes, an E4M3 scale per 16 head_dim values of a row, and the same
+ *    per-(page, kv head) fp32 scale; see the NVFP4 section below;
  *  - a sequence of length 0 yields out = 0 and lse = -inf.
  */
 #include <math.h>
@@ -175,6 +178,94 @@ int8_t oracle_int8_quantize(uint16_t x_bits, float scale) {
 void oracle_int8_quantize_array(const uint16_t* x_bits, const float* scale, int8_t* codes,
                                 int64_t n) {
   for (int64_t i = 0; i < n; ++i) codes[i] = oracle_int8_quantize(x_bits[i], scale[i]);
+}
+
+/* ----------------------------------------------------------------- NVFP4 */
+/*
+ * FP4 pools (the pages say only that FP4 quantisation needs Blackwell; the
+ * layout below is this library's reading): E2M1 element codes; the 16
+ * consecutive head_dim values of one (token, kv head) row share an E4M3
+ * block scale; the per-(page, kv head) fp32 scale of the other one-byte
+ * formats multiplies both.
+ *
+ * E2M1: 1 sign, 2 exponent (bias 1), 1 mantissa bit; no infinities, no NaN.
+ *   exponent field 0:      value = m * 0.5                 (0, 0.5)
+ *   exponent field 1..3:   value = (1 + m/2) * 2^(e-1)     (1 ... 6)
+ */
+double oracle_e2m1_decode(uint8_t code) {
+  int sign = (code >> 3) & 1;
+  int e = (code >> 1) & 3;
+  int m = code & 1;
+  double mag = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+  return sign ? -mag : mag;
+}
+
+/*
+ * Nearest E2M1 value, ties to an even mantissa code; anything at or above 6
+ * (+-inf included) saturates to +-6.  The sign is kept for zero and for
+ * values that round to zero; NaN gives +0 (E2M1 has no NaN).
+ */
+uint8_t oracle_e2m1_encode(float y) {
+  static const double mags[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+  if (isnan(y)) return 0;
+  uint8_t sign = signbit(y) ? 8 : 0;
+  double a = fabs((double)y);
+  if (a >= 6.0) return (uint8_t)(sign | 7);
+  /* spacing of the grid around a: 0.5 on [0, 2), 1 on [2, 4), 2 on [4, 6] */
+  double quantum = a < 2.0 ? 0.5 : (a < 4.0 ? 1.0 : 2.0);
+  /* nearest multiple, ties to the even multiple: on every stretch the even
+   * multiples are exactly the even codes */
+  double v = nearbyint(a / quantum) * quantum;
+  for (int c = 0; c < 8; ++c)
+    if (mags[c] == v) return (uint8_t)(sign | c);
+  return (uint8_t)(sign | 7); /* not reached: v is on the grid */
+}
+
+/*
+ * One row of n values (n a multiple of 16) of a (page, kv head) whose fp32
+ * scale is s, block by block:
+ *   amax   = max |x| over the block's 16 values (NaN ignored)
+ *   sb     = e4m3_rne_satfinite(fp32(amax / fp32(6 * s)))     block scale code
+ *   d      = fp32(decode(sb) * s)                              the block's unit
+ *   code_i = e2m1_encode(d > 0 ? fp32(x_i / d) : 0)
+ * so that value_i = e2m1(code_i) * decode(sb) * s.  Two codes per byte, the
+ * even element in the low nibble; one block-scale byte per 16 values.
+ */
+void oracle_nvfp4_quantize_row(const uint16_t* x_bits, int64_t n, float s, uint8_t* packed,
+                               uint8_t* block_scales) {
+  for (int64_t b = 0; b < n / 16; ++b) {
+    float amax = 0.f;
+    for (int i = 0; i < 16; ++i) {
+      float x = bf16_to_f32(x_bits[b * 16 + i]);
+      if (!isnan(x) && fabsf(x) > amax) amax = fabsf(x);
+    }
+    volatile float six_s = 6.0f * s;
+    volatile float ratio = amax / six_s;
+    uint8_t sb = oracle_e4m3_encode(ratio);
+    volatile float d = (float)oracle_e4m3_decode(sb) * s;
+    block_scales[b] = sb;
+    for (int i = 0; i < 16; i += 2) {
+      uint8_t c[2];
+      for (int k = 0; k < 2; ++k) {
+        volatile float x = bf16_to_f32(x_bits[b * 16 + i + k]);
+        volatile float y = d > 0.f ? x / d : 0.f;
+        c[k] = oracle_e2m1_encode(y);
+      }
+      packed[(b * 16 + i) / 2] = (uint8_t)(c[0] | (c[1] << 4));
+    }
+  }
+}
+
+/* The stored value of element i of a row quantised as above, in fp64 (exact). */
+double oracle_nvfp4_value(const uint8_t* packed, const uint8_t* block_scales, float s,
+                          int64_t i) {
+  uint8_t byte = packed[i / 2];
+  uint8_t code = (i & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF);
+  return oracle_e2m1_decode(code) * oracle_e4m3_decode(block_scales[i / 16]) * (double)s;
+}
+
+void oracle_e2m1_encode_array(const float* y, uint8_t* codes, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) codes[i] = oracle_e2m1_encode(y[i]);
 }
 
 /* Array helpers for exhaustive codec checks. */
