@@ -44,6 +44,7 @@ _LIB = os.path.join(_BUILD, "liboracle.so")
 KV_BF16 = 0
 KV_E4M3 = 1
 KV_INT8 = 2
+KV_NVFP4 = 3
 
 _lib = None
 
@@ -217,7 +218,12 @@ def nvfp4_dequantize(packed, blocks, scale) -> np.ndarray:
 
 # ------------------------------------------------------------------- cache
 class Cache:
-    """A host KV pool image: K and V byte pools ``[pages][Hkv][P][D]`` plus scales."""
+    """A host KV pool image: K and V byte pools ``[pages][Hkv][P][D]`` plus scales.
+
+    FP4 (``"nvfp4"``) pools hold the codes ``[pages][Hkv][P][D/2]`` (two per
+    byte, the even element in the low nibble) followed by the E4M3 block
+    scales ``[pages][Hkv][P][D/16]``.
+    """
 
     def __init__(self, num_pages, page_size, num_kv_heads, head_dim, kv_dtype="bf16",
                  k_pool=None, v_pool=None, k_scale=None, v_scale=None):
@@ -226,9 +232,13 @@ class Cache:
         self.num_kv_heads = int(num_kv_heads)
         self.head_dim = int(head_dim)
         self.kv_dtype = kv_dtype
-        self.code = {"bf16": KV_BF16, "e4m3": KV_E4M3, "int8": KV_INT8}[kv_dtype]
-        eb = 2 if self.code == KV_BF16 else 1
-        nbytes = self.num_pages * self.num_kv_heads * self.page_size * self.head_dim * eb
+        self.code = {"bf16": KV_BF16, "e4m3": KV_E4M3, "int8": KV_INT8,
+                     "nvfp4": KV_NVFP4}[kv_dtype]
+        rows = self.num_pages * self.num_kv_heads * self.page_size
+        if self.code == KV_NVFP4:
+            nbytes = rows * (self.head_dim // 2 + self.head_dim // 16)
+        else:
+            nbytes = rows * self.head_dim * (2 if self.code == KV_BF16 else 1)
         self.k_pool = _c(k_pool, np.uint8) if k_pool is not None else np.zeros(nbytes, np.uint8)
         self.v_pool = _c(v_pool, np.uint8) if v_pool is not None else np.zeros(nbytes, np.uint8)
         assert self.k_pool.size == nbytes and self.v_pool.size == nbytes

@@ -63,6 +63,7 @@
 #define KV_BF16 0
 #define KV_E4M3 1
 #define KV_INT8 2
+#define KV_NVFP4 3
 
 int oracle_num_threads(void) {
 #ifdef _OPENMP
@@ -297,10 +298,30 @@ typedef struct {
 
 static int elem_bytes(int kv_dtype) { return kv_dtype == KV_BF16 ? 2 : 1; }
 
-/* Byte offset of element (page, kv head, slot, d) in a pool. */
+/* Index of the pool row (page, kv head, slot). */
+static int64_t row_index(const cache_t* c, int64_t page, int g, int slot) {
+  return (page * c->num_kv_heads + g) * (int64_t)c->page_size + slot;
+}
+
+/*
+ * FP4 pools hold two regions, rows in the same [page][kv head][slot] order:
+ * the codes (head_dim / 2 bytes a row, two per byte, the even element in the
+ * low nibble), then the E4M3 block scales (head_dim / 16 bytes a row).
+ */
+static int64_t nvfp4_codes_bytes(const cache_t* c) {
+  return (int64_t)c->num_pages * c->num_kv_heads * c->page_size * (c->head_dim / 2);
+}
+
+/* Byte offset of element (page, kv head, slot, d) in a pool: for FP4 pools,
+ * the byte holding its code. */
 static int64_t pool_offset(const cache_t* c, int64_t page, int g, int slot, int d) {
-  int64_t idx = ((page * c->num_kv_heads + g) * (int64_t)c->page_size + slot) * c->head_dim + d;
-  return idx * elem_bytes(c->kv_dtype);
+  if (c->kv_dtype == KV_NVFP4) return row_index(c, page, g, slot) * (c->head_dim / 2) + d / 2;
+  return (row_index(c, page, g, slot) * c->head_dim + d) * elem_bytes(c->kv_dtype);
+}
+
+/* Byte offset of the block scale of element d of row (page, kv head, slot). */
+static int64_t nvfp4_scale_offset(const cache_t* c, int64_t page, int g, int slot, int d) {
+  return nvfp4_codes_bytes(c) + row_index(c, page, g, slot) * (c->head_dim / 16) + d / 16;
 }
 
 /* Physical page holding logical token t of a sequence (page table lookup). */
@@ -322,6 +343,12 @@ static double stored_value(const cache_t* c, const uint8_t* pool, const float* s
     return oracle_e4m3_decode(pool[off]) * (double)scale[page * c->num_kv_heads + g];
   if (c->kv_dtype == KV_INT8)
     return (double)(int8_t)pool[off] * (double)scale[page * c->num_kv_heads + g];
+  if (c->kv_dtype == KV_NVFP4) {
+    uint8_t code = (d & 1) ? (uint8_t)(pool[off] >> 4) : (uint8_t)(pool[off] & 0xF);
+    uint8_t sb = pool[nvfp4_scale_offset(c, page, g, slot, d)];
+    return oracle_e2m1_decode(code) * oracle_e4m3_decode(sb) *
+           (double)scale[page * c->num_kv_heads + g];
+  }
   uint16_t bits;
   memcpy(&bits, pool + off, 2);
   return bf16_value(bits);
@@ -329,8 +356,10 @@ static double stored_value(const cache_t* c, const uint8_t* pool, const float* s
 
 static int check_cache(const cache_t* c) {
   if (!c->k_pool || !c->v_pool) return ORC_ERR_ARG;
-  if (c->kv_dtype != KV_BF16 && c->kv_dtype != KV_E4M3 && c->kv_dtype != KV_INT8)
+  if (c->kv_dtype != KV_BF16 && c->kv_dtype != KV_E4M3 && c->kv_dtype != KV_INT8 &&
+      c->kv_dtype != KV_NVFP4)
     return ORC_ERR_ARG;
+  if (c->kv_dtype == KV_NVFP4 && c->head_dim % 16) return ORC_ERR_ARG;
   if (c->kv_dtype != KV_BF16 && (!c->k_scale || !c->v_scale)) return ORC_ERR_ARG;
   if (c->num_pages < 0 || c->page_size <= 0 || c->num_kv_heads <= 0 || c->head_dim <= 0)
     return ORC_ERR_ARG;
@@ -342,7 +371,7 @@ static int check_cache(const cache_t* c) {
  * Paged KV store.  New token j of sequence b sits at logical position
  * pos = seq_lens_before[b] + j; its page is page_table[b][pos / P] and its
  * slot pos % P.  bf16 stores the input bits; E4M3 and INT8 store the
- * quantised code.
+ * quantised code; FP4 stores the row's codes and block scales.
  * k_new/v_new: bf16 bits [total_new][num_kv_heads][head_dim], ordered by
  * sequence through cu_new [batch+1].
  */
@@ -365,6 +394,17 @@ int oracle_append(uint8_t* k_pool, uint8_t* v_pool, const float* k_scale, const 
       if (st) return st;
       int slot = (int)(pos % page_size);
       for (int g = 0; g < num_kv_heads; ++g) {
+        if (kv_dtype == KV_NVFP4) { /* the whole row: its blocks share scales */
+          int64_t src = (j * num_kv_heads + g) * (int64_t)head_dim;
+          int64_t r = row_index(&c, page, g, slot);
+          float ks = k_scale[page * num_kv_heads + g];
+          float vs = v_scale[page * num_kv_heads + g];
+          oracle_nvfp4_quantize_row(k_new + src, head_dim, ks, k_pool + r * (head_dim / 2),
+                                    k_pool + nvfp4_codes_bytes(&c) + r * (head_dim / 16));
+          oracle_nvfp4_quantize_row(v_new + src, head_dim, vs, v_pool + r * (head_dim / 2),
+                                    v_pool + nvfp4_codes_bytes(&c) + r * (head_dim / 16));
+          continue;
+        }
         for (int d = 0; d < head_dim; ++d) {
           int64_t src = (j * num_kv_heads + g) * (int64_t)head_dim + d;
           int64_t off = pool_offset(&c, page, g, slot, d);

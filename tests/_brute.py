@@ -2,8 +2,9 @@
 
 An independent restatement of the definition used to pin the C oracle: it
 walks the page table token by token with plain Python integers, decodes bf16
-bits with ``struct`` and E4M3 codes through torch's ``float8_e4m3fn`` (a
-library routine), and sums with ``math.fsum``.  It shares nothing with
+bits with ``struct``, E4M3 codes (and FP4 block scales) through torch's
+``float8_e4m3fn`` (a library routine), E2M1 codes through the format's
+value table, and sums with ``math.fsum``.  It shares nothing with
 ``oracle/oracle.c``.
 """
 from __future__ import annotations
@@ -27,10 +28,21 @@ def e4m3_to_float(code: int) -> float:
     return _E4M3[int(code)]
 
 
+# E2M1 magnitudes in code order (sign in bit 3), from the format definition
+_E2M1 = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
 def element(cache, pool, scales, page, g, slot, d) -> float:
     """Value of one stored K or V element, read from the raw byte pool."""
     H, P, D = cache.num_kv_heads, cache.page_size, cache.head_dim
-    idx = ((page * H + g) * P + slot) * D + d
+    row = (page * H + g) * P + slot
+    if cache.kv_dtype == "nvfp4":  # code region, then block-scale region
+        byte = int(pool[row * (D // 2) + d // 2])
+        code = (byte >> 4) if d % 2 else (byte & 0xF)
+        mag = _E2M1[code & 7]
+        sb = int(pool[cache.num_pages * H * P * (D // 2) + row * (D // 16) + d // 16])
+        return (-mag if code & 8 else mag) * e4m3_to_float(sb) * float(scales[page, g])
+    idx = row * D + d
     if cache.kv_dtype == "e4m3":
         return e4m3_to_float(pool[idx]) * float(scales[page, g])
     if cache.kv_dtype == "int8":  # two's-complement byte times the scale

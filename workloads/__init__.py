@@ -49,16 +49,20 @@ E4M3_MAX = 448.0
 # bytes no sequence owns.
 INT8_UNOWNED = 0x80
 INT8_MAX = 127.0
+# FP4 pools (E2M1 codes + E4M3 block scales): the per-(page, kv head) scale
+# divides by 448 * 6 so that block scales stay within E4M3's range; unowned
+# bytes hold 0x7F, whose block scale reads as NaN.
+NVFP4_SCALE_DIV = E4M3_MAX * 6.0
 
 
 def sentinel_byte(kv_dtype: str) -> int:
-    """Fill byte of unowned pool bytes of an 8-bit pool."""
-    return {"e4m3": E4M3_NAN_CODE, "int8": INT8_UNOWNED}[kv_dtype]
+    """Fill byte of unowned pool bytes of a one-byte or FP4 pool."""
+    return {"e4m3": E4M3_NAN_CODE, "int8": INT8_UNOWNED, "nvfp4": E4M3_NAN_CODE}[kv_dtype]
 
 
 def code_max(kv_dtype: str) -> float:
-    """Largest stored magnitude of an 8-bit format (the scale divisor)."""
-    return {"e4m3": E4M3_MAX, "int8": INT8_MAX}[kv_dtype]
+    """Largest stored magnitude of a format relative to its scale (the divisor)."""
+    return {"e4m3": E4M3_MAX, "int8": INT8_MAX, "nvfp4": NVFP4_SCALE_DIV}[kv_dtype]
 
 _STREAM_KV = 1
 _STREAM_QDEC = 2
@@ -90,7 +94,7 @@ class Workload:
     num_q_heads: int
     num_kv_heads: int
     head_dim: int
-    kv_dtype: str  # "bf16", "e4m3" or "int8"
+    kv_dtype: str  # "bf16", "e4m3", "int8" or "nvfp4" (oracle only so far)
     ctx_lens: np.ndarray  # int32 [B], tokens already cached
     new_lens: np.ndarray  # int32 [B], tokens appended this step
     num_pages: int
@@ -127,6 +131,9 @@ class Workload:
         return (self.num_pages, self.num_kv_heads, self.page_size, self.head_dim)
 
     def pool_bytes(self) -> int:
+        if self.kv_dtype == "nvfp4":  # codes (D/2 a row) then block scales (D/16 a row)
+            rows = self.num_pages * self.num_kv_heads * self.page_size
+            return rows * (self.head_dim // 2 + self.head_dim // 16)
         return int(np.prod(self.pool_shape())) * self.elem_bytes
 
     def pages_of(self, b: int) -> np.ndarray:
@@ -172,8 +179,8 @@ class Workload:
 
     # ------------------------------------------------------ FP8 scale policy
     def kv_scales_for(self, b: int, k: torch.Tensor = None, v: torch.Tensor = None):
-        """Per-(page, kv head) scales of sequence ``b``: absmax/448 (E4M3) or
-        absmax/127 (INT8) in fp32.
+        """Per-(page, kv head) scales of sequence ``b``: absmax/448 (E4M3),
+        absmax/127 (INT8) or absmax/(448*6) (FP4) in fp32.
 
         The absmax runs over every element the page will hold after this
         step's append, so no stored value saturates.  Returns
