@@ -229,7 +229,7 @@ int paged_prefill_chunk_attention(const pkv_cache* cache, const void* q, int32_t
                                   void* stream);
 
 /*
- * Decode attention without any device allocation.  The paper has no
+ * Decode attention without any device allocation.  The pages have no
  * counterpart: this entry point exists for callers that cannot call
  * cudaMalloc or take memory from an allocator (code handed only input and
  * output pointers by a host framework or plugin interface, code running where
