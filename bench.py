@@ -540,8 +540,9 @@ def oracle_sample(w, n_seqs: int):
     return np.unique(order[idx])
 
 
-def run_oracle(w, n_seqs: int, repeats: int = 1):
-    """Time the oracle (append of the step's tokens + decode) on a sample."""
+def run_oracle(w, n_seqs: int, repeats: int = 1, one_core: bool = False):
+    """Time the oracle (append of the step's tokens + decode) on a sample, on all
+    host cores; with ``one_core``, also once on a single core."""
     import oracle
 
     sample = oracle_sample(w, n_seqs)
@@ -561,6 +562,21 @@ def run_oracle(w, n_seqs: int, repeats: int = 1):
     dt = statistics.median(times)
     nbytes = decode_bytes(w, rows=sample) + int(w.new_lens[sample].sum()) * w.num_kv_heads * \
         w.head_dim * 2 * (2 + w.elem_bytes)
+    single = None
+    if one_core:
+        # the same sample once more on one core (the append rewrites the same bytes)
+        cores = oracle.num_threads()
+        oracle.set_num_threads(1)
+        try:
+            t = time.perf_counter()
+            c.append(w.page_table[sample], w.ctx_lens[sample], cu, oracle.bf16_bits(k_new),
+                     oracle.bf16_bits(v_new))
+            c.decode(q[qi], w.page_table[sample], w.lens_after[sample], w.softmax_scale)
+            t1 = time.perf_counter() - t
+        finally:
+            oracle.set_num_threads(cores)
+        single = {"value": round(nbytes / t1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                  "seconds": round(t1, 3)}
     return {
         "value": round(nbytes / dt / 1e9, 4),
         "unit": "GB/s",
@@ -571,6 +587,7 @@ def run_oracle(w, n_seqs: int, repeats: int = 1):
                   f"with OpenMP, median of {repeats}",
         "seconds": round(dt, 3),
         "tokens_per_s": round(len(sample) / dt, 3),
+        "single_core": single,
     }
 
 
@@ -620,7 +637,7 @@ def main():
     torch.cuda.set_device(device)
     w, res = run_ours(args, rank, world, device, dist)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = run_oracle(w, args.cpu_sample_seqs, repeats=5)
+        res["cpu_baseline"] = run_oracle(w, args.cpu_sample_seqs, repeats=5, one_core=True)
     if dist:
         dist.barrier()
         dist.destroy_process_group()

@@ -79,6 +79,7 @@ _F = ctypes.c_float
 
 def _declare(L):
     L.oracle_num_threads.restype = _I
+    L.oracle_set_num_threads.argtypes = [_I]
     L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
     L.oracle_e4m3_decode.restype = _D
     L.oracle_e4m3_encode.argtypes = [_F]
@@ -114,6 +115,11 @@ def _declare(L):
 
 def num_threads() -> int:
     return int(lib().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads of the oracle's OpenMP loops from now on."""
+    lib().oracle_set_num_threads(int(n))
 
 
 def _ptr(a: Optional[np.ndarray]):

@@ -73,6 +73,15 @@ int oracle_num_threads(void) {
 #endif
 }
 
+/* Threads of the OpenMP loops from now on (n >= 1). */
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n >= 1) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
 /* ------------------------------------------------------------------ bf16 */
 /* A bf16 value is the upper half of an IEEE binary32; widening is exact. */
 static double bf16_value(uint16_t bits) {
