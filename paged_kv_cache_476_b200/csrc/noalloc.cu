@@ -70,9 +70,17 @@ extern "C" int paged_decode_attention_noalloc(const pkv_cache* cache, const void
   if ((st = check_group(cache, num_q_heads, gqa_group))) return st;
   if (batch < 0 || max_pages_per_seq < 1 || max_seq_len < 0 || num_ctas < 0) return PKV_ERR_SHAPE;
   if (batch == 0) return PKV_OK;
+  // the checks paged_decode_attention makes on its own, first: sizing the
+  // scratch below already queries the device
+  if (!q || !page_table || !seq_lens || !out) return PKV_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(out)) & 15u)
+    return PKV_ERR_ALIGN;
+  if (!(softmax_scale == softmax_scale) || softmax_scale > 3.0e38f || softmax_scale < -3.0e38f)
+    return PKV_ERR_SHAPE;
+  if ((int64_t)max_seq_len > (int64_t)max_pages_per_seq * cache->page_size) return PKV_ERR_SHAPE;
   const size_t need = paged_decode_workspace_bytes(batch, num_q_heads, cache->num_kv_heads,
                                                    cache->head_dim, max_seq_len, num_ctas);
-  if (need == 0) return PKV_ERR_SHAPE;
+  if (need == 0) return PKV_ERR_CUDA;  // the arguments passed above: the device query failed
   if (need > (size_t)PKV_NOALLOC_SCRATCH_BYTES) return PKV_ERR_SCRATCH_LIMIT;
   void* scratch = nullptr;
   if ((st = scratch_address(&scratch))) return st;

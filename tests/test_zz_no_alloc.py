@@ -85,8 +85,11 @@ def test_noalloc_rejects_requests_beyond_the_scratch():
     # 4096 sequences x 8 kv heads x 8 q heads of partials exceed 16 MiB
     need = pkv.paged_decode_workspace_bytes(4096, 64, 8, 128, 8192)
     assert need > pkv.NOALLOC_SCRATCH_BYTES
+    # well-formed but fake (never dereferenced) pointers: the size check comes
+    # after the argument checks and before anything is read or enqueued
+    fake = 0x10000
     code = pkv.lib().paged_decode_attention_noalloc(
-        ctypes.byref(st.cache.c_struct), None, 64, 8, None, 128, None, 4096, 8192, 0.1, None,
+        ctypes.byref(st.cache.c_struct), fake, 64, 8, fake, 128, fake, 4096, 8192, 0.1, fake,
         None, 0, None)
     assert code == -11
     assert "16 MiB" in pkv.pkv_status_string(code)
