@@ -11,6 +11,7 @@ What the format fixes, checked against things other than the oracle itself:
   allow; all-zero blocks, NaN elements and the nibble order.
 """
 import math
+import os
 
 import numpy as np
 import pytest
@@ -130,3 +131,28 @@ def test_zero_block_nan_and_nibble_order():
     assert packed[0, 9] & 0xF == 8 | 5      # element 18: -1.5 / 0.5 = -3
     vals = oracle.nvfp4_dequantize(packed, blocks, np.float32(1.0))
     assert vals[0, 16] == 3.0 and vals[0, 17] == 0.0 and vals[0, 18] == -1.5
+
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "nvfp4_points.txt")
+
+
+def test_golden_points():
+    elems, blocks = [], []
+    for line in open(GOLDEN):
+        line = line.split("#")[0].strip()
+        if not line:
+            continue
+        f = line.split()
+        if f[0] == "block":
+            blocks.append(f[1:])
+        else:
+            elems.append((np.float32(float(f[0])), int(f[1], 16)))
+    assert len(elems) >= 15 and blocks
+    got = oracle.e2m1_encode(np.array([v for v, _ in elems], np.float32))
+    assert got.tolist() == [c for _, c in elems]
+    for b in blocks:
+        s = np.float32(float(b[0]))
+        x = np.array([float(v) for v in b[1:17]], np.float32)
+        packed, scales = oracle.nvfp4_quantize(_bf16_bits(x)[None], s)
+        assert scales[0, 0] == int(b[17], 16)
+        assert packed[0].tolist() == [int(v, 16) for v in b[18:26]]
