@@ -44,6 +44,13 @@ int check_cache(const pkv_cache* c) {
   return PKV_OK;
 }
 
+// Tokens a page-table row can address, max_pages_per_seq * page_size, must
+// fit in int32: the kernels compare lengths against it in 32-bit arithmetic.
+int check_table_span(const pkv_cache* c, int32_t max_pages_per_seq) {
+  if ((int64_t)max_pages_per_seq * c->page_size > INT32_MAX) return PKV_ERR_SHAPE;
+  return PKV_OK;
+}
+
 int check_group(const pkv_cache* c, int32_t num_q_heads, int32_t gqa_group) {
   if (gqa_group != 1 && gqa_group != 2 && gqa_group != 4 && gqa_group != 8) return PKV_ERR_GQA;
   if (num_q_heads != gqa_group * c->num_kv_heads) return PKV_ERR_GQA;
@@ -90,10 +97,19 @@ int encode_pool_map(CUtensorMap* map, void* base, bool fp8, int64_t rows, int ro
 }
 
 static int decode_ctas_per_sm(int head_dim, int fmt, int group, int* out) {
-  // cached per variant: the occupancy of a kernel does not change at run time
-  static int cache[2][3][4] = {};
+  // Cached per device and variant: a kernel's occupancy does not change at
+  // run time, but the shared-memory attribute that decode_occupancy sets
+  // belongs to the device that is current, so every device fills its own
+  // entry (and sets its own attribute) on first use.
+  constexpr int kMaxDevices = 64;
+  static int cache[kMaxDevices][2][kNumKvFormats][4] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices || fmt < 0 || fmt >= kNumKvFormats) return PKV_ERR_UNSUPPORTED;
   const int gi = group == 1 ? 0 : group == 2 ? 1 : group == 4 ? 2 : 3;
-  int& slot = cache[head_dim == 128][fmt][gi];
+  std::lock_guard<std::mutex> lock(mu);
+  int& slot = cache[dev][head_dim == 128][fmt][gi];
   if (slot == 0) {
     int n = 0;
     if (decode_occupancy(head_dim, fmt, group, &n) != cudaSuccess || n < 1) return PKV_ERR_CUDA;
@@ -141,6 +157,7 @@ int paged_kv_append(const pkv_cache* cache, const int32_t* page_table, int32_t m
   int st = check_cache(cache);
   if (st) return st;
   if (batch < 0 || total_new_tokens < 0 || max_pages_per_seq < 1) return PKV_ERR_SHAPE;
+  if ((st = check_table_span(cache, max_pages_per_seq))) return st;
   if (total_new_tokens == 0 || batch == 0) return PKV_OK;
   if (!page_table || !seq_lens_before || !cu_new_tokens || !k_new || !v_new) return PKV_ERR_NULL;
   if (!aligned16(k_new) || !aligned16(v_new)) return PKV_ERR_ALIGN;
@@ -222,7 +239,8 @@ static int decode_entry(const pkv_cache* cache, const void* q, int32_t num_q_hea
   if (batch == 0) return PKV_OK;
   if (!q || !page_table || !seq_lens || !out) return PKV_ERR_NULL;
   if (!aligned16(q) || !aligned16(out)) return PKV_ERR_ALIGN;
-  if (max_seq_len > max_pages_per_seq * cache->page_size) return PKV_ERR_SHAPE;
+  if ((st = check_table_span(cache, max_pages_per_seq))) return st;
+  if ((int64_t)max_seq_len > (int64_t)max_pages_per_seq * cache->page_size) return PKV_ERR_SHAPE;
   const size_t need = paged_decode_workspace_bytes(batch, num_q_heads, cache->num_kv_heads,
                                                    cache->head_dim, max_seq_len, num_ctas);
   if (need == 0) return PKV_ERR_CUDA;

@@ -23,10 +23,11 @@
 //    which converts exactly), with the online softmax in registers; a flush
 //    warp turns the consumers' per-warp snapshots at each segment end into
 //    the output or a split partial while the consumers stream on.
-//  * E4M3 K/V: K codes are converted to f16 in registers after ldmatrix (the
-//    d order inside each 16-wide block is permuted identically in Q); V codes
-//    are converted into a per-warp f16 tile for the transposed ldmatrix.  The
-//    per-(page, head) scales fold into the scores (K) and into P (V).
+//  * One-byte K/V (E4M3, INT8): K codes are converted to f16 in registers
+//    after ldmatrix (the d order inside each 16-wide block is permuted
+//    identically in Q); V codes go from a transposed ldmatrix of byte pairs
+//    straight into the f16 A fragments of V^T.  The per-(page, head) scales
+//    fold into the scores (K) and into P (V).
 //  * Every wait is bounded; a bad page id or length is skipped and flagged.
 #include "common.cuh"
 #include "kernels.h"

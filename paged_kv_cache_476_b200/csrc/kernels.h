@@ -10,6 +10,9 @@
 
 namespace pkv {
 
+// Number of pkv_kv_dtype values.
+constexpr int kNumKvFormats = 3;
+
 // KV formats of the pools (pkv_kv_dtype): is the stored code one byte?
 __host__ __device__ constexpr bool k8(int fmt) { return fmt != PKV_KV_BF16; }
 
@@ -72,6 +75,7 @@ cudaError_t launch_combine(const void* parts, const float* lse_parts, int num_pa
 
 int check_cache(const pkv_cache* c);
 int check_group(const pkv_cache* c, int32_t num_q_heads, int32_t gqa_group);
+int check_table_span(const pkv_cache* c, int32_t max_pages_per_seq);
 int encode_pool_map(CUtensorMap* map, void* base, bool fp8, int64_t rows, int row_elems,
                     int box_cols, int box_rows);
 int prefill_entry(const pkv_cache* cache, const void* q, int32_t num_q_heads, int32_t gqa_group,

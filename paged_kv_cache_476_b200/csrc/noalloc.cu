@@ -21,6 +21,17 @@
 //  * The first call on a device looks up the array's device address (host
 //    code cannot use the array's name as a device pointer).  Make that first
 //    call before capturing any stream into a CUDA graph.
+//  * Under CUDA's default lazy module loading, the array's device memory is
+//    committed by that first call on each device, not when the library
+//    loads.  So the first call is the one that can fail for lack of device
+//    memory (it returns PKV_ERR_CUDA).  A caller whose device memory is later
+//    handed over to a foreign allocator should make one call first, while
+//    memory is still free, or run with CUDA_MODULE_LOADING=EAGER, which
+//    commits the array when the CUDA context is created.  Later calls
+//    allocate nothing.
+//  * The looked-up address is cached per device for the life of the process.
+//    It does not survive a reset of the device's primary context
+//    (cudaDeviceReset): do not use this entry point after one.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -69,6 +80,7 @@ extern "C" int paged_decode_attention_noalloc(const pkv_cache* cache, const void
   if (st) return st;
   if ((st = check_group(cache, num_q_heads, gqa_group))) return st;
   if (batch < 0 || max_pages_per_seq < 1 || max_seq_len < 0 || num_ctas < 0) return PKV_ERR_SHAPE;
+  if ((st = check_table_span(cache, max_pages_per_seq))) return st;
   if (batch == 0) return PKV_OK;
   // the checks paged_decode_attention makes on its own, first: sizing the
   // scratch below already queries the device

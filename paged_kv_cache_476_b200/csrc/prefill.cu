@@ -38,6 +38,8 @@
 //    64-key block; the V scales ride on P, kept in f16 (11-bit mantissa) so
 //    that PV is an f16 x f16 product.
 //  * Every wait is bounded; TMEM is freed on every exit path.
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -929,12 +931,23 @@ template <int D, int kFmt>
 cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const Params& p, cudaStream_t stream) {
   const size_t smem = smem_bytes<D, kFmt>();
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, kFmt>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr = true;
+  // The shared-memory attribute belongs to the current device: set it once
+  // per device and instantiation.
+  constexpr int kMaxDevices = 64;
+  static bool attr[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!attr[dev]) {
+      e = cudaFuncSetAttribute(prefill_kernel<D, kFmt>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      attr[dev] = true;
+    }
   }
   const unsigned blocks = (unsigned)p.pair_slots * (unsigned)p.num_kv_heads * (unsigned)p.num_chunks;
   prefill_kernel<D, kFmt><<<blocks, Smem<D, kFmt>::kThreads, smem, stream>>>(tq, tk, tv, p);
@@ -956,6 +969,7 @@ int prefill_entry(const pkv_cache* cache, const void* q, int32_t num_q_heads, in
   if ((st = check_group(cache, num_q_heads, gqa_group))) return st;
   if (num_chunks < 0 || total_q < 0 || max_q_len < 0 || max_pages_per_seq < 1)
     return PKV_ERR_SHAPE;
+  if ((st = check_table_span(cache, max_pages_per_seq))) return st;
   if (!(softmax_scale == softmax_scale) || softmax_scale > 3.0e38f || softmax_scale < -3.0e38f)
     return PKV_ERR_SHAPE;
   if (num_chunks == 0 || total_q == 0 || max_q_len == 0) return PKV_OK;
