@@ -249,6 +249,13 @@ int paged_prefill_chunk_attention(const pkv_cache* cache, const void* q, int32_t
  *    race and give wrong results.  Order them on one stream.
  *  - The first call on a device looks up the array's device address with that
  *    device current; make that first call before any stream capture.
+ *  - Under CUDA's default lazy module loading the array's memory is committed
+ *    by that first call on each device, so the first call is the one that
+ *    can fail for lack of device memory (PKV_ERR_CUDA).  Make one call while
+ *    memory is still free, or set CUDA_MODULE_LOADING=EAGER, before handing
+ *    the device's memory to another allocator.
+ *  - The address is cached per device for the life of the process and does
+ *    not survive cudaDeviceReset: do not call this entry point after a reset.
  */
 #define PKV_NOALLOC_SCRATCH_BYTES (16u << 20)
 int paged_decode_attention_noalloc(const pkv_cache* cache, const void* q, int32_t num_q_heads,
@@ -276,6 +283,24 @@ int paged_decode_attention_noalloc(const pkv_cache* cache, const void* q, int32_
 int paged_attention_combine(const void* parts, const float* lse_parts, int32_t num_parts,
                             int32_t rows, int32_t head_dim, void* out, float* lse,
                             void* stream);
+
+/*
+ * Check of the bounded waits (failure detection without a fault).  Every wait
+ * inside this library's kernels (a TMA tile landing, a ring slot freed, a
+ * tensor-core product done) gives up after a time limit, ORs
+ * PKV_FLAG_TIMEOUT into cache->error_flags and lets the kernel return, so a
+ * lost arrival ends in a status the host reads and the context stays usable.
+ * This call enqueues one CTA that runs that same wait on an mbarrier nothing
+ * arrives on, with no copy or tensor-core operation in flight.  Source: the
+ * murmur post's evaluation criteria, which list fault recovery (故障恢復).
+ *   error_flags  device int32; PKV_FLAG_TIMEOUT is OR-ed in when the wait gives up
+ *   limit_ns     how long to wait: 0 = the limit the kernels use (2 s);
+ *                at most that limit, else PKV_ERR_SHAPE
+ *   waited_ns    optional device int64: the time waited (-1 if it was not cut off)
+ * Returns PKV_ERR_NULL without error_flags, PKV_ERR_CUDA if the launch fails.
+ */
+int pkv_check_bounded_wait(int32_t* error_flags, int64_t limit_ns, int64_t* waited_ns,
+                           void* stream);
 
 /* Human-readable name of a pkv_status value (static storage). */
 const char* pkv_status_string(int status);

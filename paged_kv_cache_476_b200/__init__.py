@@ -48,6 +48,7 @@ EXPORTED = (
     "paged_decode_attention_noalloc",
     "paged_attention_combine",
     "paged_decode_attention_append",
+    "pkv_check_bounded_wait",
     # include/paged_kv_runtime.h: host page allocator and step planner
     "pkv_allocator_create",
     "pkv_allocator_destroy",
@@ -128,6 +129,8 @@ def _load() -> ctypes.CDLL:
     lib.paged_decode_attention_noalloc.restype = ctypes.c_int
     lib.paged_attention_combine.argtypes = [P, P, I32, I32, I32, P, P, P]
     lib.paged_attention_combine.restype = ctypes.c_int
+    lib.pkv_check_bounded_wait.argtypes = [P, ctypes.c_int64, P, P]
+    lib.pkv_check_bounded_wait.restype = ctypes.c_int
     lib.pkv_status_string.argtypes = [ctypes.c_int]
     lib.pkv_status_string.restype = ctypes.c_char_p
     lib.pkv_abi_version.restype = ctypes.c_int
@@ -417,6 +420,21 @@ def paged_attention_combine(parts, lse_parts, out=None, lse=None, stream=None):
            _lib.paged_attention_combine(_ptr(parts), _ptr(lse_parts), R, B * Hq, D, _ptr(out),
                                         _ptr(lse), _stream(stream)))
     return out, lse
+
+
+def pkv_check_bounded_wait(error_flags, limit_ns: int = 0, waited_ns=None, stream=None) -> None:
+    """Run the kernels' bounded mbarrier wait on a barrier nothing arrives on.
+
+    ``error_flags`` int32 device scalar receives ``PKV_FLAG_TIMEOUT`` when the
+    wait gives up after ``limit_ns`` (0: the kernels' own limit);
+    ``waited_ns`` (optional int64 device scalar) receives the time waited.
+    """
+    _dev("error_flags", error_flags, torch.int32)
+    if waited_ns is not None:
+        _dev("waited_ns", waited_ns, torch.int64)
+    _check("pkv_check_bounded_wait",
+           _lib.pkv_check_bounded_wait(_ptr(error_flags), int(limit_ns), _ptr(waited_ns),
+                                       _stream(stream)))
 
 
 # ----------------------------------------------------- host runtime (paged_kv_runtime.h)

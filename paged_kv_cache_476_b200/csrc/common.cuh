@@ -88,16 +88,19 @@ __device__ __forceinline__ uint64_t global_ns() {
 // Bounded wait for the phase with the given parity to complete.  With
 // suspend_ns > 0 a waiting thread may sleep up to that long per try (it is
 // woken when the phase completes), so an idle warp costs no issue slots.
-// Returns false (and raises PKV_FLAG_TIMEOUT) after kWaitLimitNs.
+// Returns false (and raises PKV_FLAG_TIMEOUT) after limit_ns.  Every wait of
+// every kernel in this library goes through here with the default limit;
+// pkv_check_bounded_wait runs the same code with a short one.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* flags,
-                                          uint32_t suspend_ns = 0) {
+                                          uint32_t suspend_ns = 0,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   while (true) {
     const bool ok =
         suspend_ns ? mbar_try_wait_sleep(bar, parity, suspend_ns) : mbar_try_wait(bar, parity);
     if (ok) return true;
-    if (global_ns() - t0 > kWaitLimitNs) break;
+    if (global_ns() - t0 > limit_ns) break;
   }
   flag_error(flags, PKV_FLAG_TIMEOUT);
   return false;

@@ -149,3 +149,22 @@ def test_append_rejects_null_inputs(pkv):
         args[i] = None
         st = L.paged_kv_append(ctypes.byref(c), *args, None)
         assert st == NULL, (i, st)
+
+
+def test_bounded_wait_check_rejects_bad_arguments(pkv):
+    L = pkv.lib()
+    assert L.pkv_check_bounded_wait(None, 1000, None, None) == NULL
+    assert L.pkv_check_bounded_wait(A, -1, None, None) == SHAPE
+    assert L.pkv_check_bounded_wait(A, 2_000_000_001, None, None) == SHAPE
+
+
+def test_page_table_span_must_fit_int32(pkv):
+    # max_pages_per_seq * page_size above INT32_MAX: rejected, no int32 overflow
+    L = pkv.lib()
+    c = _cache(pkv)
+    big = (1 << 31) // 64  # * 64 = 2^31
+    assert _decode(pkv, c=c, maxp=big) == SHAPE
+    assert _decode(pkv, fn="paged_decode_attention_noalloc", c=c, maxp=big) == SHAPE
+    assert L.paged_kv_append(ctypes.byref(c), A, big, A, A, 2, 5, A, A, None) == SHAPE
+    assert L.paged_prefill_chunk_attention(ctypes.byref(c), A, 32, 4, A, A, big, A, 2, 10, 5,
+                                           0.1, A, None, None) == SHAPE
