@@ -125,13 +125,30 @@ def bf16_half_ulp(x):
     return np.where(x == 0, 0.0, np.ldexp(1.0, e - 9))
 
 
+def bf16_round(x):
+    """fp64 values rounded to the nearest bf16 (8 significant bits), ties to
+    even: the correctly rounded bf16 answer of an exact value."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)  # x = m * 2^e, |m| in [0.5, 1)
+    return np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)
+
+
+# Elements that met the bound only through its second form, per compare() call
+# (a record for the test log).
+ROUNDED_ONLY = []
+
+
 def compare(out, lse, ref_out, ref_lse, rows=None, max_abs=1e-2, mean_abs=1e-3, lse_abs=2e-3):
     """bf16 output vs fp64 oracle; fp32 lse bound.
 
-    Per element |out - ref| <= max_abs + half a bf16 ulp of ref: the bound
-    holds for the computation (P rounding, fp32 sums) and the output's own
-    rounding to bf16 comes on top (at |ref| >= 4 half an ulp alone is 2^-6 >
-    1e-2).  The mean of |out - ref| must stay <= mean_abs.
+    Every element must satisfy |out - exact| <= max_abs.  An element that does
+    not must instead be within max_abs of the correctly rounded bf16 value of
+    the exact result, bf16_round(exact): a bf16 output cannot be closer to
+    the exact value than that.  This second form can only admit an element
+    whose half bf16 ulp exceeds max_abs, i.e. |exact| >= 4 (there the bf16
+    spacing is 2^-5, so it requires out == bf16_round(exact)); the test
+    asserts that, and records how many elements needed it.  The mean of
+    |out - exact| must stay <= mean_abs.
     """
     o = out.float().cpu().numpy().astype(np.float64)
     r = ref_out
@@ -139,10 +156,21 @@ def compare(out, lse, ref_out, ref_lse, rows=None, max_abs=1e-2, mean_abs=1e-3, 
         o, r = o[rows], r[rows]
     assert np.all(np.isfinite(o)), "non-finite output"
     err = np.abs(o - r)
-    excess = err - (max_abs + bf16_half_ulp(r))
+    plain = err <= max_abs
+    err_rounded = np.abs(o - bf16_round(r))
+    rounded_only = ~plain & (err_rounded <= max_abs)
+    bad = ~plain & ~rounded_only
     info = (f"max_abs={err.max():.3e} mean_abs={err.mean():.3e} "
-            f"worst excess over bound={excess.max():.3e}")
-    assert excess.max() <= 0, info
+            f"elements over {max_abs} of both the exact and the rounded value: {int(bad.sum())}"
+            + (f" (worst at exact={r[bad][np.argmax(err[bad])]:.6f}, "
+               f"out={o[bad][np.argmax(err[bad])]:.6f})" if bad.any() else ""))
+    assert not bad.any(), info
+    n_rounded = int(rounded_only.sum())
+    if n_rounded:
+        assert np.all(np.abs(r[rounded_only]) >= 4.0), "second form admitted |exact| < 4"
+        print(f"compare: {n_rounded} of {err.size} elements within {max_abs} of the correctly "
+              f"rounded bf16 value only (|exact| >= 4)")
+    ROUNDED_ONLY.append(n_rounded)
     assert err.mean() <= mean_abs, info
     if lse is not None and ref_lse is not None:
         l = lse.cpu().numpy().astype(np.float64)

@@ -208,19 +208,16 @@ def test_config_llama8b_decode_full():
     assert int(st.flags.item()) == 0
 
 
-def test_config_long_context_decode_sampled():
+def test_config_long_context_decode_full():
+    # all 8 sequences (32k-131k tokens each) against the oracle
     w = workloads.long_context_decode()
     st = GpuState(w)
     st.append_step()
     out, lse = st.decode()
     torch.cuda.synchronize()
-    la = w.lens_after
-    sample = sorted({int(np.argmax(la)), int(np.argmin(la)), 3})
-    ref, ref_lse = _oracle_decode(w, seq_ids=sample)
-    compare(out, lse, ref, ref_lse, rows=sample)
-    o = out.float().cpu()
-    assert torch.all(torch.isfinite(o)) and o.abs().max() < 6
     assert int(st.flags.item()) == 0
+    ref, ref_lse = _oracle_decode(w)
+    compare(out, lse, ref, ref_lse)
 
 
 def test_config_70b_fp8_decode_full():
@@ -262,8 +259,8 @@ def test_config_mixed_decode_part():
 
 
 def test_workspace_reused_across_batch_shapes():
-    # one workspace, zeroed once, serves calls with other shapes after it:
-    # the granule counter sits at a fixed offset and every call leaves it zero
+    # one workspace serves calls with other shapes after it: each call writes
+    # every workspace value it reads, so the previous call's contents are harmless
     import paged_kv_cache_476_b200 as pkv
 
     big = workloads.build("wsA", 15, [3000, 9000, 40, 2500] * 8, [1] * 32, page_size=64,
