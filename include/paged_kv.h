@@ -21,17 +21,34 @@
  *  - Pools: separate K and V pools, each [num_pages][num_kv_heads][page_size]
  *    [head_dim], row-major, element type bf16 or FP8 E4M3 (1 byte).  Base
  *    addresses must be 16-byte aligned.
- *  - FP8 scales: one fp32 per (page, kv head) for K and one for V, layout
- *    [num_pages][num_kv_heads]; the stored value of an element is
- *    decode_e4m3(code) * scale.  Scales must be finite and in (0, 2^15].
+ *  - Scales of the one-byte and FP4 pools: one fp32 per (page, kv head) for
+ *    K and one for V, layout [num_pages][num_kv_heads]; the stored value of
+ *    an E4M3 element is decode_e4m3(code) * scale.  Scales must be finite
+ *    and in (0, 2^15].
  *    The caller chooses them (e.g. absmax/448 of what the page will hold);
  *    the library reads them and never updates them.
+ *  - INT8 pools: code = nearest integer (ties to even) of fp32(x) / scale,
+ *    clamped to +-127 (NaN stored as 0); stored value = code * scale.
+ *  - FP4 pools (PKV_KV_NVFP4; solosoft post, FAQ: FP4 quantisation on
+ *    Blackwell).  Each pool is ONE buffer of rows * (head_dim/2 + head_dim/16)
+ *    bytes, rows = num_pages * num_kv_heads * page_size, row index
+ *    (page * num_kv_heads + kv_head) * page_size + slot:
+ *      codes   [rows][head_dim/2]   two E2M1 codes per byte, the even element
+ *                                    in the low nibble;
+ *      blocks  [rows][head_dim/16]  one E4M3 block scale per 16 consecutive
+ *                                    elements of a row, after all the codes.
+ *    With s the (page, kv head) fp32 scale and amax the largest |x| of a
+ *    block: sb = e4m3_rne_satfinite(amax / fp32(6 * s)), d = fp32(decode(sb) * s),
+ *    code = e2m1_rne_satfinite(x / d) (0 when d = 0, +0 for NaN); stored
+ *    value = e2m1(code) * decode(sb) * s.  The caller picks s (e.g.
+ *    absmax / (448 * 6) of what the page will hold).
  *  - Page table: int32 [batch][max_pages_per_seq], row-major; entry j holds the
  *    physical page of tokens [j*page_size, (j+1)*page_size).  Entries past the
  *    last page a sequence needs are ignored (-1 by convention).
  *  - GQA: q head h reads kv head h / gqa_group (contiguous groups).
  *  - Supported: page_size in {64, 128}; head_dim in {64, 128};
- *    gqa_group in {1, 2, 4, 8}; bf16 Q/K/V/out; K/V pools bf16 or E4M3.
+ *    gqa_group in {1, 2, 4, 8}; bf16 Q/K/V/out; K/V pools bf16, E4M3, INT8
+ *    or FP4.
  *  - Asynchronous: a call validates its arguments on the host, returns a
  *    negative pkv_status before launching anything if they are wrong, and
  *    otherwise enqueues its kernels on `stream` (a cudaStream_t; NULL = the
@@ -60,7 +77,7 @@ typedef enum {
   PKV_ERR_PAGE_SIZE = -3,   /* page_size not in {64, 128} */
   PKV_ERR_HEAD_DIM = -4,    /* head_dim not in {64, 128} */
   PKV_ERR_GQA = -5,         /* num_q_heads != gqa_group*num_kv_heads, or group unsupported */
-  PKV_ERR_DTYPE = -6,       /* unknown kv_dtype, or E4M3 without scales */
+  PKV_ERR_DTYPE = -6,       /* unknown kv_dtype, or a quantised pool without scales */
   PKV_ERR_WORKSPACE = -7,   /* decode workspace NULL, misaligned or too small */
   PKV_ERR_CUDA = -8,        /* a CUDA runtime call or kernel launch failed */
   PKV_ERR_ALIGN = -9,       /* a pointer that must be 16-byte aligned is not */
@@ -69,7 +86,13 @@ typedef enum {
   PKV_ERR_NO_PAGES = -12     /* the free pages cannot cover a growth (paged_kv_runtime.h) */
 } pkv_status;
 
-typedef enum { PKV_KV_BF16 = 0, PKV_KV_FP8_E4M3 = 1, PKV_KV_INT8 = 2 } pkv_kv_dtype;
+typedef enum {
+  PKV_KV_BF16 = 0,     /* bf16 elements */
+  PKV_KV_FP8_E4M3 = 1, /* one E4M3 code per element, per-(page, kv head) fp32 scale */
+  PKV_KV_INT8 = 2,     /* one INT8 code per element (+-127), per-(page, kv head) scale */
+  PKV_KV_NVFP4 = 3     /* E2M1 codes, an E4M3 scale per 16 elements, per-(page, kv head)
+                          scale: see "FP4 pools" above */
+} pkv_kv_dtype;
 
 /* Device-side error bits OR-ed into pkv_cache.error_flags. */
 #define PKV_FLAG_BAD_PAGE 0x1    /* a page-table entry outside [0, num_pages) */
@@ -80,10 +103,11 @@ typedef enum { PKV_KV_BF16 = 0, PKV_KV_FP8_E4M3 = 1, PKV_KV_INT8 = 2 } pkv_kv_dt
 
 /* The paged KV cache: pools, optional FP8 scales, geometry. */
 typedef struct pkv_cache {
-  void* k_pool;          /* [num_pages][num_kv_heads][page_size][head_dim] */
+  void* k_pool;          /* [num_pages][num_kv_heads][page_size][head_dim] (FP4: codes,
+                            then block scales, as above) */
   void* v_pool;          /* same shape as k_pool */
-  const float* k_scale;  /* [num_pages][num_kv_heads] fp32, E4M3 only (else NULL) */
-  const float* v_scale;  /* [num_pages][num_kv_heads] fp32, E4M3 only (else NULL) */
+  const float* k_scale;  /* [num_pages][num_kv_heads] fp32; NULL for bf16 pools */
+  const float* v_scale;  /* [num_pages][num_kv_heads] fp32; NULL for bf16 pools */
   int32_t num_pages;     /* >= 1 */
   int32_t page_size;     /* tokens per page: 64 or 128 */
   int32_t num_kv_heads;  /* >= 1 */
@@ -99,7 +123,8 @@ typedef struct pkv_cache {
  * page_table[b][pos / page_size], slot pos % page_size.  bf16 pools receive
  * the input bits unchanged; E4M3 pools receive
  * e4m3_round_nearest_even_satfinite(fp32(x) / scale[page][kv_head]) with an
- * IEEE fp32 division.  Source: concept page "PagedAttention 及 KV 快取管理"
+ * IEEE fp32 division; INT8 and FP4 pools the codes defined above (FP4: a
+ * token's row is quantised block by block, its block scales included).  Source: concept page "PagedAttention 及 KV 快取管理"
  * and "執行時執行模型" (attention updates the KV pages).
  *   page_table        int32 [batch][max_pages_per_seq]
  *   seq_lens_before   int32 [batch], tokens already cached

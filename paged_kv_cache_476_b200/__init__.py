@@ -7,7 +7,7 @@ CUDA kernels; there is no CPU or PyTorch fallback.  If the library is missing
 or cannot load, importing this package raises.
 
 Entry points (same names as the C ABI):
-    paged_kv_append                 paged store of new tokens' K/V (bf16 or E4M3)
+    paged_kv_append                 paged store of new tokens' K/V (bf16, E4M3, INT8, FP4)
     paged_decode_attention          split-KV decode, persistent and balanced
     paged_prefill_chunk_attention   causal prefill chunks on tcgen05
     paged_decode_workspace_bytes, paged_decode_plan, pkv_status_string
@@ -29,7 +29,9 @@ LIB_PATH = os.path.join(_PKG, "libpagedkv.so")
 PKV_KV_BF16 = 0
 PKV_KV_FP8_E4M3 = 1
 PKV_KV_INT8 = 2
-_KV_CODES = {"bf16": PKV_KV_BF16, "e4m3": PKV_KV_FP8_E4M3, "int8": PKV_KV_INT8}
+PKV_KV_NVFP4 = 3
+_KV_CODES = {"bf16": PKV_KV_BF16, "e4m3": PKV_KV_FP8_E4M3, "int8": PKV_KV_INT8,
+             "nvfp4": PKV_KV_NVFP4}
 PKV_FLAG_BAD_PAGE = 0x1
 PKV_FLAG_BAD_LENGTH = 0x2
 PKV_FLAG_TIMEOUT = 0x4
@@ -198,29 +200,49 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
 
 
+def nvfp4_pool_bytes(num_pages: int, num_kv_heads: int, page_size: int, head_dim: int) -> int:
+    """Bytes of one FP4 pool: every row's E2M1 codes (head_dim/2 bytes), then
+    every row's E4M3 block scales (head_dim/16 bytes)."""
+    rows = num_pages * num_kv_heads * page_size
+    return rows * (head_dim // 2 + head_dim // 16)
+
+
 class PagedKVCache:
     """Caller-owned paged KV pool: K and V ``[num_pages, Hkv, page_size, head_dim]``.
 
     ``kv_dtype`` is ``"bf16"`` (torch.bfloat16 pools), ``"e4m3"`` (uint8 or
-    float8_e4m3fn pools) or ``"int8"`` (int8 or uint8 pools); the one-byte
-    formats take fp32 ``k_scale``/``v_scale`` ``[num_pages, Hkv]``.
+    float8_e4m3fn pools), ``"int8"`` (int8 or uint8 pools) or ``"nvfp4"``
+    (FP4: flat uint8 pools of ``nvfp4_pool_bytes(...)`` bytes, codes then
+    block scales, with ``geometry=(num_pages, Hkv, page_size, head_dim)``).
+    The quantised formats take fp32 ``k_scale``/``v_scale`` ``[num_pages, Hkv]``.
     ``error_flags`` is an optional int32 device scalar that kernels OR
     ``PKV_FLAG_*`` bits into.
     """
 
     def __init__(self, k_pool, v_pool, kv_dtype="bf16", k_scale=None, v_scale=None,
-                 error_flags=None):
+                 error_flags=None, geometry=None):
         if kv_dtype not in _KV_CODES:
-            raise ValueError("kv_dtype must be 'bf16', 'e4m3' or 'int8'")
-        dt = {"bf16": torch.bfloat16, "e4m3": (torch.uint8, torch.float8_e4m3fn),
-              "int8": (torch.int8, torch.uint8)}[kv_dtype]
-        _dev("k_pool", k_pool, dt, 4)
-        _dev("v_pool", v_pool, dt, 4)
-        if k_pool.shape != v_pool.shape:
-            raise ValueError("k_pool and v_pool shapes differ")
+            raise ValueError("kv_dtype must be 'bf16', 'e4m3', 'int8' or 'nvfp4'")
+        if kv_dtype == "nvfp4":
+            if geometry is None or len(geometry) != 4:
+                raise ValueError("FP4 pools need geometry=(num_pages, Hkv, page_size, head_dim)")
+            _dev("k_pool", k_pool, torch.uint8, 1)
+            _dev("v_pool", v_pool, torch.uint8, 1)
+            need = nvfp4_pool_bytes(*geometry)
+            if k_pool.numel() != need or v_pool.numel() != need:
+                raise ValueError(f"FP4 pools of this geometry hold {need} bytes")
+            shape = tuple(int(x) for x in geometry)
+        else:
+            dt = {"bf16": torch.bfloat16, "e4m3": (torch.uint8, torch.float8_e4m3fn),
+                  "int8": (torch.int8, torch.uint8)}[kv_dtype]
+            _dev("k_pool", k_pool, dt, 4)
+            _dev("v_pool", v_pool, dt, 4)
+            if k_pool.shape != v_pool.shape:
+                raise ValueError("k_pool and v_pool shapes differ")
+            shape = tuple(k_pool.shape)
         if kv_dtype != "bf16":
             if k_scale is None or v_scale is None:
-                raise ValueError("one-byte pools need k_scale and v_scale")
+                raise ValueError("quantised pools need k_scale and v_scale")
             _dev("k_scale", k_scale, torch.float32, 2)
             _dev("v_scale", v_scale, torch.float32, 2)
         if error_flags is not None:
@@ -229,7 +251,7 @@ class PagedKVCache:
         self.k_scale, self.v_scale = k_scale, v_scale
         self.error_flags = error_flags
         self.kv_dtype = kv_dtype
-        self.num_pages, self.num_kv_heads, self.page_size, self.head_dim = k_pool.shape
+        self.num_pages, self.num_kv_heads, self.page_size, self.head_dim = shape
         self._c = PkvCache(k_pool.data_ptr(), v_pool.data_ptr(),
                            None if k_scale is None else k_scale.data_ptr(),
                            None if v_scale is None else v_scale.data_ptr(),

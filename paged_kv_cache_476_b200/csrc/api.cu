@@ -26,6 +26,11 @@ static int device_sms(int* sms) {
   return PKV_OK;
 }
 
+// Byte offset of an FP4 pool's block-scale region: all rows' codes come first.
+int64_t block_region_offset(const pkv_cache* c) {
+  return (int64_t)c->num_pages * c->num_kv_heads * c->page_size * (c->head_dim / 2);
+}
+
 // Validation shared by every entry point that reads the cache.
 int check_cache(const pkv_cache* c) {
   if (!c) return PKV_ERR_NULL;
@@ -35,7 +40,7 @@ int check_cache(const pkv_cache* c) {
   if (c->page_size != 64 && c->page_size != 128) return PKV_ERR_PAGE_SIZE;
   if (c->head_dim != 64 && c->head_dim != 128) return PKV_ERR_HEAD_DIM;
   if (c->kv_dtype != PKV_KV_BF16 && c->kv_dtype != PKV_KV_FP8_E4M3 &&
-      c->kv_dtype != PKV_KV_INT8)
+      c->kv_dtype != PKV_KV_INT8 && c->kv_dtype != PKV_KV_NVFP4)
     return PKV_ERR_DTYPE;
   if (c->kv_dtype != PKV_KV_BF16 && (!c->k_scale || !c->v_scale)) return PKV_ERR_DTYPE;
   // pool rows (pages * heads * page_size) index a TMA tensor: keep them in int32
@@ -77,20 +82,23 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D view [rows][row_elems] of a pool with a [64 rows][box_cols] box.
-int encode_pool_map(CUtensorMap* map, void* base, bool fp8, int64_t rows, int row_elems,
+// 2-D view [rows][row_elems] of a pool's codes (bytes, or bf16 elements)
+// with a [box_rows][box_cols] box and the swizzle of the box's row width
+// (128, 64 or 32 bytes).
+int encode_pool_map(CUtensorMap* map, void* base, bool bytes, int64_t rows, int row_elems,
                     int box_cols, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return PKV_ERR_CUDA;
-  const int eb = fp8 ? 1 : 2;
+  const int eb = bytes ? 1 : 2;
   const int box_bytes = box_cols * eb;
   cuuint64_t dims[2] = {(cuuint64_t)row_elems, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)row_elems * eb};
   cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUtensorMapSwizzle sw =
-      box_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  CUresult r = fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+  CUtensorMapSwizzle sw = box_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : box_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                            : CU_TENSOR_MAP_SWIZZLE_32B;
+  CUresult r = fn(map, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                   base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_CUDA;
@@ -166,6 +174,8 @@ int paged_kv_append(const pkv_cache* cache, const int32_t* page_table, int32_t m
   AppendParams p;
   p.k_pool = static_cast<uint8_t*>(cache->k_pool);
   p.v_pool = static_cast<uint8_t*>(cache->v_pool);
+  p.k_blocks = fp4(cache->kv_dtype) ? p.k_pool + block_region_offset(cache) : nullptr;
+  p.v_blocks = fp4(cache->kv_dtype) ? p.v_pool + block_region_offset(cache) : nullptr;
   p.k_scale = cache->k_scale;
   p.v_scale = cache->v_scale;
   p.page_table = page_table;
@@ -247,7 +257,6 @@ static int decode_entry(const pkv_cache* cache, const void* q, int32_t num_q_hea
   if (!workspace || !aligned16(workspace) || workspace_bytes < need) return PKV_ERR_WORKSPACE;
 
   const int fmt = cache->kv_dtype;
-  const bool fp8 = k8(fmt);  // one-byte codes (E4M3 or INT8)
   int sms = 0, per_sm = 0;
   if ((st = device_sms(&sms))) return st;
   if ((st = decode_ctas_per_sm(cache->head_dim, fmt, gqa_group, &per_sm))) return st;
@@ -259,10 +268,14 @@ static int decode_entry(const pkv_cache* cache, const void* q, int32_t num_q_hea
 
   const int D = cache->head_dim;
   const int64_t rows = (int64_t)cache->num_pages * cache->num_kv_heads * cache->page_size;
-  const int box_cols = fp8 ? (D >= 128 ? 128 : D) : 64;
+  // quantised pools are viewed as bytes: a row holds D codes (one-byte
+  // formats) or D/2 (FP4); bf16 rows are loaded in 64-element boxes
+  const bool bytes = quant(fmt);
+  const int row_elems = fp4(fmt) ? D / 2 : D;
+  const int box_cols = bytes ? (row_elems >= 128 ? 128 : row_elems) : 64;
   CUtensorMap tk, tv;
-  if ((st = encode_pool_map(&tk, cache->k_pool, fp8, rows, D, box_cols, 64))) return st;
-  if ((st = encode_pool_map(&tv, cache->v_pool, fp8, rows, D, box_cols, 64))) return st;
+  if ((st = encode_pool_map(&tk, cache->k_pool, bytes, rows, row_elems, box_cols, 64))) return st;
+  if ((st = encode_pool_map(&tv, cache->v_pool, bytes, rows, row_elems, box_cols, 64))) return st;
 
   const size_t G = (size_t)gqa_group;
   const size_t units = (size_t)batch * cache->num_kv_heads;
@@ -291,11 +304,19 @@ static int decode_entry(const pkv_cache* cache, const void* q, int32_t num_q_hea
   p.part_ml = part_ml;
   p.unit_info = unit_info;
   p.flags = cache->error_flags;
+  if (fp4(fmt)) {
+    p.k_blocks = static_cast<const uint8_t*>(cache->k_pool) + block_region_offset(cache);
+    p.v_blocks = static_cast<const uint8_t*>(cache->v_pool) + block_region_offset(cache);
+  }
   if (k_new) {
     p.k_new = static_cast<const __nv_bfloat16*>(k_new);
     p.v_new = static_cast<const __nv_bfloat16*>(v_new);
     p.k_pool = static_cast<uint8_t*>(cache->k_pool);
     p.v_pool = static_cast<uint8_t*>(cache->v_pool);
+    if (fp4(fmt)) {
+      p.k_blocks_w = p.k_pool + block_region_offset(cache);
+      p.v_blocks_w = p.v_pool + block_region_offset(cache);
+    }
   }
   p.batch = batch;
   p.num_q_heads = num_q_heads;

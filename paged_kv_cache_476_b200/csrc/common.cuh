@@ -128,6 +128,17 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// Plain bulk copy (no multicast) of `bytes` contiguous bytes into this CTA's
+// shared memory; both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // 3-D tiled TMA load (no multicast).
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, int32_t x,
                                             int32_t y, int32_t z, uint64_t* bar) {
@@ -226,6 +237,29 @@ __device__ __forceinline__ uint16_t encode8x2(__nv_bfloat162 x, float scale) {
     return static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3));
 }
 
+// Four 8-bit KV codes of format kFmt (one 32-bit word, byte 0 first) to two
+// f16x2: lo = codes 0, 1 and hi = codes 2, 3 (exact for both formats).  INT8
+// flips the four sign bits at once, then puts each code under the f16
+// exponent of 1024 as s8x2_to_f16x2 does; E4M3 converts each 16-bit half.
+template <int kFmt>
+__device__ __forceinline__ void kv8x4_to_f16x2(uint32_t codes, uint32_t& lo, uint32_t& hi) {
+  if constexpr (kFmt == PKV_KV_INT8) {
+    const uint32_t u = codes ^ 0x80808080u;
+    const uint32_t bias = 0x64806480u;  // f16x2 {1152, 1152}
+    lo = __byte_perm(u, 0x6464u, 0x4140);  // bytes: u0, 0x64, u1, 0x64
+    hi = __byte_perm(u, 0x6464u, 0x4342);  // bytes: u2, 0x64, u3, 0x64
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(lo) : "r"(lo), "r"(bias));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(hi) : "r"(hi), "r"(bias));
+  } else {
+    asm("{\n\t.reg .b16 l, h;\n\t"
+        "mov.b32 {l, h}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, l;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(codes));
+  }
+}
+
 // Two 8-bit KV codes of format kFmt to an f16x2 (exact for both formats).
 template <int kFmt>
 __device__ __forceinline__ uint32_t kv8x2_to_f16x2(uint16_t codes) {
@@ -233,6 +267,90 @@ __device__ __forceinline__ uint32_t kv8x2_to_f16x2(uint16_t codes) {
     return s8x2_to_f16x2(codes);
   else
     return e4m3x2_to_f16x2(codes);
+}
+
+// ------------------------------------------------------------ FP4 (E2M1)
+// E2M1 code of y (1 sign, 2 exponent bits with bias 1, 1 mantissa bit:
+// magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), nearest with ties to the even
+// code, |y| >= 6 saturating to 6, NaN as +0.  The magnitude code counts the
+// midpoints between neighbours that |y| lies above; a midpoint itself goes
+// to the even neighbour, hence '>' towards an even upper code's left and '>='
+// where the upper neighbour is the even one.
+__device__ __forceinline__ uint32_t e2m1_code(float y) {
+  if (y != y) return 0u;
+  const float a = fabsf(y);
+  const uint32_t m = (uint32_t)(a > 0.25f) + (uint32_t)(a >= 0.75f) + (uint32_t)(a > 1.25f) +
+                     (uint32_t)(a >= 1.75f) + (uint32_t)(a > 2.5f) + (uint32_t)(a >= 3.5f) +
+                     (uint32_t)(a > 5.0f);
+  return m | (__float_as_uint(y) >> 31 << 3);
+}
+
+// One FP4 block: 16 bf16 values (lo = elements 0-7, hi = 8-15) under the
+// (page, kv head) scale s.  sb = e4m3_rne_satfinite(amax / fp32(6 s)) with
+// NaN ignored in amax; d = fp32(decode(sb) * s); code_i =
+// e2m1(d > 0 ? fp32(x_i / d) : 0).  Returns the 8 code bytes (element 2k in
+// the low nibble of byte k) and the block-scale byte.  Every writer of FP4
+// pools goes through here, so all write the same bytes.
+__device__ __forceinline__ uint2 nvfp4_encode_block(const uint4& lo, const uint4& hi, float s,
+                                                    uint32_t* sb_out) {
+  float x[16];
+  const __nv_bfloat162* p0 = reinterpret_cast<const __nv_bfloat162*>(&lo);
+  const __nv_bfloat162* p1 = reinterpret_cast<const __nv_bfloat162*>(&hi);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 a = __bfloat1622float2(p0[k]);
+    const float2 b = __bfloat1622float2(p1[k]);
+    x[2 * k] = a.x;
+    x[2 * k + 1] = a.y;
+    x[8 + 2 * k] = b.x;
+    x[8 + 2 * k + 1] = b.y;
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));  // fmaxf drops NaN
+  const float ratio = __fdiv_rn(amax, __fmul_rn(6.0f, s));
+  const uint32_t sb = (uint32_t)__nv_cvt_float_to_fp8(ratio, __NV_SATFINITE, __NV_E4M3);
+  __half_raw hr = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)sb, __NV_E4M3);
+  const float d = __fmul_rn(__half2float(__half(hr)), s);
+  uint32_t w[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t c = e2m1_code(d > 0.f ? __fdiv_rn(x[i], d) : 0.f);
+    w[i >> 3] |= c << (4 * (i & 7));
+  }
+  *sb_out = sb;
+  return make_uint2(w[0], w[1]);
+}
+
+// Four bytes of E2M1 code pairs to four f16x2 (exact; the low nibble of a
+// byte becomes the low half).
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t codes, uint32_t* out) {
+  asm("{\n\t.reg .b8 c0, c1, c2, c3;\n\t"
+      "mov.b32 {c0, c1, c2, c3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, c0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, c1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, c2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, c3;\n\t}"
+      : "=r"(out[0]), "=r"(out[1]), "=r"(out[2]), "=r"(out[3])
+      : "r"(codes));
+}
+
+// The E4M3 block-scale byte k (0-3) of `word` as an f16x2 with that value in
+// both halves (exact).
+__device__ __forceinline__ uint32_t e4m3_splat_f16x2(uint32_t word, uint32_t k) {
+  return e4m3x2_to_f16x2((uint16_t)__byte_perm(word, 0u, k | (k << 4)));
+}
+
+// Two E4M3 bytes (k0 of word a, k1 of word b) as an f16x2 {a.k0, b.k1}.
+__device__ __forceinline__ uint32_t e4m3_pair_f16x2(uint32_t a, uint32_t k0, uint32_t b,
+                                                    uint32_t k1) {
+  return e4m3x2_to_f16x2((uint16_t)__byte_perm(a, b, k0 | ((k1 + 4) << 4)));
+}
+
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
 }
 
 // 2^x on the MUFU unit (flush-to-zero for tiny results).
@@ -250,5 +368,8 @@ __device__ __forceinline__ uint32_t swz128(uint32_t off) {
 
 // Same for the 64-byte swizzle (512-byte aligned tile base).
 __device__ __forceinline__ uint32_t swz64(uint32_t off) { return off ^ (((off >> 7) & 3u) << 4); }
+
+// Same for the 32-byte swizzle (256-byte aligned tile base).
+__device__ __forceinline__ uint32_t swz32(uint32_t off) { return off ^ (((off >> 7) & 1u) << 4); }
 
 }  // namespace pkv

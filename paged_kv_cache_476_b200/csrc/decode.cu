@@ -29,6 +29,8 @@
 //    straight into the f16 A fragments of V^T.  The per-(page, head) scales
 //    fold into the scores (K) and into P (V).
 //  * Every wait is bounded; a bad page id or length is skipped and flagged.
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -71,13 +73,16 @@ struct FlushDesc {
 
 template <int D, int kFmt>
 struct Layout {
-  static constexpr int kEB = k8(kFmt) ? 1 : 2;
-  static constexpr int kRowB = D * kEB;                        // bytes of a token row
+  static constexpr int kMapEB = kFmt == PKV_KV_BF16 ? 2 : 1;   // element bytes of the TMA map
+  static constexpr int kRowB = row_code_bytes(kFmt, D);        // code bytes of a token row
   static constexpr int kBoxRowB = kRowB >= 128 ? 128 : kRowB;  // TMA box inner bytes
   static constexpr int kNumBox = kRowB / kBoxRowB;             // boxes per tile row
   static constexpr int kBoxB = kTile * kBoxRowB;
-  static constexpr int kTileB = kNumBox * kBoxB;  // one K (or V) tile
-  static constexpr int kStageB = 2 * kTileB;
+  static constexpr int kTileB = kNumBox * kBoxB;  // codes of one K (or V) tile
+  // FP4: the E4M3 block scales of a tile's rows, after the two code tiles
+  static constexpr int kScaleRowB = row_scale_bytes(kFmt, D);
+  static constexpr int kScaleB = kTile * kScaleRowB;
+  static constexpr int kStageB = 2 * kTileB + 2 * kScaleB;
 };
 
 // Shared-memory carve-up; the Q slices and the reduction buffers are sized
@@ -113,16 +118,33 @@ __host__ __device__ inline SmemPlan smem_plan(int G) {
   return s;
 }
 
-// Byte address of 16-byte chunk `chunk` of row `row` in a TMA-swizzled tile
-// made of kNumBox boxes of [rows][kBoxRowB].
+// Byte addresses in a TMA-swizzled tile made of kNumBox boxes of
+// [rows][kBoxRowB]: chunk c (16 bytes) of row r lies at box (c / chunks per
+// box), row offset r * kBoxRowB, chunk (c % chunks per box) XOR the row bits
+// of the swizzle (128-, 64- or 32-byte pattern).
+// Each lane's address is split into its own part, computed once, and a part
+// known at compile time.  A lane reads chunk ce + lo of row `row` for even
+// chunks ce; with xk the row bits the swizzle XORs into the chunk index,
+// (ce + lo) ^ xk = (ce ^ (xk & ~1)) + (lo ^ (xk & 1)), so the address is
+// base + box(ce) + a + ((ce % chunks-per-box) * 16 ^ x).
+struct LaneTile {
+  uint32_t a;  // row * box row bytes + 16 * (lo ^ (xk & 1))
+  uint32_t x;  // 16 * (xk & ~1)
+};
+
+template <int kBoxRowB>
+__device__ __forceinline__ LaneTile lane_tile(int row, int lo) {
+  constexpr int kShift = kBoxRowB == 128 ? 0 : kBoxRowB == 64 ? 1 : 2;
+  constexpr int kMask = kBoxRowB / 16 - 1;
+  const int xk = (row >> kShift) & kMask;
+  return {(uint32_t)(row * kBoxRowB + ((lo ^ (xk & 1)) << 4)), (uint32_t)((xk & ~1) << 4)};
+}
+
 template <int kBoxRowB, int kRows>
-__device__ __forceinline__ uint32_t tile_addr(uint32_t base, int row, int chunk) {
+__device__ __forceinline__ uint32_t tile_at(uint32_t base, LaneTile lt, int ce) {
   constexpr int kChunksPerBox = kBoxRowB / 16;
-  const int box = chunk / kChunksPerBox;
-  const int c = chunk % kChunksPerBox;
-  const uint32_t off = row * kBoxRowB + c * 16;
-  const uint32_t sw = kBoxRowB == 128 ? swz128(off) : swz64(off);
-  return base + box * (kRows * kBoxRowB) + sw;
+  return base + (ce / kChunksPerBox) * (kRows * kBoxRowB) + lt.a +
+         (((uint32_t)(ce % kChunksPerBox) << 4) ^ lt.x);
 }
 
 // CTA (of C <= T over T tiles) whose range [c*T/C, (c+1)*T/C) holds global
@@ -151,6 +173,20 @@ __device__ __forceinline__ void append_newest(const DecodeParams& p, int b, int 
                                               int slot, float ks, float vs, int lane) {
   const int64_t src = ((int64_t)b * p.num_kv_heads + g) * D;
   const int64_t dst = (((int64_t)pid * p.num_kv_heads + g) * p.page_size + slot) * D;
+  if constexpr (fp4(kFmt)) {
+    // lanes 0..D/16-1 quantise K's blocks, lanes 16..16+D/16-1 V's
+    const int blk = lane & 15;
+    const bool is_v = lane >= 16;
+    if (blk < D / 16) {
+      const uint4* x = reinterpret_cast<const uint4*>((is_v ? p.v_new : p.k_new) + src + blk * 16);
+      uint32_t sb;
+      const uint2 codes = nvfp4_encode_block(x[0], x[1], is_v ? vs : ks, &sb);
+      const int64_t row = dst / D;
+      *reinterpret_cast<uint2*>((is_v ? p.v_pool : p.k_pool) + row * (D / 2) + blk * 8) = codes;
+      (is_v ? p.v_blocks_w : p.k_blocks_w)[row * (D / 16) + blk] = static_cast<uint8_t>(sb);
+    }
+    return;
+  }
   for (int e = lane * 4; e < D; e += 128) {
     const uint2 kx = *reinterpret_cast<const uint2*>(p.k_new + src + e);
     const uint2 vx = *reinterpret_cast<const uint2*>(p.v_new + src + e);
@@ -357,13 +393,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int j = t / tiles_per_page;
       const int sub = t - j * tiles_per_page;
       const int pages_b = (len + p.page_size - 1) / p.page_size;
-      const int key = k8(kFmt) ? b * Hkv + g : b;
+      const int key = quant(kFmt) ? b * Hkv + g : b;
       if (cache_key != key || j < cache_j0 || j >= cache_j0 + 32) {
         cache_key = key;
         cache_j0 = j;
         const int jj = j + lane;
         my_pid = jj < pages_b ? __ldg(p.page_table + (int64_t)b * p.max_pages + jj) : 0;
-        if constexpr (k8(kFmt)) {
+        if constexpr (quant(kFmt)) {
           if (jj < pages_b && my_pid >= 0 && my_pid < p.num_pages) {
             my_ks = __ldg(p.k_scale + (int64_t)my_pid * Hkv + g);
             my_vs = __ldg(p.v_scale + (int64_t)my_pid * Hkv + g);
@@ -373,12 +409,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       int pid = __shfl_sync(0xffffffffu, my_pid, j - cache_j0);
       const bool page_ok = pid >= 0 && pid < p.num_pages;
       float ks = 1.f, vs = 1.f;
-      if constexpr (k8(kFmt)) {
+      if constexpr (quant(kFmt)) {
         ks = __shfl_sync(0xffffffffu, my_ks, j - cache_j0);
         vs = __shfl_sync(0xffffffffu, my_vs, j - cache_j0);
       }
       bool bad = pid < 0 || pid >= p.num_pages;
-      if constexpr (k8(kFmt)) {
+      if constexpr (quant(kFmt)) {
         if (!bad && !(ks > 0.f && ks <= 32768.f && vs > 0.f && vs <= 32768.f)) {
           bad = true;
           if (lane == 0) flag_error(p.flags, PKV_FLAG_BAD_SCALE);
@@ -435,9 +471,17 @@ __global__ void __launch_bounds__(kThreads, 2)
         uint8_t* vdst = kdst + Ly::kTileB;
 #pragma unroll
         for (int bx = 0; bx < Ly::kNumBox; ++bx) {
-          const int32_t xc = bx * (Ly::kBoxRowB / Ly::kEB);
+          const int32_t xc = bx * (Ly::kBoxRowB / Ly::kMapEB);
           tma_load_2d(kdst + bx * Ly::kBoxB, &tmap_k, xc, y, &full[stage], pol);
           tma_load_2d(vdst + bx * Ly::kBoxB, &tmap_v, xc, y, &full[stage], pol);
+        }
+        if constexpr (fp4(kFmt)) {
+          // the tile's block scales: kTile consecutive rows of the
+          // block-scale region, one contiguous run of kScaleB bytes
+          const int64_t soff = (int64_t)y * Ly::kScaleRowB;
+          bulk_load(vdst + Ly::kTileB, p.k_blocks + soff, Ly::kScaleB, &full[stage]);
+          bulk_load(vdst + Ly::kTileB + Ly::kScaleB, p.v_blocks + soff, Ly::kScaleB,
+                    &full[stage]);
         }
         if (first) {
           const __nv_bfloat16* src = p.q + ((int64_t)b * p.num_q_heads + (int64_t)g * G) * D;
@@ -489,6 +533,11 @@ __global__ void __launch_bounds__(kThreads, 2)
   float ot[D / 16][4];
   float m_run = -INFINITY, l_part = 0.f;
   float qk_mul = p.scale_log2;  // multiplier of the raw scores into log2 units
+  // ldmatrix lanes: K (and bf16 V) matrices (tokens 0-7 | 8-15) x (chunk even |
+  // odd) in the order (0-7, ce), (0-7, ce+1), (8-15, ce), (8-15, ce+1); the
+  // quantised V loads order them (0-7, ce), (8-15, ce), (0-7, ce+1), (8-15, ce+1)
+  const LaneTile ltk = lane_tile<Ly::kBoxRowB>(16 * warp + mrow + (mat >> 1) * 8, mat & 1);
+  const LaneTile ltv = lane_tile<Ly::kBoxRowB>(16 * warp + mrow + (mat & 1) * 8, mat >> 1);
 
   for (int64_t i = 0; i < n_tiles; ++i) {
     const int stage = (int)(i % kStages);
@@ -498,15 +547,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     // bookkeeping is read from the (still unreleased) stage at hand-off
     const int t_flags = info[stage].flags;
     const int t_valid = info[stage].valid;
-    const float t_ks = k8(kFmt) ? info[stage].ks : 1.f;
-    const float t_vs = k8(kFmt) ? info[stage].vs : 1.f;
+    const float t_ks = quant(kFmt) ? info[stage].ks : 1.f;
+    const float t_vs = quant(kFmt) ? info[stage].vs : 1.f;
     const uint8_t* qs = qbuf + stage * kQStride;
     if (t_flags & kSegFirst) {
       m_run = -INFINITY;
       l_part = 0.f;
 #pragma unroll
       for (int m = 0; m < D / 16; ++m) ot[m][0] = ot[m][1] = ot[m][2] = ot[m][3] = 0.f;
-      if constexpr (!k8(kFmt)) {
+      if constexpr (!quant(kFmt)) {
 #pragma unroll
         for (int kk = 0; kk < KS; ++kk) {
           const uint32_t* qrow = reinterpret_cast<const uint32_t*>(qs + gid * D * 2);
@@ -515,18 +564,22 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         qk_mul = p.scale_log2;
       } else {
-        // f16 Q with a per-row power-of-two prescale; inside each 16-wide d
-        // block, the fragment's k pair (2*tid4, +1) holds d = 4*tid4 + {0,1}
-        // and the pair (2*tid4+8, +9) holds d = 4*tid4 + {2,3}, matching the
-        // byte order of the E4M3 K rows delivered by ldmatrix.
+        // f16 Q with a per-row power-of-two prescale, in the d order of the
+        // K codes that ldmatrix delivers.  One-byte codes: inside each
+        // 16-wide d block, the fragment's k pair (2*tid4, +1) holds d =
+        // 4*tid4 + {0,1} and the pair (2*tid4+8, +9) holds d = 4*tid4 + {2,3}.
+        // FP4: a 16-byte chunk c holds d = 32c..32c+31 and a thread's 4 bytes
+        // are d = 32c + 8*tid4 + {0..7}; k-step 2c takes the first four of
+        // them, k-step 2c+1 the last four.
         float amax = 0.f;
         float qv[KS][4];
 #pragma unroll
         for (int kk = 0; kk < KS; ++kk) {
           const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(qs) + gid * D;
+          const int d0 = fp4(kFmt) ? 32 * (kk >> 1) + 8 * tid4 + 4 * (kk & 1) : 16 * kk + 4 * tid4;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            qv[kk][e] = row_ok ? __bfloat162float(qrow[16 * kk + 4 * tid4 + e]) : 0.f;
+            qv[kk][e] = row_ok ? __bfloat162float(qrow[d0 + e]) : 0.f;
             amax = fmaxf(amax, fabsf(qv[kk][e]));
           }
         }
@@ -554,15 +607,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint32_t vbase = kbase + Ly::kTileB;
       // ---- S = Q K^T over my 16 tokens (two n-tiles of 8) ----
       float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      if constexpr (!k8(kFmt)) {
+      if constexpr (!quant(kFmt)) {
         // two independent accumulation chains per n-tile (even / odd k-steps)
         float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
         for (int kk = 0; kk < KS; ++kk) {
-          const int row = 16 * warp + mrow + (mat >> 1) * 8;
-          const int chunk = 2 * kk + (mat & 1);
           uint32_t b0, b1, b2, b3;
-          ldsm_x4(tile_addr<Ly::kBoxRowB, kTile>(kbase, row, chunk), b0, b1, b2, b3);
+          ldsm_x4(tile_at<Ly::kBoxRowB, kTile>(kbase, ltk, 2 * kk), b0, b1, b2, b3);
           float(*acc)[4] = (kk & 1) ? s2 : s;
           mma_bf16(acc[0], qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
           mma_bf16(acc[1], qa[kk][0], 0u, qa[kk][1], 0u, b2, b3);
@@ -571,26 +622,53 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int n = 0; n < 2; ++n)
 #pragma unroll
           for (int e = 0; e < 4; ++e) s[n][e] += s2[n][e];
+      } else if constexpr (fp4(kFmt)) {
+        // FP4 codes: a register of 4 bytes holds d = 32c + 8*tid4 + {0..7} of
+        // one token, all in block 2c + tid4/2; its four f16x2 (exact), each
+        // times the token's block scale (exact in f16), are the B fragments
+        // of k-steps 2c (bytes 0, 1) and 2c+1 (bytes 2, 3).
+        const uint8_t* ksc = tiles + stage * Ly::kStageB + 2 * Ly::kTileB;
+        uint32_t sk[2][Ly::kScaleRowB / 4];  // block scales of tokens gid and gid+8
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+          for (int w4 = 0; w4 < Ly::kScaleRowB / 4; ++w4)
+            sk[n][w4] = *reinterpret_cast<const uint32_t*>(
+                ksc + (16 * warp + 8 * n + gid) * Ly::kScaleRowB + 4 * w4);
+#pragma unroll
+        for (int c = 0; c < D / 32; c += 2) {
+          // matrices: (tokens 0-7, chunk c), (0-7, c+1), (8-15, c), (8-15, c+1)
+          uint32_t r[4];
+          ldsm_x4(tile_at<Ly::kBoxRowB, kTile>(kbase, ltk, c), r[0], r[1], r[2], r[3]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int n = i >> 1, cc = c + (i & 1);
+            const uint32_t blk = 2 * cc + (tid4 >> 1);
+            const uint32_t sbh = e4m3_splat_f16x2(sk[n][blk >> 2], blk & 3);
+            uint32_t f[4];
+            e2m1x8_to_f16x2(r[i], f);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) f[k] = hmul2_u32(f[k], sbh);
+            mma_f16(s[n], qa[2 * cc][0], 0u, qa[2 * cc][1], 0u, f[0], f[1]);
+            mma_f16(s[n], qa[2 * cc + 1][0], 0u, qa[2 * cc + 1][1], 0u, f[2], f[3]);
+          }
+        }
       } else {
 #pragma unroll
         for (int kp = 0; kp < KS / 2; ++kp) {
           // matrices: (tokens 0-7, chunk 2kp), (0-7, 2kp+1), (8-15, 2kp), (8-15, 2kp+1)
-          const int row = 16 * warp + mrow + (mat >> 1) * 8;
-          const int chunk = 2 * kp + (mat & 1);
-          uint32_t r0, r1, r2, r3;
-          ldsm_x4(tile_addr<Ly::kBoxRowB, kTile>(kbase, row, chunk), r0, r1, r2, r3);
-          mma_f16(s[0], qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, kv8x2_to_f16x2<kFmt>(r0 & 0xffff),
-                  kv8x2_to_f16x2<kFmt>(r0 >> 16));
-          mma_f16(s[0], qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u,
-                  kv8x2_to_f16x2<kFmt>(r1 & 0xffff), kv8x2_to_f16x2<kFmt>(r1 >> 16));
-          mma_f16(s[1], qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, kv8x2_to_f16x2<kFmt>(r2 & 0xffff),
-                  kv8x2_to_f16x2<kFmt>(r2 >> 16));
-          mma_f16(s[1], qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u,
-                  kv8x2_to_f16x2<kFmt>(r3 & 0xffff), kv8x2_to_f16x2<kFmt>(r3 >> 16));
+          uint32_t r[4];
+          ldsm_x4(tile_at<Ly::kBoxRowB, kTile>(kbase, ltk, 2 * kp), r[0], r[1], r[2], r[3]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint32_t lo, hi;
+            kv8x4_to_f16x2<kFmt>(r[i], lo, hi);
+            mma_f16(s[i >> 1], qa[2 * kp + (i & 1)][0], 0u, qa[2 * kp + (i & 1)][1], 0u, lo, hi);
+          }
         }
       }
       // ---- online softmax on row gid (log2 domain) ----
-      const float mul = k8(kFmt) ? qk_mul * t_ks : qk_mul;
+      const float mul = quant(kFmt) ? qk_mul * t_ks : qk_mul;
       float x[4];
 #pragma unroll
       for (int n = 0; n < 2; ++n)
@@ -624,61 +702,117 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       // ---- O^T += V^T P^T over my 16 tokens (P^T comes straight from S) ----
       uint32_t pa0, pa2;
-      if constexpr (!k8(kFmt)) {
+      if constexpr (!quant(kFmt)) {
         pa0 = pack_bf16(pr[0], pr[1]);
         pa2 = pack_bf16(pr[2], pr[3]);
       } else {
         pa0 = pack_f16(pr[0] * t_vs, pr[1] * t_vs);
         pa2 = pack_f16(pr[2] * t_vs, pr[3] * t_vs);
       }
-      // V rows past the length may hold anything (NaN); zero them in the
-      // fragments so that 0 * NaN never reaches the accumulator.
-      uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;
-      if (valid < 16) {
-        vm0 = (2 * tid4 < valid ? 0x0000ffffu : 0u) | (2 * tid4 + 1 < valid ? 0xffff0000u : 0u);
-        vm1 = (2 * tid4 + 8 < valid ? 0x0000ffffu : 0u) |
-              (2 * tid4 + 9 < valid ? 0xffff0000u : 0u);
-      }
-      if constexpr (!k8(kFmt)) {
-#pragma unroll
-        for (int m = 0; m < D / 16; ++m) {
-          // A = V^T rows d 16m..16m+15: matrices (tokens 0-7, chunk 2m), (0-7, 2m+1),
-          // (8-15, 2m), (8-15, 2m+1), transposed on load
-          const int chunk = 2 * m + (mat & 1);
-          const int row = 16 * warp + mrow + (mat >> 1) * 8;
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4_t(tile_addr<Ly::kBoxRowB, kTile>(vbase, row, chunk), a0, a1, a2, a3);
-          mma_bf16(ot[m], a0 & vm0, a1 & vm0, a2 & vm1, a3 & vm1, pa0, pa2);
+      // V rows past the length may hold anything (NaN): on a partial tile
+      // they are zeroed in the fragments, so that 0 * NaN never reaches the
+      // accumulator.  Full tiles, nearly all, take the product without masks.
+      auto pv_product = [&](auto masked) {
+        constexpr bool kMasked = decltype(masked)::value;
+        uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;
+        if constexpr (kMasked) {
+          vm0 = (2 * tid4 < valid ? 0x0000ffffu : 0u) | (2 * tid4 + 1 < valid ? 0xffff0000u : 0u);
+          vm1 = (2 * tid4 + 8 < valid ? 0x0000ffffu : 0u) |
+                (2 * tid4 + 9 < valid ? 0xffff0000u : 0u);
         }
-      } else {
-        // One-byte V codes straight from the landed tile.  A transposed load
-        // of 16-bit elements (byte pairs d, d+1) gives each thread, per 8x8
-        // matrix, codes of tokens (2*tid4, 2*tid4+1) x bytes (2*gid, 2*gid+1)
-        // of a 16-byte chunk; two exact conversions and a swap of 16-bit
-        // halves make the A fragment of V^T with row gid = d 16m + 2*gid and
-        // row gid+8 = d 16m + 2*gid + 1 (the snapshot below undoes the order).
-        auto v_rows = [&](uint32_t codes, uint32_t& even_d, uint32_t& odd_d) {
-          const uint32_t t0 = kv8x2_to_f16x2<kFmt>(codes & 0xffff);  // token 2*tid4
-          const uint32_t t1 = kv8x2_to_f16x2<kFmt>(codes >> 16);     // token 2*tid4+1
-          even_d = __byte_perm(t0, t1, 0x5410);
-          odd_d = __byte_perm(t0, t1, 0x7632);
-        };
+        // tokens 2*tid4, 2*tid4+1 (m0) or 2*tid4+8, 2*tid4+9 (m1) of a fragment
+        auto m0 = [&](uint32_t a) -> uint32_t { return kMasked ? (a & vm0) : a; };
+        auto m1 = [&](uint32_t a) -> uint32_t { return kMasked ? (a & vm1) : a; };
+        if constexpr (!quant(kFmt)) {
 #pragma unroll
-        for (int m = 0; m < D / 16; m += 2) {
-          // matrices: (tokens 0-7, chunk m), (8-15, m), (0-7, m+1), (8-15, m+1)
-          const int row = 16 * warp + mrow + (mat & 1) * 8;
-          const int chunk = m + (mat >> 1);
-          uint32_t r0, r1, r2, r3;
-          ldsm_x4_t(tile_addr<Ly::kBoxRowB, kTile>(vbase, row, chunk), r0, r1, r2, r3);
-          uint32_t a0, a1, a2, a3;
-          v_rows(r0, a0, a1);
-          v_rows(r1, a2, a3);
-          mma_f16(ot[m], a0 & vm0, a1 & vm0, a2 & vm1, a3 & vm1, pa0, pa2);
-          v_rows(r2, a0, a1);
-          v_rows(r3, a2, a3);
-          mma_f16(ot[m + 1], a0 & vm0, a1 & vm0, a2 & vm1, a3 & vm1, pa0, pa2);
+          for (int m = 0; m < D / 16; ++m) {
+            // A = V^T rows d 16m..16m+15: matrices (tokens 0-7, chunk 2m), (0-7, 2m+1),
+            // (8-15, 2m), (8-15, 2m+1), transposed on load
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_t(tile_at<Ly::kBoxRowB, kTile>(vbase, ltk, 2 * m), a0, a1, a2, a3);
+            mma_bf16(ot[m], m0(a0), m0(a1), m1(a2), m1(a3), pa0, pa2);
+          }
+        } else if constexpr (fp4(kFmt)) {
+          // FP4 V codes from the landed tile.  A transposed load of 16-bit
+          // elements (byte pairs) gives each thread, per 8x8 matrix, tokens
+          // (2*tid4, 2*tid4+1) x codes d = 32c + 4*gid + {0..3} (low half:
+          // the first token).  Interleaving the two tokens' nibbles makes
+          // four bytes, one per d, each the token pair of that d, which
+          // convert exactly to f16x2; times the two tokens' block scales
+          // (block 2c + gid/4) they are the A fragments of V^T.  Fragment
+          // rows: m-tile 2c holds d = 32c + 4*gid + {0, 1} (rows gid, gid+8),
+          // m-tile 2c+1 holds d = 32c + 4*gid + {2, 3}; the snapshot below
+          // undoes the order.
+          const uint8_t* vsc = tiles + stage * Ly::kStageB + 2 * Ly::kTileB + Ly::kScaleB;
+          uint32_t sv[4][Ly::kScaleRowB / 4];  // tokens 2t, 2t+1, 2t+8, 2t+9 of the warp
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+#pragma unroll
+            for (int w4 = 0; w4 < Ly::kScaleRowB / 4; ++w4)
+              sv[k][w4] = *reinterpret_cast<const uint32_t*>(
+                  vsc + (16 * warp + 2 * tid4 + (k & 1) + 8 * (k >> 1)) * Ly::kScaleRowB + 4 * w4);
+          auto v_pairs = [&](uint32_t codes, uint32_t scale_pair, uint32_t* f) {
+            const uint32_t x = __byte_perm(codes, 0u, 0x3120);  // A.d01 B.d01 A.d23 B.d23
+            const uint32_t lo = x & 0x0f0f0f0fu;                // A.d0 B.d0 A.d2 B.d2
+            const uint32_t hi = (x >> 4) & 0x0f0f0f0fu;         // A.d1 B.d1 A.d3 B.d3
+            const uint32_t z = __byte_perm(lo | (lo >> 4), hi | (hi >> 4), 0x6240);
+            e2m1x8_to_f16x2(z, f);                              // pairs of d0, d1, d2, d3
+#pragma unroll
+            for (int k = 0; k < 4; ++k) f[k] = hmul2_u32(f[k], scale_pair);
+          };
+#pragma unroll
+          for (int c = 0; c < D / 32; c += 2) {
+            // matrices: (tokens 0-7, chunk c), (8-15, c), (0-7, c+1), (8-15, c+1)
+            uint32_t r0, r1, r2, r3;
+            ldsm_x4_t(tile_at<Ly::kBoxRowB, kTile>(vbase, ltv, c), r0, r1, r2, r3);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int cc = c + h;
+              const uint32_t blk = 2 * cc + (gid >> 2);
+              const uint32_t s01 =
+                  e4m3_pair_f16x2(sv[0][blk >> 2], blk & 3, sv[1][blk >> 2], blk & 3);
+              const uint32_t s89 =
+                  e4m3_pair_f16x2(sv[2][blk >> 2], blk & 3, sv[3][blk >> 2], blk & 3);
+              uint32_t pf[4], qf[4];
+              v_pairs(h ? r2 : r0, s01, pf);  // tokens 2t, 2t+1
+              v_pairs(h ? r3 : r1, s89, qf);  // tokens 2t+8, 2t+9
+              mma_f16(ot[2 * cc], m0(pf[0]), m0(pf[1]), m1(qf[0]), m1(qf[1]), pa0, pa2);
+              mma_f16(ot[2 * cc + 1], m0(pf[2]), m0(pf[3]), m1(qf[2]), m1(qf[3]), pa0, pa2);
+            }
+          }
+        } else {
+          // One-byte V codes straight from the landed tile.  A transposed
+          // load of 16-bit elements (byte pairs d, d+1) gives each thread,
+          // per 8x8 matrix, codes of tokens (2*tid4, 2*tid4+1) x bytes
+          // (2*gid, 2*gid+1) of a 16-byte chunk; two exact conversions and a
+          // swap of 16-bit halves make the A fragment of V^T with row gid = d
+          // 16m + 2*gid and row gid+8 = d 16m + 2*gid + 1 (the snapshot
+          // below undoes the order).
+          auto v_rows = [&](uint32_t codes, uint32_t& even_d, uint32_t& odd_d) {
+            uint32_t t0, t1;  // tokens 2*tid4 and 2*tid4+1
+            kv8x4_to_f16x2<kFmt>(codes, t0, t1);
+            even_d = __byte_perm(t0, t1, 0x5410);
+            odd_d = __byte_perm(t0, t1, 0x7632);
+          };
+#pragma unroll
+          for (int m = 0; m < D / 16; m += 2) {
+            // matrices: (tokens 0-7, chunk m), (8-15, m), (0-7, m+1), (8-15, m+1)
+            uint32_t r0, r1, r2, r3;
+            ldsm_x4_t(tile_at<Ly::kBoxRowB, kTile>(vbase, ltv, m), r0, r1, r2, r3);
+            uint32_t a0, a1, a2, a3;
+            v_rows(r0, a0, a1);
+            v_rows(r1, a2, a3);
+            mma_f16(ot[m], m0(a0), m0(a1), m1(a2), m1(a3), pa0, pa2);
+            v_rows(r2, a0, a1);
+            v_rows(r3, a2, a3);
+            mma_f16(ot[m + 1], m0(a0), m0(a1), m1(a2), m1(a3), pa0, pa2);
+          }
         }
-      }
+      };
+      if (valid >= 16)
+        pv_product(std::false_type{});
+      else
+        pv_product(std::true_type{});
     }
     if (t_flags & kSegLast) {
     // ------------------------------------------- hand the segment over
@@ -696,12 +830,14 @@ __global__ void __launch_bounds__(kThreads, 2)
       float* r0 = red_o + (warp * G + h0) * D;
       float* r1 = red_o + (warp * G + h1) * D;
       // fragment rows gid and gid+8 of d-tile m hold d 16m + gid and +8
-      // (bf16), or 16m + 2*gid and +1 (one-byte codes, see the PV product)
-      const int d_step = k8(kFmt) ? 1 : 8;
-      const int d_lane = k8(kFmt) ? 2 * gid : gid;
+      // (bf16), 16m + 2*gid and +1 (one-byte codes), or 32(m/2) + 4*gid +
+      // 2(m%2) and +1 (FP4), as the PV products lay them out
+      const int d_step = quant(kFmt) ? 1 : 8;
 #pragma unroll
       for (int m = 0; m < D / 16; ++m) {
-        const int d = 16 * m + d_lane;
+        const int d = fp4(kFmt) ? 32 * (m >> 1) + 4 * gid + 2 * (m & 1)
+                     : k8(kFmt) ? 16 * m + 2 * gid
+                                : 16 * m + gid;
         if (h0 < G) {
           r0[d] = ot[m][0];
           r0[d + d_step] = ot[m][2];
@@ -892,6 +1028,9 @@ cudaError_t run_for(const CUtensorMap& tk, const CUtensorMap& tv, const DecodePa
 cudaError_t decode_occupancy(int head_dim, int fmt, int group, int* ctas_per_sm) {
   const bool d128 = head_dim == 128;
   switch (fmt) {
+    case PKV_KV_NVFP4:
+      return d128 ? occupancy_for<128, PKV_KV_NVFP4>(group, ctas_per_sm)
+                  : occupancy_for<64, PKV_KV_NVFP4>(group, ctas_per_sm);
     case PKV_KV_INT8:
       return d128 ? occupancy_for<128, PKV_KV_INT8>(group, ctas_per_sm)
                   : occupancy_for<64, PKV_KV_INT8>(group, ctas_per_sm);
@@ -908,6 +1047,9 @@ cudaError_t decode_run(int head_dim, int fmt, const CUtensorMap& tk, const CUten
                        const DecodeParams& p, int num_ctas, cudaStream_t stream) {
   const bool d128 = head_dim == 128;
   switch (fmt) {
+    case PKV_KV_NVFP4:
+      return d128 ? run_for<128, PKV_KV_NVFP4>(tk, tv, p, num_ctas, stream)
+                  : run_for<64, PKV_KV_NVFP4>(tk, tv, p, num_ctas, stream);
     case PKV_KV_INT8:
       return d128 ? run_for<128, PKV_KV_INT8>(tk, tv, p, num_ctas, stream)
                   : run_for<64, PKV_KV_INT8>(tk, tv, p, num_ctas, stream);

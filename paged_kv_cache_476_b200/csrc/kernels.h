@@ -11,14 +11,32 @@
 namespace pkv {
 
 // Number of pkv_kv_dtype values.
-constexpr int kNumKvFormats = 3;
+constexpr int kNumKvFormats = 4;
 
-// KV formats of the pools (pkv_kv_dtype): is the stored code one byte?
-__host__ __device__ constexpr bool k8(int fmt) { return fmt != PKV_KV_BF16; }
+// KV formats of the pools (pkv_kv_dtype).
+// One-byte element codes (E4M3, INT8)?
+__host__ __device__ constexpr bool k8(int fmt) {
+  return fmt == PKV_KV_FP8_E4M3 || fmt == PKV_KV_INT8;
+}
+// FP4: E2M1 code pairs plus E4M3 block scales?
+__host__ __device__ constexpr bool fp4(int fmt) { return fmt == PKV_KV_NVFP4; }
+// Quantised, with per-(page, kv head) scales (every format but bf16)?
+__host__ __device__ constexpr bool quant(int fmt) { return fmt != PKV_KV_BF16; }
+
+// Bytes of one token row of one kv head in a pool: element codes, and the
+// FP4 block scales (stored after every row's codes).
+__host__ __device__ constexpr int row_code_bytes(int fmt, int head_dim) {
+  return fmt == PKV_KV_BF16 ? 2 * head_dim : fp4(fmt) ? head_dim / 2 : head_dim;
+}
+__host__ __device__ constexpr int row_scale_bytes(int fmt, int head_dim) {
+  return fp4(fmt) ? head_dim / 16 : 0;
+}
 
 struct AppendParams {
   uint8_t* k_pool;
   uint8_t* v_pool;
+  uint8_t* k_blocks;  // FP4: block scales of the K pool (after its codes); else null
+  uint8_t* v_blocks;
   const float* k_scale;
   const float* v_scale;
   const int32_t* page_table;
@@ -54,6 +72,11 @@ struct DecodeParams {
   const __nv_bfloat16* v_new;
   uint8_t* k_pool;
   uint8_t* v_pool;
+  uint8_t* k_blocks_w;  // FP4 fused append: block-scale regions to write
+  uint8_t* v_blocks_w;
+  // FP4 pools: the block-scale regions (after the codes) that the loads read
+  const uint8_t* k_blocks;
+  const uint8_t* v_blocks;
   int32_t batch;
   int32_t num_q_heads;
   int32_t num_kv_heads;
@@ -76,7 +99,8 @@ cudaError_t launch_combine(const void* parts, const float* lse_parts, int num_pa
 int check_cache(const pkv_cache* c);
 int check_group(const pkv_cache* c, int32_t num_q_heads, int32_t gqa_group);
 int check_table_span(const pkv_cache* c, int32_t max_pages_per_seq);
-int encode_pool_map(CUtensorMap* map, void* base, bool fp8, int64_t rows, int row_elems,
+int64_t block_region_offset(const pkv_cache* c);
+int encode_pool_map(CUtensorMap* map, void* base, bool bytes, int64_t rows, int row_elems,
                     int box_cols, int box_rows);
 int prefill_entry(const pkv_cache* cache, const void* q, int32_t num_q_heads, int32_t gqa_group,
                   const int32_t* cu_q_lens, const int32_t* page_table, int32_t max_pages_per_seq,

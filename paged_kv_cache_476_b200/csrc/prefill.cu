@@ -62,8 +62,10 @@ __device__ __forceinline__ uint32_t col_s(int x) { return x ? 128u : 0u; }
 __device__ __forceinline__ uint32_t col_o(int x) { return x ? 384u : 256u; }
 
 struct Params {
-  const float* k_scale;  // [pages][Hkv] (E4M3 pools)
+  const float* k_scale;  // [pages][Hkv] (quantised pools)
   const float* v_scale;
+  const uint8_t* k_blocks;  // FP4 pools: the block-scale regions (after the codes)
+  const uint8_t* v_blocks;
   const int32_t* cu_q;
   const int32_t* page_table;
   const int32_t* seq_lens;
@@ -223,11 +225,16 @@ struct Smem {
   static constexpr int kQB = kRows * D * 2;         // one Q tile
   static constexpr int kTileB = kKeys * D * 2;      // bf16 K (or V) tile
   static constexpr int kHalfB = kKeys * 128;        // one 64-column half of a bf16 tile
-  static constexpr int kTile8B = kKeys * D;         // E4M3 K (or V) tile as it lands
-  static constexpr int kStageB = k8(kFmt) ? 2 * kTile8B : 2 * kTileB;
-  static constexpr int kConvB = k8(kFmt) ? 2 * kTileB : 0;  // converted K, then V
+  // a quantised K (or V) tile as it lands: the codes of its rows, then (FP4)
+  // their block scales
+  static constexpr int kCodeRowB = row_code_bytes(kFmt, D);
+  static constexpr int kScaleRowB = row_scale_bytes(kFmt, D);
+  static constexpr int kCodesB = kKeys * kCodeRowB;
+  static constexpr int kTileQB = kCodesB + kKeys * kScaleRowB;
+  static constexpr int kStageB = quant(kFmt) ? 2 * kTileQB : 2 * kTileB;
+  static constexpr int kConvB = quant(kFmt) ? 2 * kTileB : 0;  // converted K, then V
   static constexpr int kBytes = 2 * kQB + kStages * kStageB + kConvB;
-  static constexpr int kThreads = k8(kFmt) ? 384 : 320;  // + two converter warps
+  static constexpr int kThreads = quant(kFmt) ? 384 : 320;  // + two converter warps
 };
 
 // Per-KV-tile facts the producer passes on: rejected 64-key blocks and the
@@ -246,14 +253,16 @@ __device__ __forceinline__ uint32_t bf16_chunk(uint32_t base, int r, int c) {
   return base + (c >> 3) * (kKeys * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
 }
 
-// Same for an E4M3 tile as TMA writes it: rows of D bytes, 128-byte swizzle
-// (D = 128) or 64-byte swizzle (D = 64).
-template <int D>
-__device__ __forceinline__ uint32_t e4m3_chunk(uint32_t base, int r, int c) {
-  if constexpr (D == 128)
+// Same for a tile of codes as TMA writes it: rows of kRowB bytes with the
+// swizzle of that width (128, 64 or 32 bytes).
+template <int kRowB>
+__device__ __forceinline__ uint32_t code_chunk(uint32_t base, int r, int c) {
+  if constexpr (kRowB == 128)
     return base + r * 128 + ((c ^ (r & 7)) << 4);
-  else
+  else if constexpr (kRowB == 64)
     return base + r * 64 + ((c ^ ((r >> 1) & 3)) << 4);
+  else
+    return base + r * 32 + ((c ^ ((r >> 2) & 1)) << 4);
 }
 
 // E4M3 tile -> bf16 or f16 tile (both exact: every E4M3 value is an f16 and a
@@ -275,7 +284,7 @@ __device__ __forceinline__ void convert_tile(uint32_t src, uint32_t dst, int t, 
       uint32_t w[4];
       asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                    : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
-                   : "r"(e4m3_chunk<D>(src, r, c)));
+                   : "r"(code_chunk<D>(src, r, c)));
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const uint32_t h01 = kv8x2_to_f16x2<kFmt>(w[k] & 0xffff);
@@ -298,6 +307,54 @@ __device__ __forceinline__ void convert_tile(uint32_t src, uint32_t dst, int t, 
                      bf16_chunk<D>(dst, r, 2 * c + 1)),
                  "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7])
                  : "memory");
+  }
+}
+
+// FP4 tile (codes, then one E4M3 block scale per 16 values of a row) ->
+// bf16 or f16 tile, values e2m1(code) * decode(sb): exact in both, since the
+// product has at most 6 significant bits and lies in [2^-10, 2688].  Rows
+// in `zero_mask` or at/after `zero_from` are written as zeros.  64 threads.
+template <int D, bool kToF16>
+__device__ __forceinline__ void convert_fp4_tile(uint32_t src, uint32_t dst, int t, int zero_from,
+                                                 int zero_mask) {
+  constexpr int kRowB = D / 2;            // code bytes of a row
+  constexpr int kChunks = kKeys * D / 32;  // 16-byte chunks of codes (32 values, 2 blocks)
+  const uint32_t scales = src + kKeys * kRowB;
+#pragma unroll 2
+  for (int ci = t; ci < kChunks; ci += 64) {
+    const int r = ci / (D / 32);
+    const int c = ci - r * (D / 32);
+    uint32_t o[16];
+    if (r >= zero_from || ((zero_mask >> (r >> 6)) & 1)) {
+#pragma unroll
+      for (int k = 0; k < 16; ++k) o[k] = 0u;
+    } else {
+      uint32_t w[4];
+      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                   : "r"(code_chunk<kRowB>(src, r, c)));
+      uint32_t sb2;
+      asm volatile("ld.shared.u16 %0, [%1];" : "=r"(sb2) : "r"(scales + r * (D / 16) + 2 * c));
+      const uint32_t s0 = e4m3_splat_f16x2(sb2, 0), s1 = e4m3_splat_f16x2(sb2, 1);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        e2m1x8_to_f16x2(w[k], o + 4 * k);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[4 * k + i] = hmul2_u32(o[4 * k + i], k < 2 ? s0 : s1);
+      }
+      if constexpr (!kToF16) {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&o[k]));
+          o[k] = pack_bf16(f.x, f.y);
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(bf16_chunk<D>(dst, r, 4 * c + q)),
+                   "r"(o[4 * q]), "r"(o[4 * q + 1]), "r"(o[4 * q + 2]), "r"(o[4 * q + 3])
+                   : "memory");
   }
 }
 
@@ -466,8 +523,8 @@ __global__ void __launch_bounds__(Smem<D, kFmt>::kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
-      mbar_init(&k_empty[s], k8(kFmt) ? 2 : 1);  // E4M3: released by the two converter warps
-      mbar_init(&v_empty[s], k8(kFmt) ? 2 : 1);
+      mbar_init(&k_empty[s], quant(kFmt) ? 2 : 1);  // quantised: released by the two converter warps
+      mbar_init(&v_empty[s], quant(kFmt) ? 2 : 1);
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&s_full[x], 1);
@@ -560,7 +617,7 @@ __global__ void __launch_bounds__(Smem<D, kFmt>::kThreads, 1)
             lk.tf.bad |= 1 << sb;
             continue;
           }
-          if constexpr (k8(kFmt)) {
+          if constexpr (quant(kFmt)) {
             const float ks = __ldg(p.k_scale + (int64_t)pid * p.num_kv_heads + g);
             const float vs = __ldg(p.v_scale + (int64_t)pid * p.num_kv_heads + g);
             if (!(ks > 0.f && ks <= 32768.f && vs > 0.f && vs <= 32768.f)) {
@@ -578,14 +635,19 @@ __global__ void __launch_bounds__(Smem<D, kFmt>::kThreads, 1)
         return lk;
       };
       // bytes of one operand (K or V) per live 64-key block
-      constexpr uint32_t kBlockBytes = k8(kFmt) ? 64u * D : Sm::kHalves * 64u * 128u;
+      constexpr uint32_t kBlockBytes =
+          quant(kFmt) ? 64u * (Sm::kCodeRowB + Sm::kScaleRowB) : Sm::kHalves * 64u * 128u;
       // load one operand of a tile into its slot
-      auto load = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, const Lookup& lk) {
+      auto load = [&](const CUtensorMap* map, const uint8_t* blocks, uint8_t* dst, uint64_t* bar,
+                      const Lookup& lk) {
         mbar_arrive_expect_tx(bar, (uint32_t)__popc(lk.live) * kBlockBytes);
         for (int sb = 0; sb < 2; ++sb) {
           if (!((lk.live >> sb) & 1)) continue;
-          if constexpr (k8(kFmt)) {
-            tma_load_2d(dst + sb * 64 * D, map, 0, lk.ys[sb], bar, pol);
+          if constexpr (quant(kFmt)) {
+            tma_load_2d(dst + sb * 64 * Sm::kCodeRowB, map, 0, lk.ys[sb], bar, pol);
+            if constexpr (fp4(kFmt))  // the block scales of the same 64 rows
+              bulk_load(dst + Sm::kCodesB + sb * 64 * Sm::kScaleRowB,
+                        blocks + (int64_t)lk.ys[sb] * Sm::kScaleRowB, 64u * Sm::kScaleRowB, bar);
           } else {
 #pragma unroll
             for (int h = 0; h < Sm::kHalves; ++h)
@@ -605,13 +667,13 @@ __global__ void __launch_bounds__(Smem<D, kFmt>::kThreads, 1)
         if (j >= kStages && !mbar_wait(&k_empty[st], ph, p.flags)) break;
         facts[j % kFactsRing] = cur.tf;
         mbar_arrive(&facts_full[j % kFactsRing]);
-        load(&tmap_k, kd, &k_full[st], cur);
+        load(&tmap_k, p.k_blocks, kd, &k_full[st], cur);
         if (j >= kStages && !mbar_wait(&v_empty[st], ph, p.flags)) break;
-        load(&tmap_v, vd, &v_full[st], cur);
+        load(&tmap_v, p.v_blocks, vd, &v_full[st], cur);
         if (j + 1 < n_kv) cur = lookup(j + 1);  // ahead of the next slot wait
       }
     }
-  } else if (k8(kFmt) && warp >= kConvWarp0) {
+  } else if (quant(kFmt) && warp >= kConvWarp0) {
     // ------------------------------------------------- E4M3 -> 16-bit converters
     const int t = threadIdx.x - kConvWarp0 * 32;  // 0..63
     const uint32_t kc = smem_u32(sconv), vc = kc + Sm::kTileB;
@@ -626,7 +688,10 @@ __global__ void __launch_bounds__(Smem<D, kFmt>::kThreads, 1)
       const int zero_from = key0 + kKeys > L ? max(0, L - key0) : kKeys;
       // K (rows that must not count are masked in the scores; keep them finite)
       if (j >= 1 && !mbar_wait(kc_free, (uint32_t)((j - 1) & 1), p.flags)) break;
-      convert_tile<D, kFmt, false>(k_codes, kc, t, zero_from, bad);  // bf16, like Q
+      if constexpr (fp4(kFmt))
+        convert_fp4_tile<D, false>(k_codes, kc, t, zero_from, bad);  // bf16, like Q
+      else
+        convert_tile<D, kFmt, false>(k_codes, kc, t, zero_from, bad);
       fence_async_smem();
       __syncwarp();
       if (lane == 0) {
@@ -636,7 +701,10 @@ __global__ void __launch_bounds__(Smem<D, kFmt>::kThreads, 1)
       if (!mbar_wait(&v_full[st], par, p.flags)) break;
       // V (rows that must not count are zeros: 0 * NaN would poison O)
       if (j >= 1 && !mbar_wait(vc_free, (uint32_t)((j - 1) & 1), p.flags)) break;
-      convert_tile<D, kFmt, true>(v_codes, vc, t, zero_from, bad);  // f16, like P
+      if constexpr (fp4(kFmt))
+        convert_fp4_tile<D, true>(v_codes, vc, t, zero_from, bad);  // f16, like P
+      else
+        convert_tile<D, kFmt, true>(v_codes, vc, t, zero_from, bad);
       fence_async_smem();
       __syncwarp();
       if (lane == 0) {
@@ -650,11 +718,11 @@ __global__ void __launch_bounds__(Smem<D, kFmt>::kThreads, 1)
     // tensor core always has the other tile's work while a softmax runs.
     const uint32_t id_s = idesc_f16kind(kRows, kKeys, 0, true);
     // E4M3: P (scaled by the V scales) and V are f16 for the PV product
-    const uint32_t id_o = idesc_f16kind(kRows, D, 1, !k8(kFmt));
+    const uint32_t id_o = idesc_f16kind(kRows, D, 1, !quant(kFmt));
     const uint32_t q_addr = smem_u32(sq);
     bool ok = mbar_wait(q_full, 0, p.flags);
     auto k_ready = [&](int j, uint32_t* addr) -> bool {
-      if constexpr (k8(kFmt)) {
+      if constexpr (quant(kFmt)) {
         *addr = smem_u32(sconv);
         return mbar_wait(kc_full, (uint32_t)(j & 1), p.flags);
       } else {
@@ -681,7 +749,7 @@ __global__ void __launch_bounds__(Smem<D, kFmt>::kThreads, 1)
     // V of tile j, made safe for the PV product (rows past the end or of a
     // rejected page zeroed); returns false on a timeout
     auto v_ready = [&](int j, uint32_t* addr) -> bool {
-      if constexpr (k8(kFmt)) {
+      if constexpr (quant(kFmt)) {
         *addr = smem_u32(sconv) + Sm::kTileB;
         return mbar_wait(vc_full, (uint32_t)(j & 1), p.flags);
       } else {
@@ -731,7 +799,7 @@ __global__ void __launch_bounds__(Smem<D, kFmt>::kThreads, 1)
     if (ok) {
       issue_s(0, k_addr);
       if (hasB) issue_s(1, k_addr);
-      if (lane == 0) tc_commit(k8(kFmt) ? kc_free : &k_empty[0]);  // K_0 is read by both S products
+      if (lane == 0) tc_commit(quant(kFmt) ? kc_free : &k_empty[0]);  // K_0 is read by both S products
       __syncwarp();
     }
     for (int j = 0; j < n_kv && ok; ++j) {
@@ -744,10 +812,10 @@ __global__ void __launch_bounds__(Smem<D, kFmt>::kThreads, 1)
       if (j < nkv[1] && !(ok = issue_pv(1, j, v_addr))) break;
       // V_j is consumed once both PV products have run, K_{j+1} once both
       // S products have
-      if (lane == 0) tc_commit(k8(kFmt) ? vc_free : &v_empty[j % kStages]);
+      if (lane == 0) tc_commit(quant(kFmt) ? vc_free : &v_empty[j % kStages]);
       __syncwarp();
       if (j + 1 < nkv[1]) issue_s(1, k_addr);
-      if (next && lane == 0) tc_commit(k8(kFmt) ? kc_free : &k_empty[(j + 1) % kStages]);
+      if (next && lane == 0) tc_commit(quant(kFmt) ? kc_free : &k_empty[(j + 1) % kStages]);
       __syncwarp();
     }
     // every MMA this thread issued must finish before TMEM is released
@@ -779,8 +847,8 @@ __global__ void __launch_bounds__(Smem<D, kFmt>::kThreads, 1)
         // blocks of a rejected page; E4M3 K scales per 64-key block
         const int32_t key0 = j * kKeys;
         const bool diag = key0 + kKeys - 1 > p_min;
-        const float mul0 = k8(kFmt) ? p.scale_log2 * tf.ks[0] : p.scale_log2;
-        const float mul1 = k8(kFmt) ? p.scale_log2 * tf.ks[1] : p.scale_log2;
+        const float mul0 = quant(kFmt) ? p.scale_log2 * tf.ks[0] : p.scale_log2;
+        const float mul1 = quant(kFmt) ? p.scale_log2 * tf.ks[1] : p.scale_log2;
         auto scaled = [&](float v, int c) -> float {
           const bool keep = (!diag || key0 + c <= pos) && !((tf.bad >> (c >> 6)) & 1);
           return keep ? v * (c < 64 ? mul0 : mul1) : -INFINITY;
@@ -799,7 +867,7 @@ __global__ void __launch_bounds__(Smem<D, kFmt>::kThreads, 1)
         // waits for this tile's P.
         float alpha = 1.f;
         auto set_max = [&](float mt) -> float {
-          const bool need = mt > m_ref + (k8(kFmt) ? 0.f : 8.f);  // true on the first visible tile
+          const bool need = mt > m_ref + (quant(kFmt) ? 0.f : 8.f);  // true on the first visible tile
           const float m_new = need ? mt : m_ref;
           if (j >= 1 && need) alpha = fast_exp2(m_ref - m_new);
           m_ref = m_new;
@@ -836,7 +904,8 @@ __global__ void __launch_bounds__(Smem<D, kFmt>::kThreads, 1)
             tmem_ld32(tmem + lane_base + colS + cb + 32, sv + 32);
             tmem_wait_ld();
             const float mul = cb < 64 ? mul0 : mul1;
-            const float vsc = k8(kFmt) ? (cb < 64 ? tf.vs[0] : tf.vs[1]) : 1.f;  // E4M3 V scales ride on P
+            // quantised pools: the V scales ride on P
+            const float vsc = quant(kFmt) ? (cb < 64 ? tf.vs[0] : tf.vs[1]) : 1.f;
             uint32_t pk[32];
             // (two loops rather than a branch per element, which the compiler
             // would turn into both paths under predicates)
@@ -848,7 +917,7 @@ __global__ void __launch_bounds__(Smem<D, kFmt>::kThreads, 1)
                 const float p1 = fast_exp2(fmaf(sv[i + 1], mul, -m_use));
                 r0 += p0;
                 r1 += p1;
-                pk[i / 2] = k8(kFmt) ? pack_f16(p0 * vsc, p1 * vsc) : pack_bf16(p0, p1);
+                pk[i / 2] = quant(kFmt) ? pack_f16(p0 * vsc, p1 * vsc) : pack_bf16(p0, p1);
               }
               rs += r0 + r1;
             } else {
@@ -857,7 +926,7 @@ __global__ void __launch_bounds__(Smem<D, kFmt>::kThreads, 1)
                 const float p0 = fast_exp2(scaled(sv[i], cb + i) - m_use);
                 const float p1 = fast_exp2(scaled(sv[i + 1], cb + i + 1) - m_use);
                 rs += p0 + p1;
-                pk[i / 2] = k8(kFmt) ? pack_f16(p0 * vsc, p1 * vsc) : pack_bf16(p0, p1);
+                pk[i / 2] = quant(kFmt) ? pack_f16(p0 * vsc, p1 * vsc) : pack_bf16(p0, p1);
               }
             }
             // P column c/2 lies in an S column already read
@@ -977,18 +1046,24 @@ int prefill_entry(const pkv_cache* cache, const void* q, int32_t num_q_heads, in
   if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(out) & 15))
     return PKV_ERR_ALIGN;
   const int fmt = cache->kv_dtype;
-  const bool fp8 = k8(fmt);  // one-byte codes
   const int D = cache->head_dim;
   CUtensorMap tq, tk, tv;
   if ((st = encode_q_map(&tq, q, total_q, num_q_heads, D, gqa_group))) return st;
   const int64_t rows = (int64_t)cache->num_pages * cache->num_kv_heads * cache->page_size;
-  // bf16 pools: 64-column boxes; E4M3 pools: one box of the whole D-byte row
-  const int box_cols = fp8 ? D : 64;
-  if ((st = encode_pool_map(&tk, cache->k_pool, fp8, rows, D, box_cols, 64))) return st;
-  if ((st = encode_pool_map(&tv, cache->v_pool, fp8, rows, D, box_cols, 64))) return st;
+  // bf16 pools: 64-column boxes; quantised pools: one box of the whole row of
+  // codes (D bytes, or D/2 for FP4)
+  const bool bytes = quant(fmt);
+  const int row_elems = fp4(fmt) ? D / 2 : D;
+  const int box_cols = bytes ? row_elems : 64;
+  if ((st = encode_pool_map(&tk, cache->k_pool, bytes, rows, row_elems, box_cols, 64))) return st;
+  if ((st = encode_pool_map(&tv, cache->v_pool, bytes, rows, row_elems, box_cols, 64))) return st;
   pf::Params p;
   p.k_scale = cache->k_scale;
   p.v_scale = cache->v_scale;
+  p.k_blocks = fp4(fmt) ? static_cast<const uint8_t*>(cache->k_pool) + block_region_offset(cache)
+                        : nullptr;
+  p.v_blocks = fp4(fmt) ? static_cast<const uint8_t*>(cache->v_pool) + block_region_offset(cache)
+                        : nullptr;
   p.cu_q = cu_q_lens;
   p.page_table = page_table;
   p.seq_lens = seq_lens;
@@ -1009,11 +1084,13 @@ int prefill_entry(const pkv_cache* cache, const void* q, int32_t num_q_heads, in
   if ((int64_t)p.pair_slots * p.num_kv_heads * num_chunks > INT32_MAX) return PKV_ERR_SHAPE;
   cudaError_t e;
   if (D == 128)
-    e = fmt == PKV_KV_INT8       ? pf::launch<128, PKV_KV_INT8>(tq, tk, tv, p, stream)
+    e = fmt == PKV_KV_NVFP4      ? pf::launch<128, PKV_KV_NVFP4>(tq, tk, tv, p, stream)
+        : fmt == PKV_KV_INT8     ? pf::launch<128, PKV_KV_INT8>(tq, tk, tv, p, stream)
         : fmt == PKV_KV_FP8_E4M3 ? pf::launch<128, PKV_KV_FP8_E4M3>(tq, tk, tv, p, stream)
                                  : pf::launch<128, PKV_KV_BF16>(tq, tk, tv, p, stream);
   else
-    e = fmt == PKV_KV_INT8       ? pf::launch<64, PKV_KV_INT8>(tq, tk, tv, p, stream)
+    e = fmt == PKV_KV_NVFP4      ? pf::launch<64, PKV_KV_NVFP4>(tq, tk, tv, p, stream)
+        : fmt == PKV_KV_INT8     ? pf::launch<64, PKV_KV_INT8>(tq, tk, tv, p, stream)
         : fmt == PKV_KV_FP8_E4M3 ? pf::launch<64, PKV_KV_FP8_E4M3>(tq, tk, tv, p, stream)
                                  : pf::launch<64, PKV_KV_BF16>(tq, tk, tv, p, stream);
   return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;

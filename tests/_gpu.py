@@ -10,6 +10,9 @@ import workloads
 
 def sentinel_pool(w, device):
     shape = w.pool_shape()
+    if w.kv_dtype == "nvfp4":  # one flat buffer: codes, then block scales
+        return torch.full((w.pool_bytes(),), workloads.sentinel_byte(w.kv_dtype),
+                          dtype=torch.uint8, device=device)
     if w.kv_dtype != "bf16":
         return torch.full(shape, workloads.sentinel_byte(w.kv_dtype), dtype=torch.uint8,
                           device=device)
@@ -35,7 +38,8 @@ class GpuState:
                                       device=device)
             self.v_scale = torch.ones_like(self.k_scale)
         self.cache = pkv.PagedKVCache(self.k_pool, self.v_pool, w.kv_dtype, self.k_scale,
-                                      self.v_scale, self.flags)
+                                      self.v_scale, self.flags,
+                                      geometry=w.pool_shape() if w.kv_dtype == "nvfp4" else None)
         self.table = torch.from_numpy(w.page_table).to(device)
         self.k_new, self.v_new = [], []
         # Context, in groups of sequences, through the library's append.

@@ -19,6 +19,8 @@ benchmark shapes of this library:
                       P=64, 64/8, D=128, E4M3 K/V with per-(page, head) scale
 5. in-flight mixed    32 decode U[256,4096] + 4 chunks of 512 new tokens over
                       ctx U[0,2048], P=64, 32/8, D=128
+6, 7.                 config 4's batch with INT8, and with FP4 (E2M1 + E4M3
+                      block scales), K/V pools
 
 Recipe (identical for every config):
 * ``numpy.random.default_rng(seed)`` draws the context lengths first, then one
@@ -94,7 +96,7 @@ class Workload:
     num_q_heads: int
     num_kv_heads: int
     head_dim: int
-    kv_dtype: str  # "bf16", "e4m3", "int8" or "nvfp4" (oracle only so far)
+    kv_dtype: str  # "bf16", "e4m3", "int8" or "nvfp4"
     ctx_lens: np.ndarray  # int32 [B], tokens already cached
     new_lens: np.ndarray  # int32 [B], tokens appended this step
     num_pages: int
@@ -102,6 +104,7 @@ class Workload:
     decode_rows: np.ndarray  # int64 indices into [0, B)
     chunk_rows: np.ndarray  # int64 indices into [0, B)
     softmax_scale: float
+    config_number: Optional[int] = None  # set by config(n) for the numbered workloads
 
     # ------------------------------------------------------------ structure
     @property
@@ -339,6 +342,16 @@ def llama70b_int8_decode(seed: int = 3) -> Workload:
                  kv_dtype="int8", rng=rng)
 
 
+def llama70b_nvfp4_decode(seed: int = 3) -> Workload:
+    """The 70B-shaped decode batch of ``llama70b_fp8_decode`` with FP4 K/V pools
+    (E2M1 codes, E4M3 block scales per 16 values, per-(page, head) scale)."""
+    rng = np.random.default_rng(seed)
+    ctx = np.clip(np.rint(np.exp(rng.normal(math.log(1024.0), 0.8, size=256))), 1, 8191)
+    return build("llama3_70b_nvfp4_decode_b256_p64_gqa8_d128", seed, ctx.astype(np.int64),
+                 [1] * 256, page_size=64, num_q_heads=64, num_kv_heads=8, head_dim=128,
+                 kv_dtype="nvfp4", rng=rng)
+
+
 def mixed_inflight(seed: int = 4) -> Workload:
     """32 decode seqs U[256,4096] + 4 prefill chunks of 512 over context U[0,2048]."""
     rng = np.random.default_rng(seed)
@@ -358,12 +371,15 @@ CONFIGS = {
     4: llama70b_fp8_decode,
     5: mixed_inflight,
     6: llama70b_int8_decode,
+    7: llama70b_nvfp4_decode,
 }
 
 
 def config(n: int, seed: Optional[int] = None) -> Workload:
     fn = CONFIGS[n]
-    return fn() if seed is None else fn(seed)
+    w = fn() if seed is None else fn(seed)
+    w.config_number = n
+    return w
 
 
 def empty_pool(w: Workload) -> np.ndarray:
