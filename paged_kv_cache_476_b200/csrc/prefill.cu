@@ -176,6 +176,34 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
+// Two fp32 lanes at once (sm_100 packed FMA / add / mul): each lane rounds
+// exactly as its scalar instruction would.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  unsigned long long r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(r)
+      : "l"(*reinterpret_cast<unsigned long long*>(&a)),
+        "l"(*reinterpret_cast<unsigned long long*>(&b)),
+        "l"(*reinterpret_cast<unsigned long long*>(&c)));
+  return *reinterpret_cast<float2*>(&r);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  unsigned long long r;
+  asm("add.rn.f32x2 %0, %1, %2;"
+      : "=l"(r)
+      : "l"(*reinterpret_cast<unsigned long long*>(&a)),
+        "l"(*reinterpret_cast<unsigned long long*>(&b)));
+  return *reinterpret_cast<float2*>(&r);
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  unsigned long long r;
+  asm("mul.rn.f32x2 %0, %1, %2;"
+      : "=l"(r)
+      : "l"(*reinterpret_cast<unsigned long long*>(&a)),
+        "l"(*reinterpret_cast<unsigned long long*>(&b)));
+  return *reinterpret_cast<float2*>(&r);
+}
+
 // O row (this thread's TMEM lane, D fp32 columns from taddr) *= alpha.
 template <int D>
 __device__ __forceinline__ void rescale_o(uint32_t taddr, float alpha) {
@@ -829,13 +857,15 @@ __global__ void __launch_bounds__(Smem<D, kFmt>::kThreads, 1)
       const int r = wq * 32 + lane;  // row of the tile = TMEM lane
       const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
       const uint32_t colS = col_s(x), colO = col_o(x);
-      const int t_local = q0[x] + r / G;
+      const int nkx = x ? nkv[1] : nkv[0];
+      const int q0x = x ? q0[1] : q0[0];
+      const int t_local = q0x + r / G;
       const bool row_ok = t_local < n;
-      const int32_t p_min = L - n + q0[x];
-      const int32_t pos = row_ok ? L - n + t_local : L - n + min(q0[x] + TQ, n) - 1;
+      const int32_t p_min = L - n + q0x;
+      const int32_t pos = row_ok ? L - n + t_local : L - n + min(q0x + TQ, n) - 1;
       float m_ref = -INFINITY, l = 0.f;
       bool ok = true;
-      for (int j = 0; j < nkv[x]; ++j) {
+      for (int j = 0; j < nkx; ++j) {
         if (!mbar_wait(&s_full[x], (uint32_t)(j & 1), p.flags)) { ok = false; break; }
         if (!mbar_wait(&facts_full[j % kFactsRing], (uint32_t)((j / kFactsRing) & 1), p.flags)) {
           ok = false;
@@ -910,16 +940,22 @@ __global__ void __launch_bounds__(Smem<D, kFmt>::kThreads, 1)
             // (two loops rather than a branch per element, which the compiler
             // would turn into both paths under predicates)
             if (plain) {
-              float r0 = 0.f, r1 = 0.f;
+              float2 racc = make_float2(0.f, 0.f);
+              const float2 mul_2 = make_float2(mul, mul), neg_2 = make_float2(-m_use, -m_use);
+              const float2 vsc_2 = make_float2(vsc, vsc);
 #pragma unroll
               for (int i = 0; i < 64; i += 2) {
-                const float p0 = fast_exp2(fmaf(sv[i], mul, -m_use));
-                const float p1 = fast_exp2(fmaf(sv[i + 1], mul, -m_use));
-                r0 += p0;
-                r1 += p1;
-                pk[i / 2] = quant(kFmt) ? pack_f16(p0 * vsc, p1 * vsc) : pack_bf16(p0, p1);
+                const float2 t = fma2(make_float2(sv[i], sv[i + 1]), mul_2, neg_2);
+                const float2 pp = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+                racc = add2(racc, pp);
+                if constexpr (quant(kFmt)) {
+                  const float2 ps = mul2(pp, vsc_2);
+                  pk[i / 2] = pack_f16(ps.x, ps.y);
+                } else {
+                  pk[i / 2] = pack_bf16(pp.x, pp.y);
+                }
               }
-              rs += r0 + r1;
+              rs += racc.x + racc.y;
             } else {
 #pragma unroll
               for (int i = 0; i < 64; i += 2) {
@@ -942,8 +978,8 @@ __global__ void __launch_bounds__(Smem<D, kFmt>::kThreads, 1)
         if (lane == 0) mbar_arrive(&p_full[x]);
       }
       // ------------------------------------------------------ epilogue
-      if (ok && nkv[x] > 0 &&
-          mbar_wait(&o_bar[x], (uint32_t)((nkv[x] - 1) & 1), p.flags)) {
+      if (ok && nkx > 0 &&
+          mbar_wait(&o_bar[x], (uint32_t)((nkx - 1) & 1), p.flags)) {
         tc_fence_after();
         const float inv = l > 0.f ? 1.f / l : 0.f;
         const int64_t qrow = (int64_t)q_begin + t_local;
