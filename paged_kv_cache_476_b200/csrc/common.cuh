@@ -164,6 +164,19 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                : "r"(addr));
 }
 
+// Transposing load of two 16x16 matrices of bytes: lanes 0-15 give the row
+// addresses (16 bytes each) of the first, lanes 16-31 those of the second.
+// Thread (gid, tid4) receives in r0 the bytes of the first matrix's rows
+// 4*tid4 .. 4*tid4+3 (low byte first) in column gid, in r1 the same rows in
+// column gid + 8, and in r2, r3 the same of the second matrix (lane layout
+// checked on B200 with an in-bounds probe).
+__device__ __forceinline__ void ldsm_x2_t_b8(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                             uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m16n16.x2.trans.shared.b8 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
 // D = A(16x16, row) * B(16x8, col) + D with bf16 inputs and fp32 accumulate.
 __device__ __forceinline__ void mma_bf16(float* d, uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {

@@ -538,6 +538,12 @@ __global__ void __launch_bounds__(kThreads, 2)
   // quantised V loads order them (0-7, ce), (8-15, ce), (0-7, ce+1), (8-15, ce+1)
   const LaneTile ltk = lane_tile<Ly::kBoxRowB>(16 * warp + mrow + (mat >> 1) * 8, mat & 1);
   const LaneTile ltv = lane_tile<Ly::kBoxRowB>(16 * warp + mrow + (mat & 1) * 8, mat >> 1);
+  // one-byte V: the 8-bit transposing load takes 16 row addresses per
+  // 16x16 matrix (lanes 0-15: chunk ce, lanes 16-31: chunk ce + 1); row
+  // position 4i + e holds token 2i + (e & 1) + 8 (e >> 1) of the warp's 16,
+  // so that a thread's four rows are the A fragment's token columns (below)
+  const int vrow = 16 * warp + 2 * ((lane & 15) >> 2) + (lane & 1) + 8 * ((lane >> 1) & 1);
+  const LaneTile ltb = lane_tile<Ly::kBoxRowB>(vrow, lane >> 4);
 
   for (int64_t i = 0; i < n_tiles; ++i) {
     const int stage = (int)(i % kStages);
@@ -628,6 +634,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         // times the token's block scale (exact in f16), are the B fragments
         // of k-steps 2c (bytes 0, 1) and 2c+1 (bytes 2, 3).
         const uint8_t* ksc = tiles + stage * Ly::kStageB + 2 * Ly::kTileB;
+        float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         uint32_t sk[2][Ly::kScaleRowB / 4];  // block scales of tokens gid and gid+8
 #pragma unroll
         for (int n = 0; n < 2; ++n)
@@ -649,11 +656,17 @@ __global__ void __launch_bounds__(kThreads, 2)
             e2m1x8_to_f16x2(r[i], f);
 #pragma unroll
             for (int k = 0; k < 4; ++k) f[k] = hmul2_u32(f[k], sbh);
+            // two accumulation chains per n-tile (even / odd k-steps)
             mma_f16(s[n], qa[2 * cc][0], 0u, qa[2 * cc][1], 0u, f[0], f[1]);
-            mma_f16(s[n], qa[2 * cc + 1][0], 0u, qa[2 * cc + 1][1], 0u, f[2], f[3]);
+            mma_f16(s2[n], qa[2 * cc + 1][0], 0u, qa[2 * cc + 1][1], 0u, f[2], f[3]);
           }
         }
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s[n][e] += s2[n][e];
       } else {
+        float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
         for (int kp = 0; kp < KS / 2; ++kp) {
           // matrices: (tokens 0-7, chunk 2kp), (0-7, 2kp+1), (8-15, 2kp), (8-15, 2kp+1)
@@ -663,9 +676,15 @@ __global__ void __launch_bounds__(kThreads, 2)
           for (int i = 0; i < 4; ++i) {
             uint32_t lo, hi;
             kv8x4_to_f16x2<kFmt>(r[i], lo, hi);
-            mma_f16(s[i >> 1], qa[2 * kp + (i & 1)][0], 0u, qa[2 * kp + (i & 1)][1], 0u, lo, hi);
+            // two accumulation chains per n-tile (even / odd k-steps)
+            float* acc = (i & 1) ? s2[i >> 1] : s[i >> 1];
+            mma_f16(acc, qa[2 * kp + (i & 1)][0], 0u, qa[2 * kp + (i & 1)][1], 0u, lo, hi);
           }
         }
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s[n][e] += s2[n][e];
       }
       // ---- online softmax on row gid (log2 domain) ----
       const float mul = quant(kFmt) ? qk_mul * t_ks : qk_mul;
@@ -781,31 +800,24 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
           }
         } else {
-          // One-byte V codes straight from the landed tile.  A transposed
-          // load of 16-bit elements (byte pairs d, d+1) gives each thread,
-          // per 8x8 matrix, codes of tokens (2*tid4, 2*tid4+1) x bytes
-          // (2*gid, 2*gid+1) of a 16-byte chunk; two exact conversions and a
-          // swap of 16-bit halves make the A fragment of V^T with row gid = d
-          // 16m + 2*gid and row gid+8 = d 16m + 2*gid + 1 (the snapshot
-          // below undoes the order).
-          auto v_rows = [&](uint32_t codes, uint32_t& even_d, uint32_t& odd_d) {
-            uint32_t t0, t1;  // tokens 2*tid4 and 2*tid4+1
-            kv8x4_to_f16x2<kFmt>(codes, t0, t1);
-            even_d = __byte_perm(t0, t1, 0x5410);
-            odd_d = __byte_perm(t0, t1, 0x7632);
-          };
+          // One-byte V codes straight from the landed tile.  The transposing
+          // load of 8-bit elements gives the thread (gid, tid4), for byte
+          // column gid of a 16-byte chunk m (d = 16m + gid) and for column
+          // gid + 8, the codes of rows 4*tid4 .. 4*tid4+3, which the row order
+          // above makes tokens 2t, 2t+1, 2t+8, 2t+9 (t = tid4).  Two exact
+          // conversions per register then give the A fragment of V^T (rows
+          // d = 16m + gid and + 8, as in the bf16 path) with no byte shuffles.
 #pragma unroll
           for (int m = 0; m < D / 16; m += 2) {
-            // matrices: (tokens 0-7, chunk m), (8-15, m), (0-7, m+1), (8-15, m+1)
-            uint32_t r0, r1, r2, r3;
-            ldsm_x4_t(tile_at<Ly::kBoxRowB, kTile>(vbase, ltv, m), r0, r1, r2, r3);
-            uint32_t a0, a1, a2, a3;
-            v_rows(r0, a0, a1);
-            v_rows(r1, a2, a3);
-            mma_f16(ot[m], m0(a0), m0(a1), m1(a2), m1(a3), pa0, pa2);
-            v_rows(r2, a0, a1);
-            v_rows(r3, a2, a3);
-            mma_f16(ot[m + 1], m0(a0), m0(a1), m1(a2), m1(a3), pa0, pa2);
+            uint32_t r[4];  // chunk m: r[0] (column gid), r[1] (gid + 8); chunk m+1: r[2], r[3]
+            ldsm_x2_t_b8(tile_at<Ly::kBoxRowB, kTile>(vbase, ltb, m), r[0], r[1], r[2], r[3]);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              uint32_t a0, a1, a2, a3;
+              kv8x4_to_f16x2<kFmt>(r[2 * h], a0, a2);  // d = 16(m+h) + gid: tokens (2t, 2t+1), (2t+8, 2t+9)
+              kv8x4_to_f16x2<kFmt>(r[2 * h + 1], a1, a3);  // d = 16(m+h) + gid + 8
+              mma_f16(ot[m + h], m0(a0), m0(a1), m1(a2), m1(a3), pa0, pa2);
+            }
           }
         }
       };
@@ -830,14 +842,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       float* r0 = red_o + (warp * G + h0) * D;
       float* r1 = red_o + (warp * G + h1) * D;
       // fragment rows gid and gid+8 of d-tile m hold d 16m + gid and +8
-      // (bf16), 16m + 2*gid and +1 (one-byte codes), or 32(m/2) + 4*gid +
-      // 2(m%2) and +1 (FP4), as the PV products lay them out
-      const int d_step = quant(kFmt) ? 1 : 8;
+      // (bf16 and one-byte codes), or 32(m/2) + 4*gid + 2(m%2) and +1 (FP4),
+      // as the PV products lay them out
+      const int d_step = fp4(kFmt) ? 1 : 8;
 #pragma unroll
       for (int m = 0; m < D / 16; ++m) {
-        const int d = fp4(kFmt) ? 32 * (m >> 1) + 4 * gid + 2 * (m & 1)
-                     : k8(kFmt) ? 16 * m + 2 * gid
-                                : 16 * m + gid;
+        const int d = fp4(kFmt) ? 32 * (m >> 1) + 4 * gid + 2 * (m & 1) : 16 * m + gid;
         if (h0 < G) {
           r0[d] = ot[m][0];
           r0[d + d_step] = ot[m][2];
