@@ -197,6 +197,19 @@ __device__ __forceinline__ void mma_f16(float* d, uint32_t a0, uint32_t a1, uint
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// D = A(16x32, row) * B(32x8, col) + D with signed 8-bit operands and exact
+// s32 accumulate, rows 8-15 of A zero.  a0 / a2: a thread's four A bytes at
+// columns 4*tid4 + {0..3} and + 16 of row gid; b0 / b1: its four B bytes at
+// rows 4*tid4 + {0..3} and + 16 of column gid (low byte first).
+__device__ __forceinline__ void mma_s8(int32_t* d, uint32_t a0, uint32_t a2, uint32_t b0,
+                                       uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
 // ------------------------------------------------------------------ packing
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half)

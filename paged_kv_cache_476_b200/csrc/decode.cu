@@ -185,22 +185,22 @@ __device__ __forceinline__ void append_newest(const DecodeParams& p, int b, int 
       *reinterpret_cast<uint2*>((is_v ? p.v_pool : p.k_pool) + row * (D / 2) + blk * 8) = codes;
       (is_v ? p.v_blocks_w : p.k_blocks_w)[row * (D / 16) + blk] = static_cast<uint8_t>(sb);
     }
-    return;
-  }
-  for (int e = lane * 4; e < D; e += 128) {
-    const uint2 kx = *reinterpret_cast<const uint2*>(p.k_new + src + e);
-    const uint2 vx = *reinterpret_cast<const uint2*>(p.v_new + src + e);
-    if constexpr (!k8(kFmt)) {
-      *reinterpret_cast<uint2*>(p.k_pool + (dst + e) * 2) = kx;
-      *reinterpret_cast<uint2*>(p.v_pool + (dst + e) * 2) = vx;
-    } else {
-      auto codes = [](uint2 x, float s) -> uint32_t {
-        const uint32_t lo = encode8x2<kFmt>(*reinterpret_cast<const __nv_bfloat162*>(&x.x), s);
-        const uint32_t hi = encode8x2<kFmt>(*reinterpret_cast<const __nv_bfloat162*>(&x.y), s);
-        return lo | (hi << 16);
-      };
-      *reinterpret_cast<uint32_t*>(p.k_pool + dst + e) = codes(kx, ks);
-      *reinterpret_cast<uint32_t*>(p.v_pool + dst + e) = codes(vx, vs);
+  } else {
+    for (int e = lane * 4; e < D; e += 128) {
+      const uint2 kx = *reinterpret_cast<const uint2*>(p.k_new + src + e);
+      const uint2 vx = *reinterpret_cast<const uint2*>(p.v_new + src + e);
+      if constexpr (!k8(kFmt)) {
+        *reinterpret_cast<uint2*>(p.k_pool + (dst + e) * 2) = kx;
+        *reinterpret_cast<uint2*>(p.v_pool + (dst + e) * 2) = vx;
+      } else {
+        auto codes = [](uint2 x, float s) -> uint32_t {
+          const uint32_t lo = encode8x2<kFmt>(*reinterpret_cast<const __nv_bfloat162*>(&x.x), s);
+          const uint32_t hi = encode8x2<kFmt>(*reinterpret_cast<const __nv_bfloat162*>(&x.y), s);
+          return lo | (hi << 16);
+        };
+        *reinterpret_cast<uint32_t*>(p.k_pool + dst + e) = codes(kx, ks);
+        *reinterpret_cast<uint32_t*>(p.v_pool + dst + e) = codes(vx, vs);
+      }
     }
   }
 }
@@ -570,13 +570,15 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         qk_mul = p.scale_log2;
       } else {
-        // f16 Q with a per-row power-of-two prescale, in the d order of the
-        // K codes that ldmatrix delivers.  One-byte codes: inside each
-        // 16-wide d block, the fragment's k pair (2*tid4, +1) holds d =
-        // 4*tid4 + {0,1} and the pair (2*tid4+8, +9) holds d = 4*tid4 + {2,3}.
-        // FP4: a 16-byte chunk c holds d = 32c..32c+31 and a thread's 4 bytes
-        // are d = 32c + 8*tid4 + {0..7}; k-step 2c takes the first four of
-        // them, k-step 2c+1 the last four.
+        // Q with a per-row power-of-two prescale, in the d order of the K
+        // codes that ldmatrix delivers: qv[kk] holds d = 16kk + 4*tid4 +
+        // {0..3} for one-byte codes.  E4M3 uses f16 Q against converted codes.
+        // INT8 feeds the s8 MMA (k = 32), which takes from a thread the bytes
+        // d = 32kp + 4*tid4 + {0..3} and + 16 of one row, that is qv[2kp] and
+        // qv[2kp+1], with Q split into two 8-bit operands (qa[kk][0] high,
+        // [1] low).  FP4 (f16 Q): a 16-byte chunk c holds d = 32c..32c+31 and
+        // a thread's 4 bytes are d = 32c + 8*tid4 + {0..7}; k-step 2c takes
+        // the first four of them, k-step 2c+1 the last four.
         float amax = 0.f;
         float qv[KS][4];
 #pragma unroll
@@ -591,17 +593,40 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        // power-of-two prescale putting amax in [2^(top-1), 2^top): 2^14 for
+        // f16 Q, 2^13 for the INT8 split
+        constexpr int kTop = kFmt == PKV_KV_INT8 ? 13 : 14;
         int ex = 0;
         if (amax > 0.f) {
           frexpf(amax, &ex);  // amax < 2^ex
-          ex = 14 - ex;       // amax * 2^ex < 2^14
+          ex = kTop - ex;     // amax * 2^ex < 2^kTop
           ex = max(-100, min(100, ex));
         }
         const float pre = ldexpf(1.f, ex);
+        if constexpr (kFmt == PKV_KV_INT8) {
+          // 13-bit fixed point q = round(x * pre), split as q = 128 hi + lo
+          // with hi in [-64, 64] and lo in [0, 127]: two s8 operands whose s32
+          // products with the codes are exact
 #pragma unroll
-        for (int kk = 0; kk < KS; ++kk) {
-          qa[kk][0] = pack_f16(qv[kk][0] * pre, qv[kk][1] * pre);
-          qa[kk][1] = pack_f16(qv[kk][2] * pre, qv[kk][3] * pre);
+          for (int kk = 0; kk < KS; ++kk) {
+            uint32_t hi = 0, lo = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int qf = __float2int_rn(qv[kk][e] * pre);
+              hi |= ((uint32_t)(qf >> 7) & 0xffu) << (8 * e);
+              lo |= ((uint32_t)qf & 0x7fu) << (8 * e);
+            }
+            qa[kk][0] = hi;
+            qa[kk][1] = lo;
+          }
+        } else {
+          // f16: for E4M3 the fragment's k pair (2*tid4, +1) holds d = 16kk +
+          // 4*tid4 + {0,1} and the pair (2*tid4+8, +9) holds + {2,3}
+#pragma unroll
+          for (int kk = 0; kk < KS; ++kk) {
+            qa[kk][0] = pack_f16(qv[kk][0] * pre, qv[kk][1] * pre);
+            qa[kk][1] = pack_f16(qv[kk][2] * pre, qv[kk][3] * pre);
+          }
         }
         qk_mul = p.scale_log2 * ldexpf(1.f, -ex);
       }
@@ -665,7 +690,28 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int n = 0; n < 2; ++n)
 #pragma unroll
           for (int e = 0; e < 4; ++e) s[n][e] += s2[n][e];
+      } else if constexpr (kFmt == PKV_KV_INT8) {
+        // INT8 codes feed the s8 MMA (k = 32) as they land: the matrices
+        // (tokens 0-7 | 8-15, chunk 2kp | 2kp+1) are the B fragments of the
+        // two n-tiles; products with the split Q are exact in s32, and
+        // S = 128 hi + lo.
+        int32_t sh[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}}, sl[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+#pragma unroll
+        for (int kp = 0; kp < KS / 2; ++kp) {
+          uint32_t r[4];
+          ldsm_x4(tile_at<Ly::kBoxRowB, kTile>(kbase, ltk, 2 * kp), r[0], r[1], r[2], r[3]);
+#pragma unroll
+          for (int n = 0; n < 2; ++n) {
+            mma_s8(sh[n], qa[2 * kp][0], qa[2 * kp + 1][0], r[2 * n], r[2 * n + 1]);
+            mma_s8(sl[n], qa[2 * kp][1], qa[2 * kp + 1][1], r[2 * n], r[2 * n + 1]);
+          }
+        }
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s[n][e] = (float)(sh[n][e] * 128 + sl[n][e]);
       } else {
+        // E4M3 codes convert exactly to f16 after ldmatrix, four per call
         float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
         for (int kp = 0; kp < KS / 2; ++kp) {
