@@ -115,6 +115,8 @@ PREFILL_SOURCES = ("prefill.cu", "common.cuh", "kernels.h")
 TRAFFIC_PROFILES = {
     2: ("decode", "decode_kernel_llama8b_decode.md", DECODE_SOURCES),
     4: ("decode", "decode_kernel_llama70b_e4m3.md", DECODE_SOURCES),
+    6: ("decode", "decode_kernel_llama70b_int8.md", DECODE_SOURCES),
+    7: ("decode", "decode_kernel_llama70b_nvfp4.md", DECODE_SOURCES),
 }
 
 
@@ -142,8 +144,8 @@ def decode_roofline(dec_s, dec_bytes, hbm_peak, peak_kind, traffic=None):
         "frac": round(achieved / hbm_peak, 4),
         "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth, burst)",
         "traffic": traffic,
-        "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of "
-                          "decode_kernel + decode_merge_kernel (profiles/), null if stale",
+        "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one "
+                          "decode_kernel launch (profiles/), null if the sources changed",
         "algorithmic_bytes_per_launch": int(dec_bytes),
     }
 
