@@ -7,27 +7,29 @@
 //
 // Design (B200-first, HBM-bound):
 //  * Work list.  Each (sequence, kv head) pair is a unit; a unit's tokens are
-//    cut into 64-token tiles.  The units' tiles, concatenated in (b, g) order,
-//    are split into C equal contiguous ranges, one per CTA, with C = SMs x
-//    resident CTAs per SM: one persistent wave, no tail of unequal splits.
+//    cut into tiles (64 tokens for bf16 and FP4 pools, 128 for one-byte
+//    codes, so that a tile is 32 KB of K and V in either case).  The units'
+//    tiles, concatenated in (b, g) order, are split into C equal contiguous
+//    ranges, one per CTA, with C = SMs x resident CTAs per SM: one
+//    persistent wave, no tail of unequal splits.
 //  * A range cuts a unit into segments.  A segment computes an online-softmax
 //    partial (m, l, unnormalised o) for the unit's G = Hq/Hkv q heads.  A
 //    segment that covers its whole unit writes the output directly; otherwise
 //    it stores its partial, and a small merge kernel (a programmatic
 //    dependent launch, one warp per unit) combines the pieces afterwards.
 //  * Warp roles: one producer warp walks the range and issues TMA loads of
-//    the K and V tile (page-table indirected, 128-byte swizzled) into a
-//    multi-stage mbarrier ring, plus a bulk copy of Q at each segment start;
-//    four consumer warps each take 16 of a tile's 64 tokens and run
-//    S = Q K^T and O^T += V^T P^T on mma.sync (bf16, or f16 for E4M3 K/V
-//    which converts exactly), with the online softmax in registers; a flush
-//    warp turns the consumers' per-warp snapshots at each segment end into
-//    the output or a split partial while the consumers stream on.
-//  * One-byte K/V (E4M3, INT8): K codes are converted to f16 in registers
-//    after ldmatrix (the d order inside each 16-wide block is permuted
-//    identically in Q); V codes go from a transposed ldmatrix of byte pairs
-//    straight into the f16 A fragments of V^T.  The per-(page, head) scales
-//    fold into the scores (K) and into P (V).
+//    the K and V tile (page-table indirected, one 64-row box per page and
+//    box column, swizzled) into a multi-stage mbarrier ring, plus a bulk copy
+//    of Q at each segment start; four consumer warps each take a quarter of
+//    the tile's tokens and run S = Q K^T and O^T += V^T P^T on mma.sync, with
+//    the online softmax in registers; a flush warp turns the consumers'
+//    snapshots at each segment end into the output or a split partial while
+//    the consumers stream on.
+//  * Quantised K/V: INT8 K codes feed the s8 MMA (k = 32) as they land,
+//    against a two-term fixed-point Q; E4M3 K and all V codes convert
+//    exactly to f16 in registers after ldmatrix (FP4 times its E4M3 block
+//    scales).  The per-(page, head) scales fold into the scores (K) and
+//    into P (V).
 //  * Every wait is bounded; a bad page id or length is skipped and flagged.
 #include <type_traits>
 
@@ -36,12 +38,12 @@
 
 namespace pkv {
 
-constexpr int kTile = 64;           // tokens per pipeline tile
-constexpr int kConsumerWarps = 4;   // 16 tokens of each tile per warp
+constexpr int kConsumerWarps = 4;
 constexpr int kProducerWarp = kConsumerWarps;
 constexpr int kFlushWarp = kConsumerWarps + 1;
 constexpr int kThreads = (kConsumerWarps + 2) * 32;
 constexpr int kMaxGroup = 8;
+constexpr int kBoxRows = 64;   // rows of one TMA box; a tile is one or two of them
 // Suspend hints (ns) of the waits: the flush warp idles for long stretches.
 #ifndef PKV_FLUSH_SLEEP_NS
 #define PKV_FLUSH_SLEEP_NS 20000
@@ -54,7 +56,7 @@ constexpr int kMaxGroup = 8;
 constexpr int kSegFirst = 1;   // first tile of a segment: reset state, Q in this stage
 constexpr int kSegLast = 2;    // last tile of a segment: flush after it
 constexpr int kUnitWhole = 4;  // the segment is the whole unit: write out directly
-constexpr int kBadTile = 8;    // page id invalid: tile skipped
+constexpr int kBadHalf = 8;    // kBadHalf << h: the page of 64-row half h is invalid, skipped
 
 
 struct TileInfo {
@@ -63,7 +65,7 @@ struct TileInfo {
   int32_t slot;      // partial slot of this CTA's segment
   int32_t seg_base;  // first partial slot of the unit
   int32_t nseg;      // segments of the unit
-  float ks, vs;      // E4M3 scales of the tile's page
+  float ks[2], vs[2];  // scales of the pages of the tile's 64-row halves
 };
 
 // What the consumers hand to the flush warp at the end of a segment.
@@ -73,27 +75,38 @@ struct FlushDesc {
 
 template <int D, int kFmt>
 struct Layout {
+  // One-byte codes: 128-token tiles, 32 tokens per consumer warp, so that a
+  // stage carries as many bytes as a bf16 one and a warp's work per barrier
+  // doubles.  bf16 and FP4: 64-token tiles, 16 tokens per warp.
+  static constexpr bool kWide = k8(kFmt);
+  static constexpr int kTile = kWide ? 128 : 64;
+  static constexpr int kHalves = kTile / kBoxRows;  // 64-row boxes (pages) per tile
+  static constexpr int kWarpTok = kTile / kConsumerWarps;
   static constexpr int kMapEB = kFmt == PKV_KV_BF16 ? 2 : 1;   // element bytes of the TMA map
   static constexpr int kRowB = row_code_bytes(kFmt, D);        // code bytes of a token row
   static constexpr int kBoxRowB = kRowB >= 128 ? 128 : kRowB;  // TMA box inner bytes
   static constexpr int kNumBox = kRowB / kBoxRowB;             // boxes per tile row
-  static constexpr int kBoxB = kTile * kBoxRowB;
+  static constexpr int kBoxB = kTile * kBoxRowB;               // one box column of the tile
   static constexpr int kTileB = kNumBox * kBoxB;  // codes of one K (or V) tile
   // FP4: the E4M3 block scales of a tile's rows, after the two code tiles
   static constexpr int kScaleRowB = row_scale_bytes(kFmt, D);
   static constexpr int kScaleB = kTile * kScaleRowB;
   static constexpr int kStageB = 2 * kTileB + 2 * kScaleB;
+  // bytes of one 64-row half of a stage (K and V, codes and block scales)
+  static constexpr int kHalfTx = 2 * kNumBox * kBoxRows * kBoxRowB + 2 * kBoxRows * kScaleRowB;
 };
 
 // Shared-memory carve-up; the Q slices and the reduction buffers are sized
-// by the GQA group so that two CTAs fit on one SM.
+// by the GQA group so that two CTAs fit on one SM.  kSnap snapshot slots:
+// one per consumer warp (4), or one per warp pair (2) where that buys a
+// deeper ring.
 struct SmemPlan {
   uint32_t q, red_o, red_m, red_l, bars, info, misc, total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
-template <int D, int kFmt, int kStages>
+template <int D, int kFmt, int kStages, int kSnap>
 __host__ __device__ inline SmemPlan smem_plan(int G) {
   using Ly = Layout<D, kFmt>;
   SmemPlan s;
@@ -102,14 +115,14 @@ __host__ __device__ inline SmemPlan smem_plan(int G) {
   o += kStages * align_up(G * D * 2, 128);
   o = align_up(o, 1024);
   s.red_o = o;
-  o += kConsumerWarps * G * D * 4;
+  o += kSnap * G * D * 4;
   s.red_m = o;
-  o += kConsumerWarps * G * 4;
+  o += kSnap * G * 4;
   s.red_l = o;
-  o += kConsumerWarps * G * 4;
+  o += kSnap * G * 4;
   o = align_up(o, 8);
   s.bars = o;
-  o += (2 * kStages + 2) * 8;
+  o += (2 * kStages + 3) * 8;
   s.info = o;
   o += kStages * sizeof(TileInfo) + sizeof(FlushDesc);
   s.misc = o;
@@ -126,7 +139,9 @@ __host__ __device__ inline SmemPlan smem_plan(int G) {
 // known at compile time.  A lane reads chunk ce + lo of row `row` for even
 // chunks ce; with xk the row bits the swizzle XORs into the chunk index,
 // (ce + lo) ^ xk = (ce ^ (xk & ~1)) + (lo ^ (xk & 1)), so the address is
-// base + box(ce) + a + ((ce % chunks-per-box) * 16 ^ x).
+// base + box(ce) + a + ((ce % chunks-per-box) * 16 ^ x).  Rows 16 apart share
+// the swizzle phase, so a lane tile moved by 16 rows is the base moved by
+// 16 * kBoxRowB bytes.
 struct LaneTile {
   uint32_t a;  // row * box row bytes + 16 * (lo ^ (xk & 1))
   uint32_t x;  // 16 * (xk & ~1)
@@ -153,6 +168,7 @@ __device__ __forceinline__ int64_t cta_of(int64_t x, int64_t C, int64_t T) {
   return ((x + 1) * C - 1) / T;
 }
 
+template <int kTile>
 __device__ __forceinline__ int tiles_of(int32_t len) { return (len + kTile - 1) / kTile; }
 
 __device__ __forceinline__ int32_t clamp_len(const DecodeParams& p, int32_t len, bool report) {
@@ -205,17 +221,18 @@ __device__ __forceinline__ void append_newest(const DecodeParams& p, int b, int 
   }
 }
 
-template <int D, int kFmt, int kStages>
+template <int D, int kFmt, int kStages, int kSnap>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
   using Ly = Layout<D, kFmt>;
+  constexpr int kTile = Ly::kTile;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte align the dynamic window (the swizzle pattern needs it).
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int G = p.group;
-  const SmemPlan sp = smem_plan<D, kFmt, kStages>(G);
+  const SmemPlan sp = smem_plan<D, kFmt, kStages, kSnap>(G);
   const uint32_t kQStride = align_up(G * D * 2, 128);
   uint8_t* tiles = smem;
   uint8_t* qbuf = smem + sp.q;
@@ -224,8 +241,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   float* red_l = reinterpret_cast<float*>(smem + sp.red_l);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + sp.bars);
   uint64_t* empty = full + kStages;
-  uint64_t* red_full = empty + kStages;   // consumers -> flush warp: a snapshot is ready
-  uint64_t* red_empty = red_full + 1;     // flush warp -> consumers: snapshot consumed
+  uint64_t* red_full = empty + kStages;   // consumers -> flush warp: the kSnap snapshots are ready
+  uint64_t* red_empty = red_full + 1;     // flush warp -> consumers: snapshots consumed
+  uint64_t* pair_full = red_empty + 1;    // (kSnap 2) warps 2, 3 -> warps 0, 1: written
   TileInfo* info = reinterpret_cast<TileInfo*>(smem + sp.info);
   FlushDesc* desc = reinterpret_cast<FlushDesc*>(info + kStages);
   int32_t* s_misc = reinterpret_cast<int32_t*>(smem + sp.misc);  // [0]=n tiles, [1]=is_last
@@ -244,8 +262,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kConsumerWarps);
     }
-    mbar_init(red_full, kConsumerWarps);
+    mbar_init(red_full, kSnap);
     mbar_init(red_empty, 1);
+    if (kSnap < kConsumerWarps) mbar_init(pair_full, kConsumerWarps - kSnap);
     fence_barrier_init();
   }
 
@@ -258,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     int64_t tot = 0;
     for (int base = 0; base < p.batch; base += 32) {
       const int b = base + lane;
-      const int t = b < p.batch ? tiles_of(clamp_len(p, __ldg(p.seq_lens + b), c == 0)) : 0;
+      const int t = b < p.batch ? tiles_of<kTile>(clamp_len(p, __ldg(p.seq_lens + b), c == 0)) : 0;
       tot += t;
     }
 #pragma unroll
@@ -286,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       int64_t run = 0;
       for (int base = 0; base < p.batch; base += 32) {
         const int b = base + lane;
-        const int t = b < p.batch ? tiles_of(clamp_len(p, __ldg(p.seq_lens + b), false)) : 0;
+        const int t = b < p.batch ? tiles_of<kTile>(clamp_len(p, __ldg(p.seq_lens + b), false)) : 0;
         int incl = t;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -317,21 +336,20 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   if (warp == kFlushWarp) {
     // ---------------------------------------------------------- flush warp
-    // Turns each segment's per-warp snapshots into the output (whole unit)
-    // or a split partial, then settles the unit's counter and, as the last
-    // segment of a unit, merges its partials.  All of it overlaps the
-    // consumers, which keep streaming the next segment.
+    // Turns each segment's kSnap snapshots into the output (whole unit) or a
+    // split partial.  It overlaps the consumers, which keep streaming the
+    // next segment.
     for (int k = 0;; ++k) {
       if (!mbar_wait(red_full, (uint32_t)(k & 1), p.flags, PKV_FLUSH_SLEEP_NS)) return;
       const FlushDesc fd = *desc;
       for (int r = 0; r < G; ++r) {
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red_m[w * G + r]);
-        float sc[kConsumerWarps];
+        for (int w = 0; w < kSnap; ++w) M = fmaxf(M, red_m[w * G + r]);
+        float sc[kSnap];
         float den = 0.f;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
+        for (int w = 0; w < kSnap; ++w) {
           const float mw = red_m[w * G + r];
           sc[w] = (M == -INFINITY || mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
           den += sc[w] * red_l[w * G + r];
@@ -341,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int d = lane; d < D; d += 32) {
           float num = 0.f;
 #pragma unroll
-          for (int w = 0; w < kConsumerWarps; ++w) num += sc[w] * red_o[(w * G + r) * D + d];
+          for (int w = 0; w < kSnap; ++w) num += sc[w] * red_o[(w * G + r) * D + d];
           if (fd.whole)
             p.out[orow * D + d] = __float2bfloat16(num * inv);
           else
@@ -368,36 +386,36 @@ __global__ void __launch_bounds__(kThreads, 2)
       tma_prefetch_desc(&tmap_k);
       tma_prefetch_desc(&tmap_v);
     }
-    const int tiles_per_page = p.page_size / kTile;
+    const int P = p.page_size;
     int b = pb, g = pg, t = pt;
     int len = clamp_len(p, __ldg(p.seq_lens + b), false);
-    int ntile = tiles_of(len);
+    int ntile = tiles_of<kTile>(len);
     int seg_first_t = t;
-    // page ids (and E4M3 scales) of 32 consecutive pages, one per lane
+    // page ids (and scales) of 32 consecutive pages, one per lane
     int cache_key = -1, cache_j0 = 0;
     int my_pid = 0;
     float my_ks = 1.f, my_vs = 1.f;
     int64_t x = range_start;  // global tile index
     int u_seg_base = 0, u_nseg = 1, u_slot = 0;
     int issued = 0;
-    bool ok = true;
     for (int64_t i = 0; i < n_tiles; ++i, ++x) {
       const int stage = (int)(i % kStages);
       if (i >= kStages) {
         if (!mbar_wait(&empty[stage], (uint32_t)((i / kStages - 1) & 1), p.flags,
-                       PKV_PIPE_SLEEP_NS)) {
-          ok = false;
+                       PKV_PIPE_SLEEP_NS))
           break;
-        }
       }
-      const int j = t / tiles_per_page;
-      const int sub = t - j * tiles_per_page;
-      const int pages_b = (len + p.page_size - 1) / p.page_size;
+      // A tile is kTile tokens from tok0, in 64-row halves; page sizes are
+      // multiples of 64, so each half lies in one page.
+      const int tok0 = t * kTile;
+      const int pages_b = (len + P - 1) / P;
+      const int j_first = tok0 / P;
+      const int j_last = min((tok0 + kTile - 1) / P, pages_b - 1);
       const int key = quant(kFmt) ? b * Hkv + g : b;
-      if (cache_key != key || j < cache_j0 || j >= cache_j0 + 32) {
+      if (cache_key != key || j_first < cache_j0 || j_last >= cache_j0 + 32) {
         cache_key = key;
-        cache_j0 = j;
-        const int jj = j + lane;
+        cache_j0 = j_first;
+        const int jj = j_first + lane;
         my_pid = jj < pages_b ? __ldg(p.page_table + (int64_t)b * p.max_pages + jj) : 0;
         if constexpr (quant(kFmt)) {
           if (jj < pages_b && my_pid >= 0 && my_pid < p.num_pages) {
@@ -406,32 +424,47 @@ __global__ void __launch_bounds__(kThreads, 2)
           }
         }
       }
-      int pid = __shfl_sync(0xffffffffu, my_pid, j - cache_j0);
-      const bool page_ok = pid >= 0 && pid < p.num_pages;
-      float ks = 1.f, vs = 1.f;
-      if constexpr (quant(kFmt)) {
-        ks = __shfl_sync(0xffffffffu, my_ks, j - cache_j0);
-        vs = __shfl_sync(0xffffffffu, my_vs, j - cache_j0);
-      }
-      bool bad = pid < 0 || pid >= p.num_pages;
-      if constexpr (quant(kFmt)) {
-        if (!bad && !(ks > 0.f && ks <= 32768.f && vs > 0.f && vs <= 32768.f)) {
-          bad = true;
-          if (lane == 0) flag_error(p.flags, PKV_FLAG_BAD_SCALE);
+      int hpid[Ly::kHalves], hrow[Ly::kHalves], hflags = 0;
+      bool hhas[Ly::kHalves];
+      float hks[2] = {1.f, 1.f}, hvs[2] = {1.f, 1.f};
+#pragma unroll
+      for (int h = 0; h < Ly::kHalves; ++h) {
+        const int tokh = tok0 + kBoxRows * h;
+        hhas[h] = tokh < len;  // half 0 always: t < ntile
+        const int jh = min(tokh / P, pages_b - 1);
+        hrow[h] = tokh - (tokh / P) * P;
+        int pid = __shfl_sync(0xffffffffu, my_pid, jh - cache_j0);
+        if constexpr (quant(kFmt)) {
+          hks[h] = __shfl_sync(0xffffffffu, my_ks, jh - cache_j0);
+          hvs[h] = __shfl_sync(0xffffffffu, my_vs, jh - cache_j0);
         }
+        bool bad = pid < 0 || pid >= p.num_pages;
+        if (bad && hhas[h] && lane == 0) flag_error(p.flags, PKV_FLAG_BAD_PAGE);
+        if constexpr (quant(kFmt)) {
+          if (!bad && !(hks[h] > 0.f && hks[h] <= 32768.f && hvs[h] > 0.f && hvs[h] <= 32768.f)) {
+            bad = true;
+            if (hhas[h] && lane == 0) flag_error(p.flags, PKV_FLAG_BAD_SCALE);
+          }
+        }
+        if (bad) {
+          pid = 0;
+          hflags |= kBadHalf << h;
+        }
+        hpid[h] = pid;
       }
-      if (pid < 0 || pid >= p.num_pages) {
-        if (lane == 0) flag_error(p.flags, PKV_FLAG_BAD_PAGE);
-      }
-      if (bad) pid = 0;
       // Fused append: this CTA is the one that reads the tile holding the
       // sequence's newest token (position len - 1), so it stores the token
       // first (as paged_kv_append would: whenever the page id is valid) and
       // orders those generic-proxy stores before its own bulk-tensor loads.
-      if (p.k_new && t == ntile - 1 && page_ok && __ldg(p.seq_lens + b) == len) {
-        append_newest<D, kFmt>(p, b, g, __shfl_sync(0xffffffffu, my_pid, j - cache_j0),
-                               (len - 1) % p.page_size, ks, vs, lane);
-        asm volatile("fence.proxy.async.global;" ::: "memory");
+      if (p.k_new && t == ntile - 1 && __ldg(p.seq_lens + b) == len) {
+        const int jn = (len - 1) / P;
+        const int pid_n = __shfl_sync(0xffffffffu, my_pid, jn - cache_j0);
+        if (pid_n >= 0 && pid_n < p.num_pages) {
+          const int hn = (len - 1 - tok0) / kBoxRows;  // the half holding it (same page)
+          append_newest<D, kFmt>(p, b, g, pid_n, (len - 1) % P, hn ? hks[1] : hks[0],
+                                 hn ? hvs[1] : hvs[0], lane);
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+        }
         __syncwarp();
       }
       const bool first = (i == 0) || (t == 0);
@@ -442,8 +475,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         ti.b = b;
         ti.g = g;
         ti.tile = t;
-        ti.valid = min(kTile, len - t * kTile);
-        ti.flags = (first ? kSegFirst : 0) | (last ? kSegLast : 0) | (bad ? kBadTile : 0);
+        ti.valid = min(kTile, len - tok0);
+        ti.flags = (first ? kSegFirst : 0) | (last ? kSegLast : 0) | hflags;
         if (last && seg_first_t == 0 && t == ntile - 1) ti.flags |= kUnitWhole;
         if (first) {
           // once per unit: which CTAs share it, hence its partial slots
@@ -461,27 +494,40 @@ __global__ void __launch_bounds__(kThreads, 2)
         ti.seg_base = u_seg_base;
         ti.nseg = u_nseg;
         ti.slot = u_slot;
-        ti.ks = ks;
-        ti.vs = vs;
+        ti.ks[0] = hks[0];
+        ti.vs[0] = hvs[0];
+        ti.ks[1] = hks[1];
+        ti.vs[1] = hvs[1];
         info[stage] = ti;
         const uint32_t qbytes = first ? (uint32_t)(G * D * 2) : 0u;
-        mbar_arrive_expect_tx(&full[stage], (uint32_t)Ly::kStageB + qbytes);
-        const int32_t y = (int32_t)(((int64_t)pid * Hkv + g) * p.page_size + sub * kTile);
+        uint32_t tx = qbytes;
+#pragma unroll
+        for (int h = 0; h < Ly::kHalves; ++h)
+          if (hhas[h]) tx += Ly::kHalfTx;
+        mbar_arrive_expect_tx(&full[stage], tx);
         uint8_t* kdst = tiles + stage * Ly::kStageB;
         uint8_t* vdst = kdst + Ly::kTileB;
 #pragma unroll
-        for (int bx = 0; bx < Ly::kNumBox; ++bx) {
-          const int32_t xc = bx * (Ly::kBoxRowB / Ly::kMapEB);
-          tma_load_2d(kdst + bx * Ly::kBoxB, &tmap_k, xc, y, &full[stage], pol);
-          tma_load_2d(vdst + bx * Ly::kBoxB, &tmap_v, xc, y, &full[stage], pol);
-        }
-        if constexpr (fp4(kFmt)) {
-          // the tile's block scales: kTile consecutive rows of the
-          // block-scale region, one contiguous run of kScaleB bytes
-          const int64_t soff = (int64_t)y * Ly::kScaleRowB;
-          bulk_load(vdst + Ly::kTileB, p.k_blocks + soff, Ly::kScaleB, &full[stage]);
-          bulk_load(vdst + Ly::kTileB + Ly::kScaleB, p.v_blocks + soff, Ly::kScaleB,
-                    &full[stage]);
+        for (int h = 0; h < Ly::kHalves; ++h) {
+          if (!hhas[h]) continue;
+          const int32_t y = (int32_t)(((int64_t)hpid[h] * Hkv + g) * P + hrow[h]);
+          const int hoff = h * kBoxRows * Ly::kBoxRowB;
+#pragma unroll
+          for (int bx = 0; bx < Ly::kNumBox; ++bx) {
+            const int32_t xc = bx * (Ly::kBoxRowB / Ly::kMapEB);
+            tma_load_2d(kdst + bx * Ly::kBoxB + hoff, &tmap_k, xc, y, &full[stage], pol);
+            tma_load_2d(vdst + bx * Ly::kBoxB + hoff, &tmap_v, xc, y, &full[stage], pol);
+          }
+          if constexpr (fp4(kFmt)) {
+            // the half's block scales: 64 consecutive rows of the block-scale
+            // region, one contiguous run
+            const int64_t soff = (int64_t)y * Ly::kScaleRowB;
+            const int sdst = h * kBoxRows * Ly::kScaleRowB;
+            bulk_load(vdst + Ly::kTileB + sdst, p.k_blocks + soff, kBoxRows * Ly::kScaleRowB,
+                      &full[stage]);
+            bulk_load(vdst + Ly::kTileB + Ly::kScaleB + sdst, p.v_blocks + soff,
+                      kBoxRows * Ly::kScaleRowB, &full[stage]);
+          }
         }
         if (first) {
           const __nv_bfloat16* src = p.q + ((int64_t)b * p.num_q_heads + (int64_t)g * G) * D;
@@ -501,10 +547,10 @@ __global__ void __launch_bounds__(kThreads, 2)
           g = 0;
           do {
             ++b;
-          } while (b < p.batch && tiles_of(clamp_len(p, __ldg(p.seq_lens + b), false)) == 0);
+          } while (b < p.batch && tiles_of<kTile>(clamp_len(p, __ldg(p.seq_lens + b), false)) == 0);
           if (b < p.batch) {
             len = clamp_len(p, __ldg(p.seq_lens + b), false);
-            ntile = tiles_of(len);
+            ntile = tiles_of<kTile>(len);
           }
         }
       }
@@ -514,36 +560,44 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int64_t lo = issued > kStages ? issued - kStages : 0;
     for (int64_t k = lo; k < issued; ++k)
       mbar_wait(&full[k % kStages], (uint32_t)((k / kStages) & 1), p.flags);
-    (void)ok;
     return;
   }
 
   // ---------------------------------------------------------- consumers
+  constexpr int NT = Ly::kWarpTok / 8;  // n-tiles of 8 tokens in a warp's share of S
   const int gid = lane >> 2;   // row of the mma fragment = q head within the group
   const int tid4 = lane & 3;
   const int mat = lane >> 3;   // which 8x8 matrix this lane addresses in ldmatrix.x4
   const int mrow = lane & 7;
   const bool row_ok = gid < G;
+  const int wrow = Ly::kWarpTok * warp;     // this warp's first row of the tile
+  const int my_half = wrow / kBoxRows;      // the 64-row half (page) its rows lie in
   int nflush = 0;
 
-  constexpr int KS = D / 16;  // k-steps over head_dim
-  uint32_t qa[KS][2];         // A fragments of Q: rows gid, two k halves
+  constexpr int KS = D / 16;  // k-steps of 16 over head_dim
+  // A fragments of Q: rows gid, two k halves (f16 / bf16), or for INT8's
+  // k = 32 products the four bytes at d = 16kk + 4*tid4 of the two terms of
+  // a split Q ([0] high, [1] low)
+  uint32_t qa[KS][2];
   // O^T accumulators: PV runs as O^T = V^T P^T (M = head_dim, N = 8 heads).
   // ot[m][0..1] = O[heads 2*tid4, 2*tid4+1][d = 16m + gid], ot[m][2..3] the same at d + 8.
   float ot[D / 16][4];
   float m_run = -INFINITY, l_part = 0.f;
   float qk_mul = p.scale_log2;  // multiplier of the raw scores into log2 units
-  // ldmatrix lanes: K (and bf16 V) matrices (tokens 0-7 | 8-15) x (chunk even |
-  // odd) in the order (0-7, ce), (0-7, ce+1), (8-15, ce), (8-15, ce+1); the
-  // quantised V loads order them (0-7, ce), (8-15, ce), (0-7, ce+1), (8-15, ce+1)
-  const LaneTile ltk = lane_tile<Ly::kBoxRowB>(16 * warp + mrow + (mat >> 1) * 8, mat & 1);
-  const LaneTile ltv = lane_tile<Ly::kBoxRowB>(16 * warp + mrow + (mat & 1) * 8, mat >> 1);
-  // one-byte V: the 8-bit transposing load takes 16 row addresses per
+  // K rows a lane addresses in ldmatrix.x4: matrices (tokens 0-7, chunk ce),
+  // (0-7, ce+1), (8-15, ce), (8-15, ce+1); S column (n-tile nt, element e)
+  // of this thread is token 8*nt + 2*tid4 + e
+  const LaneTile ltk = lane_tile<Ly::kBoxRowB>(wrow + mrow + (mat >> 1) * 8, mat & 1);
+  // FP4 V: transposed 16-bit loads, matrices (tokens 0-7, ce), (8-15, ce),
+  // (0-7, ce+1), (8-15, ce+1)
+  const LaneTile ltv = lane_tile<Ly::kBoxRowB>(wrow + mrow + (mat & 1) * 8, mat >> 1);
+  // One-byte V: the 8-bit transposing load takes 16 row addresses per
   // 16x16 matrix (lanes 0-15: chunk ce, lanes 16-31: chunk ce + 1); row
-  // position 4i + e holds token 2i + (e & 1) + 8 (e >> 1) of the warp's 16,
-  // so that a thread's four rows are the A fragment's token columns (below)
-  const int vrow = 16 * warp + 2 * ((lane & 15) >> 2) + (lane & 1) + 8 * ((lane >> 1) & 1);
-  const LaneTile ltb = lane_tile<Ly::kBoxRowB>(vrow, lane >> 4);
+  // position 4i + e holds token 2i + (e & 1) + 8 (e >> 1) of a 16-token
+  // group, so that a thread's four rows are the f16 A fragment's token
+  // columns (below)
+  const int vrow = 2 * ((lane & 15) >> 2) + (lane & 1) + 8 * ((lane >> 1) & 1);
+  const LaneTile ltb = lane_tile<Ly::kBoxRowB>(wrow + vrow, lane >> 4);
 
   for (int64_t i = 0; i < n_tiles; ++i) {
     const int stage = (int)(i % kStages);
@@ -553,8 +607,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     // bookkeeping is read from the (still unreleased) stage at hand-off
     const int t_flags = info[stage].flags;
     const int t_valid = info[stage].valid;
-    const float t_ks = quant(kFmt) ? info[stage].ks : 1.f;
-    const float t_vs = quant(kFmt) ? info[stage].vs : 1.f;
+    const float t_ks = quant(kFmt) ? info[stage].ks[my_half] : 1.f;
+    const float t_vs = quant(kFmt) ? info[stage].vs[my_half] : 1.f;
     const uint8_t* qs = qbuf + stage * kQStride;
     if (t_flags & kSegFirst) {
       m_run = -INFINITY;
@@ -572,13 +626,14 @@ __global__ void __launch_bounds__(kThreads, 2)
       } else {
         // Q with a per-row power-of-two prescale, in the d order of the K
         // codes that ldmatrix delivers: qv[kk] holds d = 16kk + 4*tid4 +
-        // {0..3} for one-byte codes.  E4M3 uses f16 Q against converted codes.
-        // INT8 feeds the s8 MMA (k = 32), which takes from a thread the bytes
-        // d = 32kp + 4*tid4 + {0..3} and + 16 of one row, that is qv[2kp] and
-        // qv[2kp+1], with Q split into two 8-bit operands (qa[kk][0] high,
-        // [1] low).  FP4 (f16 Q): a 16-byte chunk c holds d = 32c..32c+31 and
-        // a thread's 4 bytes are d = 32c + 8*tid4 + {0..7}; k-step 2c takes
-        // the first four of them, k-step 2c+1 the last four.
+        // {0..3} for one-byte codes.  E4M3 uses f16 Q against converted codes
+        // (the fragment's k pair (2*tid4, +1) holds d = 16kk + 4*tid4 + {0,1}
+        // and the pair (2*tid4+8, +9) holds + {2,3}).  INT8 feeds the s8 MMA
+        // (k = 32), which takes from a thread the bytes d = 32kp + 4*tid4 +
+        // {0..3} and + 16 of one row, that is qv[2kp] and qv[2kp+1].  FP4 (f16
+        // Q): a 16-byte chunk c holds d = 32c..32c+31 and a thread's 4 bytes
+        // are d = 32c + 8*tid4 + {0..7}; k-step 2c takes the first four of
+        // them, k-step 2c+1 the last four.
         float amax = 0.f;
         float qv[KS][4];
 #pragma unroll
@@ -620,8 +675,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             qa[kk][1] = lo;
           }
         } else {
-          // f16: for E4M3 the fragment's k pair (2*tid4, +1) holds d = 16kk +
-          // 4*tid4 + {0,1} and the pair (2*tid4+8, +9) holds + {2,3}
+          // f16 (E4M3, FP4)
 #pragma unroll
           for (int kk = 0; kk < KS; ++kk) {
             qa[kk][0] = pack_f16(qv[kk][0] * pre, qv[kk][1] * pre);
@@ -632,15 +686,79 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
 
-    const int valid = (t_flags & kBadTile) ? 0 : t_valid - 16 * warp;  // tokens of my 16
+    // tokens of my share below the length (none when my half's page is bad)
+    const int valid = (t_flags & (kBadHalf << my_half)) ? 0 : t_valid - wrow;
     if (valid > 0) {
       const uint32_t kbase = smem_u32(tiles + stage * Ly::kStageB);
       const uint32_t vbase = kbase + Ly::kTileB;
-      // ---- S = Q K^T over my 16 tokens (two n-tiles of 8) ----
-      float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      if constexpr (!quant(kFmt)) {
+      // ---- S = Q K^T over my tokens (NT n-tiles of 8) ----
+      float s[NT][4];
+      if constexpr (kFmt == PKV_KV_INT8) {
+        // INT8 codes feed the s8 MMA (k = 32) as they land: the matrices
+        // (tokens 0-7 | 8-15, chunk 2kp | 2kp+1) are the B fragments of two
+        // n-tiles, n-tiles 2, 3 come from 16 rows further; products with the
+        // split Q are exact in s32, and S = 128 hi + lo.
+        int32_t sh[NT][4], sl[NT][4];
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sh[n][e] = sl[n][e] = 0;
+#pragma unroll
+        for (int kp = 0; kp < KS / 2; ++kp) {
+#pragma unroll
+          for (int pr = 0; pr < NT / 2; ++pr) {
+            uint32_t r[4];
+            ldsm_x4(tile_at<Ly::kBoxRowB, kTile>(kbase + pr * 16 * Ly::kBoxRowB, ltk, 2 * kp),
+                    r[0], r[1], r[2], r[3]);
+#pragma unroll
+            for (int n2 = 0; n2 < 2; ++n2) {
+              const int n = 2 * pr + n2;
+              mma_s8(sh[n], qa[2 * kp][0], qa[2 * kp + 1][0], r[2 * n2], r[2 * n2 + 1]);
+              mma_s8(sl[n], qa[2 * kp][1], qa[2 * kp + 1][1], r[2 * n2], r[2 * n2 + 1]);
+            }
+          }
+        }
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) s[n][e] = (float)(sh[n][e] * 128 + sl[n][e]);
+      } else if constexpr (kFmt == PKV_KV_FP8_E4M3) {
+        // E4M3 codes convert exactly to f16 after ldmatrix, four per call;
+        // two accumulation chains per n-tile (even / odd 16-d chunks)
+        float s2[NT][4];
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s[n][e] = s2[n][e] = 0.f;
+#pragma unroll
+        for (int kp = 0; kp < KS / 2; ++kp) {
+#pragma unroll
+          for (int pr = 0; pr < NT / 2; ++pr) {
+            // matrices: (tokens 0-7, chunk 2kp), (0-7, 2kp+1), (8-15, 2kp), (8-15, 2kp+1)
+            uint32_t r[4];
+            ldsm_x4(tile_at<Ly::kBoxRowB, kTile>(kbase + pr * 16 * Ly::kBoxRowB, ltk, 2 * kp),
+                    r[0], r[1], r[2], r[3]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              uint32_t lo, hi;
+              kv8x4_to_f16x2<kFmt>(r[i], lo, hi);
+              const int n = 2 * pr + (i >> 1);
+              float* acc = (i & 1) ? s2[n] : s[n];
+              mma_f16(acc, qa[2 * kp + (i & 1)][0], 0u, qa[2 * kp + (i & 1)][1], 0u, lo, hi);
+            }
+          }
+        }
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) s[n][e] += s2[n][e];
+      } else if constexpr (!quant(kFmt)) {
         // two independent accumulation chains per n-tile (even / odd k-steps)
         float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s[n][e] = 0.f;
 #pragma unroll
         for (int kk = 0; kk < KS; ++kk) {
           uint32_t b0, b1, b2, b3;
@@ -653,20 +771,24 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int n = 0; n < 2; ++n)
 #pragma unroll
           for (int e = 0; e < 4; ++e) s[n][e] += s2[n][e];
-      } else if constexpr (fp4(kFmt)) {
+      } else {
         // FP4 codes: a register of 4 bytes holds d = 32c + 8*tid4 + {0..7} of
         // one token, all in block 2c + tid4/2; its four f16x2 (exact), each
         // times the token's block scale (exact in f16), are the B fragments
         // of k-steps 2c (bytes 0, 1) and 2c+1 (bytes 2, 3).
         const uint8_t* ksc = tiles + stage * Ly::kStageB + 2 * Ly::kTileB;
         float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s[n][e] = 0.f;
         uint32_t sk[2][Ly::kScaleRowB / 4];  // block scales of tokens gid and gid+8
 #pragma unroll
         for (int n = 0; n < 2; ++n)
 #pragma unroll
           for (int w4 = 0; w4 < Ly::kScaleRowB / 4; ++w4)
             sk[n][w4] = *reinterpret_cast<const uint32_t*>(
-                ksc + (16 * warp + 8 * n + gid) * Ly::kScaleRowB + 4 * w4);
+                ksc + (wrow + 8 * n + gid) * Ly::kScaleRowB + 4 * w4);
 #pragma unroll
         for (int c = 0; c < D / 32; c += 2) {
           // matrices: (tokens 0-7, chunk c), (0-7, c+1), (8-15, c), (8-15, c+1)
@@ -690,67 +812,29 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int n = 0; n < 2; ++n)
 #pragma unroll
           for (int e = 0; e < 4; ++e) s[n][e] += s2[n][e];
-      } else if constexpr (kFmt == PKV_KV_INT8) {
-        // INT8 codes feed the s8 MMA (k = 32) as they land: the matrices
-        // (tokens 0-7 | 8-15, chunk 2kp | 2kp+1) are the B fragments of the
-        // two n-tiles; products with the split Q are exact in s32, and
-        // S = 128 hi + lo.
-        int32_t sh[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}}, sl[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
-#pragma unroll
-        for (int kp = 0; kp < KS / 2; ++kp) {
-          uint32_t r[4];
-          ldsm_x4(tile_at<Ly::kBoxRowB, kTile>(kbase, ltk, 2 * kp), r[0], r[1], r[2], r[3]);
-#pragma unroll
-          for (int n = 0; n < 2; ++n) {
-            mma_s8(sh[n], qa[2 * kp][0], qa[2 * kp + 1][0], r[2 * n], r[2 * n + 1]);
-            mma_s8(sl[n], qa[2 * kp][1], qa[2 * kp + 1][1], r[2 * n], r[2 * n + 1]);
-          }
-        }
-#pragma unroll
-        for (int n = 0; n < 2; ++n)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) s[n][e] = (float)(sh[n][e] * 128 + sl[n][e]);
-      } else {
-        // E4M3 codes convert exactly to f16 after ldmatrix, four per call
-        float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-        for (int kp = 0; kp < KS / 2; ++kp) {
-          // matrices: (tokens 0-7, chunk 2kp), (0-7, 2kp+1), (8-15, 2kp), (8-15, 2kp+1)
-          uint32_t r[4];
-          ldsm_x4(tile_at<Ly::kBoxRowB, kTile>(kbase, ltk, 2 * kp), r[0], r[1], r[2], r[3]);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint32_t lo, hi;
-            kv8x4_to_f16x2<kFmt>(r[i], lo, hi);
-            // two accumulation chains per n-tile (even / odd k-steps)
-            float* acc = (i & 1) ? s2[i >> 1] : s[i >> 1];
-            mma_f16(acc, qa[2 * kp + (i & 1)][0], 0u, qa[2 * kp + (i & 1)][1], 0u, lo, hi);
-          }
-        }
-#pragma unroll
-        for (int n = 0; n < 2; ++n)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) s[n][e] += s2[n][e];
       }
       // ---- online softmax on row gid (log2 domain) ----
       const float mul = quant(kFmt) ? qk_mul * t_ks : qk_mul;
-      float x[4];
+      float x[2 * NT];
 #pragma unroll
-      for (int n = 0; n < 2; ++n)
+      for (int n = 0; n < NT; ++n)
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int tok = 8 * n + 2 * tid4 + e;
-          x[2 * n + e] = tok < valid ? s[n][e] * mul : -INFINITY;
-        }
-      float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+        for (int e = 0; e < 2; ++e) x[2 * n + e] = 8 * n + 2 * tid4 + e < valid ? s[n][e] * mul : -INFINITY;
+      float mx = x[0];
+#pragma unroll
+      for (int k = 1; k < 2 * NT; ++k) mx = fmaxf(mx, x[k]);
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
       const float m_new = fmaxf(m_run, mx);  // finite: valid > 0
       const float alpha = fast_exp2(m_run - m_new);
-      float pr[4];
+      float pr[2 * NT];
+      float psum = 0.f;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) pr[e] = fast_exp2(x[e] - m_new);
-      l_part = l_part * alpha + (pr[0] + pr[1]) + (pr[2] + pr[3]);
+      for (int k = 0; k < 2 * NT; ++k) {
+        pr[k] = fast_exp2(x[k] - m_new);
+        psum += pr[k];
+      }
+      l_part = l_part * alpha + psum;
       m_run = m_new;
       // alpha belongs to head gid; O^T columns are heads 2*tid4 and 2*tid4+1.
       // Once the running max settles (most tiles), no row's alpha moves.
@@ -765,160 +849,216 @@ __global__ void __launch_bounds__(kThreads, 2)
           ot[m][3] *= a_hi;
         }
       }
-      // ---- O^T += V^T P^T over my 16 tokens (P^T comes straight from S) ----
-      uint32_t pa0, pa2;
-      if constexpr (!quant(kFmt)) {
-        pa0 = pack_bf16(pr[0], pr[1]);
-        pa2 = pack_bf16(pr[2], pr[3]);
-      } else {
-        pa0 = pack_f16(pr[0] * t_vs, pr[1] * t_vs);
-        pa2 = pack_f16(pr[2] * t_vs, pr[3] * t_vs);
-      }
+      // ---- O^T += V^T P^T over my tokens (P^T comes straight from S) ----
       // V rows past the length may hold anything (NaN): on a partial tile
       // they are zeroed in the fragments, so that 0 * NaN never reaches the
-      // accumulator.  Full tiles, nearly all, take the product without masks.
-      auto pv_product = [&](auto masked) {
-        constexpr bool kMasked = decltype(masked)::value;
-        uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;
-        if constexpr (kMasked) {
-          vm0 = (2 * tid4 < valid ? 0x0000ffffu : 0u) | (2 * tid4 + 1 < valid ? 0xffff0000u : 0u);
-          vm1 = (2 * tid4 + 8 < valid ? 0x0000ffffu : 0u) |
-                (2 * tid4 + 9 < valid ? 0xffff0000u : 0u);
-        }
-        // tokens 2*tid4, 2*tid4+1 (m0) or 2*tid4+8, 2*tid4+9 (m1) of a fragment
-        auto m0 = [&](uint32_t a) -> uint32_t { return kMasked ? (a & vm0) : a; };
-        auto m1 = [&](uint32_t a) -> uint32_t { return kMasked ? (a & vm1) : a; };
-        if constexpr (!quant(kFmt)) {
+      // accumulator.  Full shares, nearly all, take the product without masks.
+      {
+        // products over 16-token groups: P^T of group hv is n-tiles 2hv
+        // (tokens 2*tid4, +1) and 2hv+1 (tokens 8 + 2*tid4, +1)
 #pragma unroll
-          for (int m = 0; m < D / 16; ++m) {
-            // A = V^T rows d 16m..16m+15: matrices (tokens 0-7, chunk 2m), (0-7, 2m+1),
-            // (8-15, 2m), (8-15, 2m+1), transposed on load
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4_t(tile_at<Ly::kBoxRowB, kTile>(vbase, ltk, 2 * m), a0, a1, a2, a3);
-            mma_bf16(ot[m], m0(a0), m0(a1), m1(a2), m1(a3), pa0, pa2);
+        for (int hv = 0; hv < NT / 2; ++hv) {
+          const int vh = valid - 16 * hv;  // tokens of this group below the length
+          if (hv > 0 && vh <= 0) break;
+          uint32_t pa0, pa2;
+          if constexpr (!quant(kFmt)) {
+            pa0 = pack_bf16(pr[4 * hv], pr[4 * hv + 1]);
+            pa2 = pack_bf16(pr[4 * hv + 2], pr[4 * hv + 3]);
+          } else {
+            pa0 = pack_f16(pr[4 * hv] * t_vs, pr[4 * hv + 1] * t_vs);
+            pa2 = pack_f16(pr[4 * hv + 2] * t_vs, pr[4 * hv + 3] * t_vs);
           }
-        } else if constexpr (fp4(kFmt)) {
-          // FP4 V codes from the landed tile.  A transposed load of 16-bit
-          // elements (byte pairs) gives each thread, per 8x8 matrix, tokens
-          // (2*tid4, 2*tid4+1) x codes d = 32c + 4*gid + {0..3} (low half:
-          // the first token).  Interleaving the two tokens' nibbles makes
-          // four bytes, one per d, each the token pair of that d, which
-          // convert exactly to f16x2; times the two tokens' block scales
-          // (block 2c + gid/4) they are the A fragments of V^T.  Fragment
-          // rows: m-tile 2c holds d = 32c + 4*gid + {0, 1} (rows gid, gid+8),
-          // m-tile 2c+1 holds d = 32c + 4*gid + {2, 3}; the snapshot below
-          // undoes the order.
-          const uint8_t* vsc = tiles + stage * Ly::kStageB + 2 * Ly::kTileB + Ly::kScaleB;
-          uint32_t sv[4][Ly::kScaleRowB / 4];  // tokens 2t, 2t+1, 2t+8, 2t+9 of the warp
+          const uint32_t gbase = vbase + hv * 16 * Ly::kBoxRowB;
+          auto pv_product = [&](auto masked) {
+            constexpr bool kMasked = decltype(masked)::value;
+            uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;
+            if constexpr (kMasked) {
+              vm0 = (2 * tid4 < vh ? 0x0000ffffu : 0u) | (2 * tid4 + 1 < vh ? 0xffff0000u : 0u);
+              vm1 = (2 * tid4 + 8 < vh ? 0x0000ffffu : 0u) | (2 * tid4 + 9 < vh ? 0xffff0000u : 0u);
+            }
+            // tokens 2*tid4, 2*tid4+1 (m0) or 2*tid4+8, 2*tid4+9 (m1) of a fragment
+            auto m0 = [&](uint32_t a) -> uint32_t { return kMasked ? (a & vm0) : a; };
+            auto m1 = [&](uint32_t a) -> uint32_t { return kMasked ? (a & vm1) : a; };
+            if constexpr (!quant(kFmt)) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
+              for (int m = 0; m < D / 16; ++m) {
+                // A = V^T rows d 16m..16m+15: matrices (tokens 0-7, chunk 2m), (0-7, 2m+1),
+                // (8-15, 2m), (8-15, 2m+1), transposed on load
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4_t(tile_at<Ly::kBoxRowB, kTile>(gbase, ltk, 2 * m), a0, a1, a2, a3);
+                mma_bf16(ot[m], m0(a0), m0(a1), m1(a2), m1(a3), pa0, pa2);
+              }
+            } else if constexpr (fp4(kFmt)) {
+              // FP4 V codes from the landed tile.  A transposed load of 16-bit
+              // elements (byte pairs) gives each thread, per 8x8 matrix, tokens
+              // (2*tid4, 2*tid4+1) x codes d = 32c + 4*gid + {0..3} (low half:
+              // the first token).  Interleaving the two tokens' nibbles makes
+              // four bytes, one per d, each the token pair of that d, which
+              // convert exactly to f16x2; times the two tokens' block scales
+              // (block 2c + gid/4) they are the A fragments of V^T.  Fragment
+              // rows: m-tile 2c holds d = 32c + 4*gid + {0, 1} (rows gid, gid+8),
+              // m-tile 2c+1 holds d = 32c + 4*gid + {2, 3}; the snapshot below
+              // undoes the order.
+              const uint8_t* vsc = tiles + stage * Ly::kStageB + 2 * Ly::kTileB + Ly::kScaleB;
+              uint32_t sv[4][Ly::kScaleRowB / 4];  // tokens 2t, 2t+1, 2t+8, 2t+9 of the warp
 #pragma unroll
-            for (int w4 = 0; w4 < Ly::kScaleRowB / 4; ++w4)
-              sv[k][w4] = *reinterpret_cast<const uint32_t*>(
-                  vsc + (16 * warp + 2 * tid4 + (k & 1) + 8 * (k >> 1)) * Ly::kScaleRowB + 4 * w4);
-          auto v_pairs = [&](uint32_t codes, uint32_t scale_pair, uint32_t* f) {
-            const uint32_t x = __byte_perm(codes, 0u, 0x3120);  // A.d01 B.d01 A.d23 B.d23
-            const uint32_t lo = x & 0x0f0f0f0fu;                // A.d0 B.d0 A.d2 B.d2
-            const uint32_t hi = (x >> 4) & 0x0f0f0f0fu;         // A.d1 B.d1 A.d3 B.d3
-            const uint32_t z = __byte_perm(lo | (lo >> 4), hi | (hi >> 4), 0x6240);
-            e2m1x8_to_f16x2(z, f);                              // pairs of d0, d1, d2, d3
+              for (int k = 0; k < 4; ++k)
 #pragma unroll
-            for (int k = 0; k < 4; ++k) f[k] = hmul2_u32(f[k], scale_pair);
+                for (int w4 = 0; w4 < Ly::kScaleRowB / 4; ++w4)
+                  sv[k][w4] = *reinterpret_cast<const uint32_t*>(
+                      vsc + (wrow + 2 * tid4 + (k & 1) + 8 * (k >> 1)) * Ly::kScaleRowB + 4 * w4);
+              auto v_pairs = [&](uint32_t codes, uint32_t scale_pair, uint32_t* f) {
+                const uint32_t x = __byte_perm(codes, 0u, 0x3120);  // A.d01 B.d01 A.d23 B.d23
+                const uint32_t lo = x & 0x0f0f0f0fu;                // A.d0 B.d0 A.d2 B.d2
+                const uint32_t hi = (x >> 4) & 0x0f0f0f0fu;         // A.d1 B.d1 A.d3 B.d3
+                const uint32_t z = __byte_perm(lo | (lo >> 4), hi | (hi >> 4), 0x6240);
+                e2m1x8_to_f16x2(z, f);                              // pairs of d0, d1, d2, d3
+#pragma unroll
+                for (int k = 0; k < 4; ++k) f[k] = hmul2_u32(f[k], scale_pair);
+              };
+#pragma unroll
+              for (int c = 0; c < D / 32; c += 2) {
+                // matrices: (tokens 0-7, chunk c), (8-15, c), (0-7, c+1), (8-15, c+1)
+                uint32_t r0, r1, r2, r3;
+                ldsm_x4_t(tile_at<Ly::kBoxRowB, kTile>(vbase, ltv, c), r0, r1, r2, r3);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                  const int cc = c + h;
+                  const uint32_t blk = 2 * cc + (gid >> 2);
+                  const uint32_t s01 =
+                      e4m3_pair_f16x2(sv[0][blk >> 2], blk & 3, sv[1][blk >> 2], blk & 3);
+                  const uint32_t s89 =
+                      e4m3_pair_f16x2(sv[2][blk >> 2], blk & 3, sv[3][blk >> 2], blk & 3);
+                  uint32_t pf[4], qf[4];
+                  v_pairs(h ? r2 : r0, s01, pf);  // tokens 2t, 2t+1
+                  v_pairs(h ? r3 : r1, s89, qf);  // tokens 2t+8, 2t+9
+                  mma_f16(ot[2 * cc], m0(pf[0]), m0(pf[1]), m1(qf[0]), m1(qf[1]), pa0, pa2);
+                  mma_f16(ot[2 * cc + 1], m0(pf[2]), m0(pf[3]), m1(qf[2]), m1(qf[3]), pa0, pa2);
+                }
+              }
+            } else {
+              // One-byte V codes straight from the landed tile.  The transposing
+              // load of 8-bit elements gives the thread (gid, tid4), for byte
+              // column gid of a 16-byte chunk m (d = 16m + gid) and for column
+              // gid + 8, the codes of rows 4*tid4 .. 4*tid4+3, which the row
+              // order above makes tokens 2t, 2t+1, 2t+8, 2t+9 (t = tid4).  Two
+              // exact conversions per register then give the A fragment of V^T
+              // (rows d = 16m + gid and + 8, as in the bf16 path) with no byte
+              // shuffles.
+#pragma unroll
+              for (int m = 0; m < D / 16; m += 2) {
+                uint32_t r[4];  // chunk m: r[0] (column gid), r[1] (gid + 8); chunk m+1: r[2], r[3]
+                ldsm_x2_t_b8(tile_at<Ly::kBoxRowB, kTile>(gbase, ltb, m), r[0], r[1], r[2], r[3]);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                  uint32_t a0, a1, a2, a3;
+                  kv8x4_to_f16x2<kFmt>(r[2 * h], a0, a2);      // d = 16(m+h) + gid
+                  kv8x4_to_f16x2<kFmt>(r[2 * h + 1], a1, a3);  // d = 16(m+h) + gid + 8
+                  mma_f16(ot[m + h], m0(a0), m0(a1), m1(a2), m1(a3), pa0, pa2);
+                }
+              }
+            }
           };
-#pragma unroll
-          for (int c = 0; c < D / 32; c += 2) {
-            // matrices: (tokens 0-7, chunk c), (8-15, c), (0-7, c+1), (8-15, c+1)
-            uint32_t r0, r1, r2, r3;
-            ldsm_x4_t(tile_at<Ly::kBoxRowB, kTile>(vbase, ltv, c), r0, r1, r2, r3);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int cc = c + h;
-              const uint32_t blk = 2 * cc + (gid >> 2);
-              const uint32_t s01 =
-                  e4m3_pair_f16x2(sv[0][blk >> 2], blk & 3, sv[1][blk >> 2], blk & 3);
-              const uint32_t s89 =
-                  e4m3_pair_f16x2(sv[2][blk >> 2], blk & 3, sv[3][blk >> 2], blk & 3);
-              uint32_t pf[4], qf[4];
-              v_pairs(h ? r2 : r0, s01, pf);  // tokens 2t, 2t+1
-              v_pairs(h ? r3 : r1, s89, qf);  // tokens 2t+8, 2t+9
-              mma_f16(ot[2 * cc], m0(pf[0]), m0(pf[1]), m1(qf[0]), m1(qf[1]), pa0, pa2);
-              mma_f16(ot[2 * cc + 1], m0(pf[2]), m0(pf[3]), m1(qf[2]), m1(qf[3]), pa0, pa2);
-            }
-          }
-        } else {
-          // One-byte V codes straight from the landed tile.  The transposing
-          // load of 8-bit elements gives the thread (gid, tid4), for byte
-          // column gid of a 16-byte chunk m (d = 16m + gid) and for column
-          // gid + 8, the codes of rows 4*tid4 .. 4*tid4+3, which the row order
-          // above makes tokens 2t, 2t+1, 2t+8, 2t+9 (t = tid4).  Two exact
-          // conversions per register then give the A fragment of V^T (rows
-          // d = 16m + gid and + 8, as in the bf16 path) with no byte shuffles.
-#pragma unroll
-          for (int m = 0; m < D / 16; m += 2) {
-            uint32_t r[4];  // chunk m: r[0] (column gid), r[1] (gid + 8); chunk m+1: r[2], r[3]
-            ldsm_x2_t_b8(tile_at<Ly::kBoxRowB, kTile>(vbase, ltb, m), r[0], r[1], r[2], r[3]);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              uint32_t a0, a1, a2, a3;
-              kv8x4_to_f16x2<kFmt>(r[2 * h], a0, a2);  // d = 16(m+h) + gid: tokens (2t, 2t+1), (2t+8, 2t+9)
-              kv8x4_to_f16x2<kFmt>(r[2 * h + 1], a1, a3);  // d = 16(m+h) + gid + 8
-              mma_f16(ot[m + h], m0(a0), m0(a1), m1(a2), m1(a3), pa0, pa2);
-            }
-          }
+          if (vh >= 16)
+            pv_product(std::false_type{});
+          else
+            pv_product(std::true_type{});
         }
-      };
-      if (valid >= 16)
-        pv_product(std::false_type{});
-      else
-        pv_product(std::true_type{});
+      }
     }
     if (t_flags & kSegLast) {
-    // ------------------------------------------- hand the segment over
-    // Snapshot this warp's (m, l, o) for the flush warp and go on streaming.
-    float l_row = l_part;
-    l_row += __shfl_xor_sync(0xffffffffu, l_row, 1);
-    l_row += __shfl_xor_sync(0xffffffffu, l_row, 2);
-    if (nflush > 0 && !mbar_wait(red_empty, (uint32_t)((nflush - 1) & 1), p.flags)) return;
-    if (row_ok && tid4 == 0) {
-      red_m[warp * G + gid] = m_run;
-      red_l[warp * G + gid] = l_row;
-    }
-    {
+      // ----------------------------------------- hand the segment over
+      // Each warp snapshots (m, l, o) into its slot and goes on streaming,
+      // once the flush warp has read the previous segment's slots.  With two
+      // slots, warps 2 and 3 do so, and warps 0 and 1 fold their partner's
+      // snapshot (warp + 2) into their own state and write the result back.
+      float l_row = l_part;
+      l_row += __shfl_xor_sync(0xffffffffu, l_row, 1);
+      l_row += __shfl_xor_sync(0xffffffffu, l_row, 2);
+      const int slot = warp % kSnap;
+      float* so = red_o + slot * G * D;
       const int h0 = 2 * tid4, h1 = 2 * tid4 + 1;
-      float* r0 = red_o + (warp * G + h0) * D;
-      float* r1 = red_o + (warp * G + h1) * D;
       // fragment rows gid and gid+8 of d-tile m hold d 16m + gid and +8
       // (bf16 and one-byte codes), or 32(m/2) + 4*gid + 2(m%2) and +1 (FP4),
       // as the PV products lay them out
       const int d_step = fp4(kFmt) ? 1 : 8;
+      auto d_of = [&](int m) { return fp4(kFmt) ? 32 * (m >> 1) + 4 * gid + 2 * (m & 1) : 16 * m + gid; };
+      auto write_desc = [&]() {
+        const TileInfo& ti = info[stage];
+        FlushDesc fd;
+        fd.b = ti.b;
+        fd.g = ti.g;
+        fd.slot = ti.slot;
+        fd.seg_base = ti.seg_base;
+        fd.nseg = ti.nseg;
+        fd.whole = (t_flags & kUnitWhole) ? 1 : 0;
+        fd.final = (i == n_tiles - 1) ? 1 : 0;
+        *desc = fd;
+      };
+      if (kSnap == kConsumerWarps || warp >= kSnap) {
+        if (nflush > 0 && !mbar_wait(red_empty, (uint32_t)((nflush - 1) & 1), p.flags)) return;
+        if (row_ok && tid4 == 0) {
+          red_m[slot * G + gid] = m_run;
+          red_l[slot * G + gid] = l_row;
+        }
+        float* r0 = so + h0 * D;
+        float* r1 = so + h1 * D;
 #pragma unroll
-      for (int m = 0; m < D / 16; ++m) {
-        const int d = fp4(kFmt) ? 32 * (m >> 1) + 4 * gid + 2 * (m & 1) : 16 * m + gid;
-        if (h0 < G) {
-          r0[d] = ot[m][0];
-          r0[d + d_step] = ot[m][2];
+        for (int m = 0; m < D / 16; ++m) {
+          const int d = d_of(m);
+          if (h0 < G) {
+            r0[d] = ot[m][0];
+            r0[d + d_step] = ot[m][2];
+          }
+          if (h1 < G) {
+            r1[d] = ot[m][1];
+            r1[d + d_step] = ot[m][3];
+          }
         }
-        if (h1 < G) {
-          r1[d] = ot[m][1];
-          r1[d + d_step] = ot[m][3];
+        if (kSnap == kConsumerWarps) {
+          if (warp == 0 && lane == 0) write_desc();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(red_full);
+        } else {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(pair_full);
         }
+      } else {
+        if (!mbar_wait(pair_full, (uint32_t)(nflush & 1), p.flags)) return;
+        const float mp = row_ok ? red_m[slot * G + gid] : -INFINITY;
+        const float lp = row_ok ? red_l[slot * G + gid] : 0.f;
+        const float M = fmaxf(m_run, mp);
+        const float sa = m_run == -INFINITY ? 0.f : fast_exp2(m_run - M);
+        const float sb = mp == -INFINITY ? 0.f : fast_exp2(mp - M);
+        const float l_new = sa * l_row + sb * lp;
+        const float a_lo = __shfl_sync(0xffffffffu, sa, 8 * tid4);
+        const float a_hi = __shfl_sync(0xffffffffu, sa, 8 * tid4 + 4);
+        const float b_lo = __shfl_sync(0xffffffffu, sb, 8 * tid4);
+        const float b_hi = __shfl_sync(0xffffffffu, sb, 8 * tid4 + 4);
+        float* r0 = so + h0 * D;
+        float* r1 = so + h1 * D;
+#pragma unroll
+        for (int m = 0; m < D / 16; ++m) {
+          const int d = d_of(m);
+          if (h0 < G) {
+            r0[d] = ot[m][0] * a_lo + r0[d] * b_lo;
+            r0[d + d_step] = ot[m][2] * a_lo + r0[d + d_step] * b_lo;
+          }
+          if (h1 < G) {
+            r1[d] = ot[m][1] * a_hi + r1[d] * b_hi;
+            r1[d + d_step] = ot[m][3] * a_hi + r1[d + d_step] * b_hi;
+          }
+        }
+        __syncwarp();  // every lane has read the partner's (m, l) row
+        if (row_ok && tid4 == 0) {
+          red_m[slot * G + gid] = M;
+          red_l[slot * G + gid] = l_new;
+        }
+        if (warp == 0 && lane == 0) write_desc();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(red_full);
       }
-    }
-    if (warp == 0 && lane == 0) {
-      const TileInfo& ti = info[stage];
-      FlushDesc fd;
-      fd.b = ti.b;
-      fd.g = ti.g;
-      fd.slot = ti.slot;
-      fd.seg_base = ti.seg_base;
-      fd.nseg = ti.nseg;
-      fd.whole = (t_flags & kUnitWhole) ? 1 : 0;
-      fd.final = (i == n_tiles - 1) ? 1 : 0;
-      *desc = fd;
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(red_full);
-    ++nflush;
+      ++nflush;
     }
     // release the stage (all of this warp's reads of it are done)
     __syncwarp();
@@ -1021,48 +1161,52 @@ cudaError_t merge_launch(const DecodeParams& p, cudaStream_t stream) {
 }
 
 // ------------------------------------------------------------- host side
-template <int D, int kFmt, int kStages>
+template <int D, int kFmt, int kStages, int kSnap>
 size_t decode_smem_bytes(int G) {
-  return 1024 + smem_plan<D, kFmt, kStages>(G).total;  // + alignment slack
+  return 1024 + smem_plan<D, kFmt, kStages, kSnap>(G).total;  // + alignment slack
 }
 
-template <int D, int kFmt, int kStages>
+template <int D, int kFmt, int kStages, int kSnap>
 cudaError_t decode_prepare(int G, int* ctas_per_sm) {
-  auto k = decode_kernel<D, kFmt, kStages>;
-  const size_t smem = decode_smem_bytes<D, kFmt, kStages>(G);
+  auto k = decode_kernel<D, kFmt, kStages, kSnap>;
+  const size_t smem = decode_smem_bytes<D, kFmt, kStages, kSnap>(G);
   // The attribute belongs to the instantiation, which serves every group
   // size: allow the largest footprint once, not the one of this call.
-  const size_t most = decode_smem_bytes<D, kFmt, kStages>(kMaxGroup);
+  const size_t most = decode_smem_bytes<D, kFmt, kStages, kSnap>(kMaxGroup);
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most);
   if (e != cudaSuccess) return e;
   return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, k, kThreads, smem);
 }
 
-template <int D, int kFmt, int kStages>
+template <int D, int kFmt, int kStages, int kSnap>
 cudaError_t decode_launch(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                           int num_ctas, cudaStream_t stream) {
-  const size_t smem = decode_smem_bytes<D, kFmt, kStages>(p.group);
-  decode_kernel<D, kFmt, kStages><<<num_ctas, kThreads, smem, stream>>>(tk, tv, p);
+  const size_t smem = decode_smem_bytes<D, kFmt, kStages, kSnap>(p.group);
+  decode_kernel<D, kFmt, kStages, kSnap><<<num_ctas, kThreads, smem, stream>>>(tk, tv, p);
   return cudaGetLastError();
 }
 
-// Deepest ring that still lets two CTAs share an SM (228 KB of shared
-// memory per SM, 1 KB of it reserved per CTA).
+// Ring depth and snapshot slots: the deepest ring that still lets two CTAs
+// share an SM (228 KB of shared memory per SM, 1 KB of it reserved per CTA)
+// with a slot per consumer warp, unless halving the slots buys a third stage.
 constexpr size_t kSmemPerCtaFor2 = 113 * 1024;
+enum class Plan { k4x4, k3x4, k3x2, k2x4 };
 
 template <int D, int kFmt>
-int pick_stages(int G) {
-  if (decode_smem_bytes<D, kFmt, 4>(G) <= kSmemPerCtaFor2) return 4;
-  if (decode_smem_bytes<D, kFmt, 3>(G) <= kSmemPerCtaFor2) return 3;
-  return 2;
+Plan pick_plan(int G) {
+  if (decode_smem_bytes<D, kFmt, 4, 4>(G) <= kSmemPerCtaFor2) return Plan::k4x4;
+  if (decode_smem_bytes<D, kFmt, 3, 4>(G) <= kSmemPerCtaFor2) return Plan::k3x4;
+  if (decode_smem_bytes<D, kFmt, 3, 2>(G) <= kSmemPerCtaFor2) return Plan::k3x2;
+  return Plan::k2x4;
 }
 
 template <int D, int kFmt>
 cudaError_t occupancy_for(int G, int* n) {
-  switch (pick_stages<D, kFmt>(G)) {
-    case 4: return decode_prepare<D, kFmt, 4>(G, n);
-    case 3: return decode_prepare<D, kFmt, 3>(G, n);
-    default: return decode_prepare<D, kFmt, 2>(G, n);
+  switch (pick_plan<D, kFmt>(G)) {
+    case Plan::k4x4: return decode_prepare<D, kFmt, 4, 4>(G, n);
+    case Plan::k3x4: return decode_prepare<D, kFmt, 3, 4>(G, n);
+    case Plan::k3x2: return decode_prepare<D, kFmt, 3, 2>(G, n);
+    default: return decode_prepare<D, kFmt, 2, 4>(G, n);
   }
 }
 
@@ -1070,10 +1214,11 @@ template <int D, int kFmt>
 cudaError_t run_for(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
                     int num_ctas, cudaStream_t stream) {
   cudaError_t e;
-  switch (pick_stages<D, kFmt>(p.group)) {
-    case 4: e = decode_launch<D, kFmt, 4>(tk, tv, p, num_ctas, stream); break;
-    case 3: e = decode_launch<D, kFmt, 3>(tk, tv, p, num_ctas, stream); break;
-    default: e = decode_launch<D, kFmt, 2>(tk, tv, p, num_ctas, stream); break;
+  switch (pick_plan<D, kFmt>(p.group)) {
+    case Plan::k4x4: e = decode_launch<D, kFmt, 4, 4>(tk, tv, p, num_ctas, stream); break;
+    case Plan::k3x4: e = decode_launch<D, kFmt, 3, 4>(tk, tv, p, num_ctas, stream); break;
+    case Plan::k3x2: e = decode_launch<D, kFmt, 3, 2>(tk, tv, p, num_ctas, stream); break;
+    default: e = decode_launch<D, kFmt, 2, 4>(tk, tv, p, num_ctas, stream); break;
   }
   if (e != cudaSuccess) return e;
   return merge_launch<D>(p, stream);
