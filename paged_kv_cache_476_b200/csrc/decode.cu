@@ -115,7 +115,7 @@ __host__ __device__ inline SmemPlan smem_plan(int G) {
   o += kStages * align_up(G * D * 2, 128);
   o = align_up(o, 1024);
   s.red_o = o;
-  o += kSnap * G * D * 4;
+  o += kSnap * G * (D + 4) * 4;  // rows padded by 4 floats (no bank conflicts)
   s.red_m = o;
   o += kSnap * G * 4;
   s.red_l = o;
@@ -234,6 +234,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int G = p.group;
   const SmemPlan sp = smem_plan<D, kFmt, kStages, kSnap>(G);
   const uint32_t kQStride = align_up(G * D * 2, 128);
+  constexpr int kRedRow = D + 4;  // row stride (floats) of the snapshot buffers
   uint8_t* tiles = smem;
   uint8_t* qbuf = smem + sp.q;
   float* red_o = reinterpret_cast<float*>(smem + sp.red_o);
@@ -356,14 +357,26 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         const int64_t orow = (int64_t)fd.b * p.num_q_heads + fd.g * G + r;
         const float inv = den > 0.f ? 1.f / den : 0.f;
-        for (int d = lane; d < D; d += 32) {
-          float num = 0.f;
+        // four consecutive d per lane: 16-byte snapshot reads, one 8-byte
+        // (bf16 output) or 16-byte (partial) store
+        for (int d0 = 4 * lane; d0 < D; d0 += 128) {
+          float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-          for (int w = 0; w < kSnap; ++w) num += sc[w] * red_o[(w * G + r) * D + d];
-          if (fd.whole)
-            p.out[orow * D + d] = __float2bfloat16(num * inv);
-          else
-            p.part_o[((int64_t)fd.slot * G + r) * D + d] = num;
+          for (int w = 0; w < kSnap; ++w) {
+            const float4 o = *reinterpret_cast<const float4*>(red_o + (w * G + r) * kRedRow + d0);
+            num.x += sc[w] * o.x;
+            num.y += sc[w] * o.y;
+            num.z += sc[w] * o.z;
+            num.w += sc[w] * o.w;
+          }
+          if (fd.whole) {
+            uint2 packed;
+            packed.x = pack_bf16(num.x * inv, num.y * inv);
+            packed.y = pack_bf16(num.z * inv, num.w * inv);
+            *reinterpret_cast<uint2*>(p.out + orow * D + d0) = packed;
+          } else {
+            *reinterpret_cast<float4*>(p.part_o + ((int64_t)fd.slot * G + r) * D + d0) = num;
+          }
         }
         if (lane == 0) {
           if (fd.whole) {
@@ -976,7 +989,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       l_row += __shfl_xor_sync(0xffffffffu, l_row, 1);
       l_row += __shfl_xor_sync(0xffffffffu, l_row, 2);
       const int slot = warp % kSnap;
-      float* so = red_o + slot * G * D;
+      float* so = red_o + slot * G * kRedRow;
       const int h0 = 2 * tid4, h1 = 2 * tid4 + 1;
       // fragment rows gid and gid+8 of d-tile m hold d 16m + gid and +8
       // (bf16 and one-byte codes), or 32(m/2) + 4*gid + 2(m%2) and +1 (FP4),
@@ -1001,8 +1014,8 @@ __global__ void __launch_bounds__(kThreads, 2)
           red_m[slot * G + gid] = m_run;
           red_l[slot * G + gid] = l_row;
         }
-        float* r0 = so + h0 * D;
-        float* r1 = so + h1 * D;
+        float* r0 = so + h0 * kRedRow;
+        float* r1 = so + h1 * kRedRow;
 #pragma unroll
         for (int m = 0; m < D / 16; ++m) {
           const int d = d_of(m);
@@ -1035,8 +1048,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         const float a_hi = __shfl_sync(0xffffffffu, sa, 8 * tid4 + 4);
         const float b_lo = __shfl_sync(0xffffffffu, sb, 8 * tid4);
         const float b_hi = __shfl_sync(0xffffffffu, sb, 8 * tid4 + 4);
-        float* r0 = so + h0 * D;
-        float* r1 = so + h1 * D;
+        float* r0 = so + h0 * kRedRow;
+        float* r1 = so + h1 * kRedRow;
 #pragma unroll
         for (int m = 0; m < D / 16; ++m) {
           const int d = d_of(m);
