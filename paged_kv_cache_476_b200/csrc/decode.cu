@@ -577,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 
   // ---------------------------------------------------------- consumers
-  constexpr int NT = Ly::kWarpTok / 8;  // n-tiles of 8 tokens in a warp's share of S
+  constexpr int NG = Ly::kWarpTok / 16;  // 16-token groups in a warp's share of the tile
   const int gid = lane >> 2;   // row of the mma fragment = q head within the group
   const int tid4 = lane & 3;
   const int mat = lane >> 3;   // which 8x8 matrix this lane addresses in ldmatrix.x4
@@ -588,18 +588,21 @@ __global__ void __launch_bounds__(kThreads, 2)
   int nflush = 0;
 
   constexpr int KS = D / 16;  // k-steps of 16 over head_dim
-  // A fragments of Q: rows gid, two k halves (f16 / bf16), or for INT8's
-  // k = 32 products the four bytes at d = 16kk + 4*tid4 of the two terms of
-  // a split Q ([0] high, [1] low)
+  // Q as the B operand of S^T = K Q^T (column gid = head gid): two k halves
+  // (f16 / bf16), or for INT8's k = 32 products the four bytes at d = 16kk +
+  // 4*tid4 of the two terms of a split Q ([0] high, [1] low)
   uint32_t qa[KS][2];
   // O^T accumulators: PV runs as O^T = V^T P^T (M = head_dim, N = 8 heads).
   // ot[m][0..1] = O[heads 2*tid4, 2*tid4+1][d = 16m + gid], ot[m][2..3] the same at d + 8.
   float ot[D / 16][4];
-  float m_run = -INFINITY, l_part = 0.f;
-  float qk_mul = p.scale_log2;  // multiplier of the raw scores into log2 units
+  // running max and partial sum of heads 2*tid4 and 2*tid4 + 1 (the O^T
+  // columns of this thread)
+  float m_run[2] = {-INFINITY, -INFINITY}, l_part[2] = {0.f, 0.f};
+  float qk_mul = p.scale_log2;  // multiplier of head gid's raw scores into log2 units
+  float hmul[2] = {p.scale_log2, p.scale_log2};  // the same for heads 2*tid4, 2*tid4 + 1
   // K rows a lane addresses in ldmatrix.x4: matrices (tokens 0-7, chunk ce),
-  // (0-7, ce+1), (8-15, ce), (8-15, ce+1); S column (n-tile nt, element e)
-  // of this thread is token 8*nt + 2*tid4 + e
+  // (0-7, ce+1), (8-15, ce), (8-15, ce+1), the A fragments (a0, a2, a1, a3)
+  // of S^T for one 16-token group
   const LaneTile ltk = lane_tile<Ly::kBoxRowB>(wrow + mrow + (mat >> 1) * 8, mat & 1);
   // FP4 V: transposed 16-bit loads, matrices (tokens 0-7, ce), (8-15, ce),
   // (0-7, ce+1), (8-15, ce+1)
@@ -624,8 +627,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float t_vs = quant(kFmt) ? info[stage].vs[my_half] : 1.f;
     const uint8_t* qs = qbuf + stage * kQStride;
     if (t_flags & kSegFirst) {
-      m_run = -INFINITY;
-      l_part = 0.f;
+      m_run[0] = m_run[1] = -INFINITY;
+      l_part[0] = l_part[1] = 0.f;
 #pragma unroll
       for (int m = 0; m < D / 16; ++m) ot[m][0] = ot[m][1] = ot[m][2] = ot[m][3] = 0.f;
       if constexpr (!quant(kFmt)) {
@@ -696,6 +699,8 @@ __global__ void __launch_bounds__(kThreads, 2)
           }
         }
         qk_mul = p.scale_log2 * ldexpf(1.f, -ex);
+        hmul[0] = __shfl_sync(0xffffffffu, qk_mul, 8 * tid4);      // lane of head 2*tid4
+        hmul[1] = __shfl_sync(0xffffffffu, qk_mul, 8 * tid4 + 4);  // head 2*tid4 + 1
       }
     }
 
@@ -704,183 +709,184 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (valid > 0) {
       const uint32_t kbase = smem_u32(tiles + stage * Ly::kStageB);
       const uint32_t vbase = kbase + Ly::kTileB;
-      // ---- S = Q K^T over my tokens (NT n-tiles of 8) ----
-      float s[NT][4];
+      // ---- S^T = K Q^T over my tokens: a 16-token group fills the 16 rows
+      // of a product, the group's heads its 8 columns ----
+      // st[g] = S^T at (token gid, head 2*tid4), (gid, 2*tid4+1), (gid+8,
+      // 2*tid4), (gid+8, 2*tid4+1) of group g (tokens 16g..16g+15 of my share)
+      float st[NG][4];
       if constexpr (kFmt == PKV_KV_INT8) {
-        // INT8 codes feed the s8 MMA (k = 32) as they land: the matrices
-        // (tokens 0-7 | 8-15, chunk 2kp | 2kp+1) are the B fragments of two
-        // n-tiles, n-tiles 2, 3 come from 16 rows further; products with the
-        // split Q are exact in s32, and S = 128 hi + lo.
-        int32_t sh[NT][4], sl[NT][4];
+        // INT8 codes are the A operand of the s8 MMA (k = 32) as they land,
+        // the two terms of the split Q its B; S = 128 hi + lo exactly in s32
+        int32_t sh[NG][4], sl[NG][4];
 #pragma unroll
-        for (int n = 0; n < NT; ++n)
+        for (int g = 0; g < NG; ++g)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) sh[n][e] = sl[n][e] = 0;
+          for (int e = 0; e < 4; ++e) sh[g][e] = sl[g][e] = 0;
 #pragma unroll
         for (int kp = 0; kp < KS / 2; ++kp) {
 #pragma unroll
-          for (int pr = 0; pr < NT / 2; ++pr) {
+          for (int g = 0; g < NG; ++g) {
             uint32_t r[4];
-            ldsm_x4(tile_at<Ly::kBoxRowB, kTile>(kbase + pr * 16 * Ly::kBoxRowB, ltk, 2 * kp),
+            ldsm_x4(tile_at<Ly::kBoxRowB, kTile>(kbase + g * 16 * Ly::kBoxRowB, ltk, 2 * kp),
                     r[0], r[1], r[2], r[3]);
-#pragma unroll
-            for (int n2 = 0; n2 < 2; ++n2) {
-              const int n = 2 * pr + n2;
-              mma_s8(sh[n], qa[2 * kp][0], qa[2 * kp + 1][0], r[2 * n2], r[2 * n2 + 1]);
-              mma_s8(sl[n], qa[2 * kp][1], qa[2 * kp + 1][1], r[2 * n2], r[2 * n2 + 1]);
-            }
+            mma_s8_full(sh[g], r[0], r[2], r[1], r[3], qa[2 * kp][0], qa[2 * kp + 1][0]);
+            mma_s8_full(sl[g], r[0], r[2], r[1], r[3], qa[2 * kp][1], qa[2 * kp + 1][1]);
           }
         }
 #pragma unroll
-        for (int n = 0; n < NT; ++n)
+        for (int g = 0; g < NG; ++g)
 #pragma unroll
-          for (int e = 0; e < 2; ++e) s[n][e] = (float)(sh[n][e] * 128 + sl[n][e]);
-      } else if constexpr (kFmt == PKV_KV_FP8_E4M3) {
-        // E4M3 codes convert exactly to f16 after ldmatrix, four per call;
-        // two accumulation chains per n-tile (even / odd 16-d chunks)
-        float s2[NT][4];
-#pragma unroll
-        for (int n = 0; n < NT; ++n)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) s[n][e] = s2[n][e] = 0.f;
-#pragma unroll
-        for (int kp = 0; kp < KS / 2; ++kp) {
-#pragma unroll
-          for (int pr = 0; pr < NT / 2; ++pr) {
-            // matrices: (tokens 0-7, chunk 2kp), (0-7, 2kp+1), (8-15, 2kp), (8-15, 2kp+1)
-            uint32_t r[4];
-            ldsm_x4(tile_at<Ly::kBoxRowB, kTile>(kbase + pr * 16 * Ly::kBoxRowB, ltk, 2 * kp),
-                    r[0], r[1], r[2], r[3]);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              uint32_t lo, hi;
-              kv8x4_to_f16x2<kFmt>(r[i], lo, hi);
-              const int n = 2 * pr + (i >> 1);
-              float* acc = (i & 1) ? s2[n] : s[n];
-              mma_f16(acc, qa[2 * kp + (i & 1)][0], 0u, qa[2 * kp + (i & 1)][1], 0u, lo, hi);
-            }
-          }
-        }
-#pragma unroll
-        for (int n = 0; n < NT; ++n)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) s[n][e] += s2[n][e];
-      } else if constexpr (!quant(kFmt)) {
-        // two independent accumulation chains per n-tile (even / odd k-steps)
-        float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-        for (int n = 0; n < 2; ++n)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) s[n][e] = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < KS; ++kk) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(tile_at<Ly::kBoxRowB, kTile>(kbase, ltk, 2 * kk), b0, b1, b2, b3);
-          float(*acc)[4] = (kk & 1) ? s2 : s;
-          mma_bf16(acc[0], qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
-          mma_bf16(acc[1], qa[kk][0], 0u, qa[kk][1], 0u, b2, b3);
-        }
-#pragma unroll
-        for (int n = 0; n < 2; ++n)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) s[n][e] += s2[n][e];
+          for (int e = 0; e < 4; ++e) st[g][e] = (float)(sh[g][e] * 128 + sl[g][e]);
       } else {
-        // FP4 codes: a register of 4 bytes holds d = 32c + 8*tid4 + {0..7} of
-        // one token, all in block 2c + tid4/2; its four f16x2 (exact), each
-        // times the token's block scale (exact in f16), are the B fragments
-        // of k-steps 2c (bytes 0, 1) and 2c+1 (bytes 2, 3).
-        const uint8_t* ksc = tiles + stage * Ly::kStageB + 2 * Ly::kTileB;
-        float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        // f16 / bf16 products, two accumulation chains per group (even / odd
+        // k-steps)
+        float s2[NG][4];
 #pragma unroll
-        for (int n = 0; n < 2; ++n)
+        for (int g = 0; g < NG; ++g)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) s[n][e] = 0.f;
-        uint32_t sk[2][Ly::kScaleRowB / 4];  // block scales of tokens gid and gid+8
+          for (int e = 0; e < 4; ++e) st[g][e] = s2[g][e] = 0.f;
+        if constexpr (kFmt == PKV_KV_FP8_E4M3) {
+          // E4M3 codes convert exactly to f16 after ldmatrix, four per call:
+          // (lo, hi) of a register are the k pairs (2*tid4, +1) and
+          // (2*tid4+8, +9) of its token, Q permuted the same way
 #pragma unroll
-        for (int n = 0; n < 2; ++n)
+          for (int kp = 0; kp < KS / 2; ++kp) {
 #pragma unroll
-          for (int w4 = 0; w4 < Ly::kScaleRowB / 4; ++w4)
-            sk[n][w4] = *reinterpret_cast<const uint32_t*>(
-                ksc + (wrow + 8 * n + gid) * Ly::kScaleRowB + 4 * w4);
+            for (int g = 0; g < NG; ++g) {
+              uint32_t r[4];
+              ldsm_x4(tile_at<Ly::kBoxRowB, kTile>(kbase + g * 16 * Ly::kBoxRowB, ltk, 2 * kp),
+                      r[0], r[1], r[2], r[3]);
 #pragma unroll
-        for (int c = 0; c < D / 32; c += 2) {
-          // matrices: (tokens 0-7, chunk c), (0-7, c+1), (8-15, c), (8-15, c+1)
-          uint32_t r[4];
-          ldsm_x4(tile_at<Ly::kBoxRowB, kTile>(kbase, ltk, c), r[0], r[1], r[2], r[3]);
+              for (int h = 0; h < 2; ++h) {
+                uint32_t l0, h0, l1, h1;
+                kv8x4_to_f16x2<kFmt>(r[h], l0, h0);      // token gid, chunk 2kp + h
+                kv8x4_to_f16x2<kFmt>(r[2 + h], l1, h1);  // token gid + 8
+                mma_f16(h ? s2[g] : st[g], l0, l1, h0, h1, qa[2 * kp + h][0], qa[2 * kp + h][1]);
+              }
+            }
+          }
+        } else if constexpr (!quant(kFmt)) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int n = i >> 1, cc = c + (i & 1);
-            const uint32_t blk = 2 * cc + (tid4 >> 1);
-            const uint32_t sbh = e4m3_splat_f16x2(sk[n][blk >> 2], blk & 3);
-            uint32_t f[4];
-            e2m1x8_to_f16x2(r[i], f);
+          for (int kk = 0; kk < KS; ++kk) {
+            uint32_t r[4];
+            ldsm_x4(tile_at<Ly::kBoxRowB, kTile>(kbase, ltk, 2 * kk), r[0], r[1], r[2], r[3]);
+            mma_bf16((kk & 1) ? s2[0] : st[0], r[0], r[2], r[1], r[3], qa[kk][0], qa[kk][1]);
+          }
+        } else {
+          // FP4 codes: a register of 4 bytes holds d = 32c + 8*tid4 + {0..7}
+          // of one token, all in block 2c + tid4/2; its four f16x2 (exact),
+          // each times the token's block scale (exact in f16), are that
+          // token's A registers of k-steps 2c (bytes 0, 1) and 2c+1 (bytes 2, 3).
+          const uint8_t* ksc = tiles + stage * Ly::kStageB + 2 * Ly::kTileB;
+          uint32_t sk[2][Ly::kScaleRowB / 4];  // block scales of tokens gid and gid+8
 #pragma unroll
-            for (int k = 0; k < 4; ++k) f[k] = hmul2_u32(f[k], sbh);
-            // two accumulation chains per n-tile (even / odd k-steps)
-            mma_f16(s[n], qa[2 * cc][0], 0u, qa[2 * cc][1], 0u, f[0], f[1]);
-            mma_f16(s2[n], qa[2 * cc + 1][0], 0u, qa[2 * cc + 1][1], 0u, f[2], f[3]);
+          for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int w4 = 0; w4 < Ly::kScaleRowB / 4; ++w4)
+              sk[n][w4] = *reinterpret_cast<const uint32_t*>(
+                  ksc + (wrow + 8 * n + gid) * Ly::kScaleRowB + 4 * w4);
+#pragma unroll
+          for (int c = 0; c < D / 32; c += 2) {
+            // matrices: (tokens 0-7, chunk c), (0-7, c+1), (8-15, c), (8-15, c+1)
+            uint32_t r[4];
+            ldsm_x4(tile_at<Ly::kBoxRowB, kTile>(kbase, ltk, c), r[0], r[1], r[2], r[3]);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int cc = c + h;
+              const uint32_t blk = 2 * cc + (tid4 >> 1);
+              uint32_t f0[4], f1[4];
+              e2m1x8_to_f16x2(r[h], f0);
+              e2m1x8_to_f16x2(r[2 + h], f1);
+              const uint32_t sb0 = e4m3_splat_f16x2(sk[0][blk >> 2], blk & 3);
+              const uint32_t sb1 = e4m3_splat_f16x2(sk[1][blk >> 2], blk & 3);
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                f0[k] = hmul2_u32(f0[k], sb0);
+                f1[k] = hmul2_u32(f1[k], sb1);
+              }
+              mma_f16(st[0], f0[0], f1[0], f0[1], f1[1], qa[2 * cc][0], qa[2 * cc][1]);
+              mma_f16(s2[0], f0[2], f1[2], f0[3], f1[3], qa[2 * cc + 1][0], qa[2 * cc + 1][1]);
+            }
           }
         }
 #pragma unroll
-        for (int n = 0; n < 2; ++n)
+        for (int g = 0; g < NG; ++g)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) s[n][e] += s2[n][e];
+          for (int e = 0; e < 4; ++e) st[g][e] += s2[g][e];
       }
-      // ---- online softmax on row gid (log2 domain) ----
-      const float mul = quant(kFmt) ? qk_mul * t_ks : qk_mul;
-      float x[2 * NT];
+      // ---- online softmax per head (log2 domain): this thread holds heads
+      // 2*tid4 (e even) and 2*tid4 + 1 (e odd) for tokens 16g + gid + 8(e/2);
+      // the eight lanes of a head column reduce over their tokens ----
+      const float mul0 = quant(kFmt) ? hmul[0] * t_ks : hmul[0];
+      const float mul1 = quant(kFmt) ? hmul[1] * t_ks : hmul[1];
+      float x[NG][4];
+      float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-      for (int n = 0; n < NT; ++n)
+      for (int g = 0; g < NG; ++g)
 #pragma unroll
-        for (int e = 0; e < 2; ++e) x[2 * n + e] = 8 * n + 2 * tid4 + e < valid ? s[n][e] * mul : -INFINITY;
-      float mx = x[0];
+        for (int e = 0; e < 4; ++e) {
+          const bool in = 16 * g + gid + 8 * (e >> 1) < valid;
+          x[g][e] = in ? st[g][e] * ((e & 1) ? mul1 : mul0) : -INFINITY;
+          if (e & 1)
+            mx1 = fmaxf(mx1, x[g][e]);
+          else
+            mx0 = fmaxf(mx0, x[g][e]);
+        }
 #pragma unroll
-      for (int k = 1; k < 2 * NT; ++k) mx = fmaxf(mx, x[k]);
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      const float m_new = fmaxf(m_run, mx);  // finite: valid > 0
-      const float alpha = fast_exp2(m_run - m_new);
-      float pr[2 * NT];
-      float psum = 0.f;
-#pragma unroll
-      for (int k = 0; k < 2 * NT; ++k) {
-        pr[k] = fast_exp2(x[k] - m_new);
-        psum += pr[k];
+      for (int o = 4; o < 32; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
       }
-      l_part = l_part * alpha + psum;
-      m_run = m_new;
-      // alpha belongs to head gid; O^T columns are heads 2*tid4 and 2*tid4+1.
-      // Once the running max settles (most tiles), no row's alpha moves.
-      if (__any_sync(0xffffffffu, alpha != 1.f)) {
-        const float a_lo = __shfl_sync(0xffffffffu, alpha, 8 * tid4);
-        const float a_hi = __shfl_sync(0xffffffffu, alpha, 8 * tid4 + 4);
+      const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);  // finite: valid > 0
+      const float al0 = fast_exp2(m_run[0] - mn0), al1 = fast_exp2(m_run[1] - mn1);
+      float pr[NG][4];
+      float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+      for (int g = 0; g < NG; ++g) {
+        pr[g][0] = fast_exp2(x[g][0] - mn0);
+        pr[g][1] = fast_exp2(x[g][1] - mn1);
+        pr[g][2] = fast_exp2(x[g][2] - mn0);
+        pr[g][3] = fast_exp2(x[g][3] - mn1);
+        ps0 += pr[g][0] + pr[g][2];
+        ps1 += pr[g][1] + pr[g][3];
+      }
+      l_part[0] = l_part[0] * al0 + ps0;
+      l_part[1] = l_part[1] * al1 + ps1;
+      m_run[0] = mn0;
+      m_run[1] = mn1;
+      // The factors belong to this thread's own O^T columns.  Once the
+      // running max settles (most tiles), no head's factor moves.
+      if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
 #pragma unroll
         for (int m = 0; m < D / 16; ++m) {
-          ot[m][0] *= a_lo;
-          ot[m][1] *= a_hi;
-          ot[m][2] *= a_lo;
-          ot[m][3] *= a_hi;
+          ot[m][0] *= al0;
+          ot[m][1] *= al1;
+          ot[m][2] *= al0;
+          ot[m][3] *= al1;
         }
       }
-      // ---- O^T += V^T P^T over my tokens (P^T comes straight from S) ----
+      // ---- O^T += V^T P^T over my tokens (P^T: a transpose of P packed) ----
       // V rows past the length may hold anything (NaN): on a partial tile
       // they are zeroed in the fragments, so that 0 * NaN never reaches the
       // accumulator.  Full shares, nearly all, take the product without masks.
       {
-        // products over 16-token groups: P^T of group hv is n-tiles 2hv
-        // (tokens 2*tid4, +1) and 2hv+1 (tokens 8 + 2*tid4, +1)
+        // products over 16-token groups: the packed pairs (token gid, heads
+        // 2*tid4, +1) and (token gid + 8, ...) transposed are P^T's B
+        // fragments (head gid; tokens 2*tid4, +1 and 8 + 2*tid4, +1)
 #pragma unroll
-        for (int hv = 0; hv < NT / 2; ++hv) {
+        for (int hv = 0; hv < NG; ++hv) {
           const int vh = valid - 16 * hv;  // tokens of this group below the length
           if (hv > 0 && vh <= 0) break;
-          uint32_t pa0, pa2;
+          uint32_t q0, q1;
           if constexpr (!quant(kFmt)) {
-            pa0 = pack_bf16(pr[4 * hv], pr[4 * hv + 1]);
-            pa2 = pack_bf16(pr[4 * hv + 2], pr[4 * hv + 3]);
+            q0 = pack_bf16(pr[hv][0], pr[hv][1]);
+            q1 = pack_bf16(pr[hv][2], pr[hv][3]);
           } else {
-            pa0 = pack_f16(pr[4 * hv] * t_vs, pr[4 * hv + 1] * t_vs);
-            pa2 = pack_f16(pr[4 * hv + 2] * t_vs, pr[4 * hv + 3] * t_vs);
+            q0 = pack_f16(pr[hv][0] * t_vs, pr[hv][1] * t_vs);
+            q1 = pack_f16(pr[hv][2] * t_vs, pr[hv][3] * t_vs);
           }
+          const uint32_t pa0 = movmatrix_t(q0);
+          const uint32_t pa2 = movmatrix_t(q1);
           const uint32_t gbase = vbase + hv * 16 * Ly::kBoxRowB;
           auto pv_product = [&](auto masked) {
             constexpr bool kMasked = decltype(masked)::value;
@@ -985,9 +991,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       // once the flush warp has read the previous segment's slots.  With two
       // slots, warps 2 and 3 do so, and warps 0 and 1 fold their partner's
       // snapshot (warp + 2) into their own state and write the result back.
-      float l_row = l_part;
-      l_row += __shfl_xor_sync(0xffffffffu, l_row, 1);
-      l_row += __shfl_xor_sync(0xffffffffu, l_row, 2);
+      // heads h0, h1 of this thread: totals over the eight lanes of a column
+      float l_h[2] = {l_part[0], l_part[1]};
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        l_h[0] += __shfl_xor_sync(0xffffffffu, l_h[0], o);
+        l_h[1] += __shfl_xor_sync(0xffffffffu, l_h[1], o);
+      }
       const int slot = warp % kSnap;
       float* so = red_o + slot * G * kRedRow;
       const int h0 = 2 * tid4, h1 = 2 * tid4 + 1;
@@ -1010,9 +1020,15 @@ __global__ void __launch_bounds__(kThreads, 2)
       };
       if (kSnap == kConsumerWarps || warp >= kSnap) {
         if (nflush > 0 && !mbar_wait(red_empty, (uint32_t)((nflush - 1) & 1), p.flags)) return;
-        if (row_ok && tid4 == 0) {
-          red_m[slot * G + gid] = m_run;
-          red_l[slot * G + gid] = l_row;
+        if (gid == 0) {
+          if (h0 < G) {
+            red_m[slot * G + h0] = m_run[0];
+            red_l[slot * G + h0] = l_h[0];
+          }
+          if (h1 < G) {
+            red_m[slot * G + h1] = m_run[1];
+            red_l[slot * G + h1] = l_h[1];
+          }
         }
         float* r0 = so + h0 * kRedRow;
         float* r1 = so + h1 * kRedRow;
@@ -1038,16 +1054,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       } else {
         if (!mbar_wait(pair_full, (uint32_t)(nflush & 1), p.flags)) return;
-        const float mp = row_ok ? red_m[slot * G + gid] : -INFINITY;
-        const float lp = row_ok ? red_l[slot * G + gid] : 0.f;
-        const float M = fmaxf(m_run, mp);
-        const float sa = m_run == -INFINITY ? 0.f : fast_exp2(m_run - M);
-        const float sb = mp == -INFINITY ? 0.f : fast_exp2(mp - M);
-        const float l_new = sa * l_row + sb * lp;
-        const float a_lo = __shfl_sync(0xffffffffu, sa, 8 * tid4);
-        const float a_hi = __shfl_sync(0xffffffffu, sa, 8 * tid4 + 4);
-        const float b_lo = __shfl_sync(0xffffffffu, sb, 8 * tid4);
-        const float b_hi = __shfl_sync(0xffffffffu, sb, 8 * tid4 + 4);
+        // the partner's (m, l) of heads h0, h1 and the factors of both sides
+        float M[2], sa[2], sb[2], l_new[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int h = 2 * tid4 + k;
+          const float mp = h < G ? red_m[slot * G + h] : -INFINITY;
+          const float lp = h < G ? red_l[slot * G + h] : 0.f;
+          M[k] = fmaxf(m_run[k], mp);
+          sa[k] = m_run[k] == -INFINITY ? 0.f : fast_exp2(m_run[k] - M[k]);
+          sb[k] = mp == -INFINITY ? 0.f : fast_exp2(mp - M[k]);
+          l_new[k] = sa[k] * l_h[k] + sb[k] * lp;
+        }
+        const float a_lo = sa[0], a_hi = sa[1], b_lo = sb[0], b_hi = sb[1];
         float* r0 = so + h0 * kRedRow;
         float* r1 = so + h1 * kRedRow;
 #pragma unroll
@@ -1062,10 +1081,16 @@ __global__ void __launch_bounds__(kThreads, 2)
             r1[d + d_step] = ot[m][3] * a_hi + r1[d + d_step] * b_hi;
           }
         }
-        __syncwarp();  // every lane has read the partner's (m, l) row
-        if (row_ok && tid4 == 0) {
-          red_m[slot * G + gid] = M;
-          red_l[slot * G + gid] = l_new;
+        __syncwarp();  // every lane has read the partner's (m, l)
+        if (gid == 0) {
+          if (h0 < G) {
+            red_m[slot * G + h0] = M[0];
+            red_l[slot * G + h0] = l_new[0];
+          }
+          if (h1 < G) {
+            red_m[slot * G + h1] = M[1];
+            red_l[slot * G + h1] = l_new[1];
+          }
         }
         if (warp == 0 && lane == 0) write_desc();
         __syncwarp();
