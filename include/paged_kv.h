@@ -141,12 +141,15 @@ int paged_kv_append(const pkv_cache* cache, const int32_t* page_table, int32_t m
 /*
  * Split planning for decode (host only, no CUDA calls).  Decode runs as one
  * persistent wave of C CTAs.  The work list is every (sequence, kv head) unit
- * cut into 64-token tiles, concatenated in (sequence, kv head) order; CTA c
- * takes the contiguous range [c*T/C, (c+1)*T/C) of the T tiles, so every CTA
- * streams the same number of KV bytes whatever the length mix.  A unit that a
- * range boundary cuts becomes several split-KV partials merged in the same
- * launch.  C = num_ctas if num_ctas > 0, else num_sms * ctas_per_sm; C never
- * exceeds the tiles of the largest batch the arguments allow.
+ * cut into tiles (64 tokens for bf16 and FP4 pools, 128 for E4M3 and INT8, so
+ * that a tile is 32 KB of K and V at head_dim 128), concatenated in
+ * (sequence, kv head) order; CTA c takes the contiguous range
+ * [c*T/C, (c+1)*T/C) of the T tiles, so every CTA streams the same number of
+ * KV bytes whatever the length mix (when C > T only T CTAs take work).  A
+ * unit that a range boundary cuts becomes several split-KV partials merged
+ * in the same launch.  C = num_ctas if num_ctas > 0, else
+ * num_sms * ctas_per_sm; C never exceeds the 64-token tiles of the largest
+ * batch the arguments allow.
  * Output: *out_ctas = C >= 1.
  */
 int paged_decode_plan(int32_t batch, int32_t num_kv_heads, int32_t max_seq_len,

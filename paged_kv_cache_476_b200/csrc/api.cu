@@ -202,7 +202,8 @@ int paged_decode_plan(int32_t batch, int32_t num_kv_heads, int32_t max_seq_len,
   if (batch < 0 || num_kv_heads < 1 || max_seq_len < 0 || num_sms < 1 || num_ctas < 0 ||
       ctas_per_sm < 1)
     return PKV_ERR_SHAPE;
-  // Work-list tiles (64 tokens) of the largest possible batch.
+  // 64-token work-list tiles of the largest possible batch (an upper bound on
+  // the tiles of every format; the kernel lets only min(C, T) CTAs work).
   const long long max_tiles = (long long)batch * num_kv_heads * ((max_seq_len + 63) / 64);
   long long c = num_ctas > 0 ? num_ctas : (long long)num_sms * ctas_per_sm;
   if (c > max_tiles) c = max_tiles;
