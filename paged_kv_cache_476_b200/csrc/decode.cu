@@ -162,8 +162,8 @@ __device__ __forceinline__ uint32_t tile_at(uint32_t base, LaneTile lt, int ce) 
          (((uint32_t)(ce % kChunksPerBox) << 4) ^ lt.x);
 }
 
-// CTA (of C <= T over T tiles) whose range [c*T/C, (c+1)*T/C) holds global
-// tile x.  With C <= T every range holds at least one tile.
+// CTA (of C <= T over T virtual tiles) whose range [c*T/C, (c+1)*T/C) holds
+// virtual tile x.  With C <= T every range is non-empty.
 __device__ __forceinline__ int64_t cta_of(int64_t x, int64_t C, int64_t T) {
   return ((x + 1) * C - 1) / T;
 }
@@ -178,6 +178,74 @@ __device__ __forceinline__ int32_t clamp_len(const DecodeParams& p, int32_t len,
     return len < 0 ? 0 : cap;
   }
   return len;
+}
+
+// The work list counts each unit as its tiles plus kCost virtual tiles after
+// them, which load nothing: they stand for what a unit end costs the
+// consumers (a segment hand-off, and on average half a tile of idle lanes),
+// so that the equal split hands fewer real tiles to ranges in which many
+// short units end.  Quantised pools, whose consumers bound the call, count
+// one; bf16 pools, bound by HBM (a unit end hides under the tile waits),
+// count none.
+template <int kFmt>
+__host__ __device__ constexpr int unit_end_cost() { return quant(kFmt) ? 1 : 0; }
+
+// The first real tile at or after virtual index v: sequence b, kv head g,
+// tile t, its virtual index xv and its real index (real tiles before it).
+// Past the last tile, b = batch and (xv, real) are the totals.  Warp-wide.
+struct TilePos {
+  int b, g, t;
+  int64_t xv, real;
+};
+
+template <int kTile, int kCost>
+__device__ TilePos locate_tile(const DecodeParams& p, int64_t v, int lane) {
+  const int Hkv = p.num_kv_heads;
+  int64_t run_v = 0, run_r = 0;
+  for (int base = 0; base < p.batch; base += 32) {
+    const int b = base + lane;
+    const int t = b < p.batch ? tiles_of<kTile>(clamp_len(p, __ldg(p.seq_lens + b), false)) : 0;
+    const int vt = t > 0 ? t + kCost : 0;  // virtual tiles of one unit of b
+    int incl_v = vt, incl_r = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int yv = __shfl_up_sync(0xffffffffu, incl_v, o);
+      const int yr = __shfl_up_sync(0xffffffffu, incl_r, o);
+      if (lane >= o) {
+        incl_v += yv;
+        incl_r += yr;
+      }
+    }
+    const int chunk_v = __shfl_sync(0xffffffffu, incl_v, 31);
+    const int chunk_r = __shfl_sync(0xffffffffu, incl_r, 31);
+    if (run_v + (int64_t)chunk_v * Hkv > v) {
+      const bool hit = run_v + (int64_t)incl_v * Hkv > v;
+      const int l0 = __ffs(__ballot_sync(0xffffffffu, hit)) - 1;
+      const int t0 = __shfl_sync(0xffffffffu, t, l0);
+      const int vt0 = __shfl_sync(0xffffffffu, vt, l0);
+      const int ev0 = __shfl_sync(0xffffffffu, incl_v - vt, l0);
+      const int er0 = __shfl_sync(0xffffffffu, incl_r - t, l0);
+      const int64_t off = v - (run_v + (int64_t)ev0 * Hkv);  // in [0, vt0 * Hkv)
+      const int g = (int)(off / vt0);
+      const int po = (int)(off - (int64_t)g * vt0);
+      const int64_t unit_v = run_v + (int64_t)ev0 * Hkv + (int64_t)g * vt0;
+      const int64_t unit_r = run_r + (int64_t)er0 * Hkv + (int64_t)g * t0;
+      if (po < t0) return {base + l0, g, po, unit_v + po, unit_r + po};
+      // v lies on the unit's end cost: the next unit's first tile (of the
+      // next sequence with tiles, past the last kv head)
+      TilePos r = {base + l0, g + 1, 0, unit_v + vt0, unit_r + t0};
+      if (r.g == Hkv) {
+        r.g = 0;
+        do {
+          ++r.b;
+        } while (r.b < p.batch && tiles_of<kTile>(clamp_len(p, __ldg(p.seq_lens + r.b), false)) == 0);
+      }
+      return r;
+    }
+    run_v += (int64_t)chunk_v * Hkv;
+    run_r += (int64_t)chunk_r * Hkv;
+  }
+  return {p.batch, 0, 0, run_v, run_r};
 }
 
 // Fused append: the producer warp writes sequence b's newest token (K and V
@@ -274,22 +342,29 @@ __global__ void __launch_bounds__(kThreads, 2)
   int pb = 0, pg = 0, pt = 0;  // producer's position (b, g, tile) at the range start
   int64_t range_start = 0, T = 0, Ce = 1;
   if (warp == kProducerWarp) {
-    // Total tiles over all units.
+    // Total virtual tiles over all units (real tiles plus the end costs).
     int64_t tot = 0;
     for (int base = 0; base < p.batch; base += 32) {
       const int b = base + lane;
       const int t = b < p.batch ? tiles_of<kTile>(clamp_len(p, __ldg(p.seq_lens + b), c == 0)) : 0;
-      tot += t;
+      tot += t > 0 ? t + unit_end_cost<kFmt>() : 0;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
     T = tot * Hkv;
-    // Only min(C, T) CTAs take work, so that every working range is
-    // non-empty and a unit's segment count equals the CTAs that touch it.
+    // Only min(C, T) CTAs take work.  A range may hold only end costs (no
+    // real tile); a unit's segment count is the number of ranges that hold
+    // its real tiles, and every range between its first and last holds some.
     Ce = C < T ? C : T;
     if (c < Ce) {
-      range_start = (c * T) / Ce;
-      n_tiles = ((c + 1) * T) / Ce - range_start;
+      constexpr int kCost = unit_end_cost<kFmt>();
+      const TilePos s0 = locate_tile<kTile, kCost>(p, (c * T) / Ce, lane);
+      const TilePos s1 = locate_tile<kTile, kCost>(p, ((c + 1) * T) / Ce, lane);
+      n_tiles = s1.real - s0.real;
+      pb = s0.b;
+      pg = s0.g;
+      pt = s0.t;
+      range_start = s0.xv;  // virtual index of the range's first real tile
     }
     // Empty sequences (length 0): out = 0, lse = -inf, written by one CTA each.
     for (int b = (int)((c * p.batch) / C); b < (int)(((c + 1) * p.batch) / C); ++b) {
@@ -299,34 +374,6 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (p.lse)
           for (int h = lane; h < p.num_q_heads; h += 32)
             p.lse[(int64_t)b * p.num_q_heads + h] = -INFINITY;
-      }
-    }
-    if (n_tiles > 0) {
-      // Locate (b, g, tile) of global tile range_start.
-      int64_t run = 0;
-      for (int base = 0; base < p.batch; base += 32) {
-        const int b = base + lane;
-        const int t = b < p.batch ? tiles_of<kTile>(clamp_len(p, __ldg(p.seq_lens + b), false)) : 0;
-        int incl = t;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        const int chunk = __shfl_sync(0xffffffffu, incl, 31);
-        if (run + (int64_t)chunk * Hkv > range_start) {
-          const bool hit = run + (int64_t)incl * Hkv > range_start;
-          const unsigned m = __ballot_sync(0xffffffffu, hit);
-          const int l0 = __ffs(m) - 1;
-          const int t0 = __shfl_sync(0xffffffffu, t, l0);
-          const int e0 = __shfl_sync(0xffffffffu, incl - t, l0);
-          pb = base + l0;
-          const int64_t off = range_start - (run + (int64_t)e0 * Hkv);
-          pg = (int)(off / t0);
-          pt = (int)(off - (int64_t)pg * t0);
-          break;
-        }
-        run += (int64_t)chunk * Hkv;
       }
     }
     if (lane == 0) s_misc[0] = (int)n_tiles;
@@ -408,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     int cache_key = -1, cache_j0 = 0;
     int my_pid = 0;
     float my_ks = 1.f, my_vs = 1.f;
-    int64_t x = range_start;  // global tile index
+    int64_t x = range_start;  // virtual index of the tile at hand
     int u_seg_base = 0, u_nseg = 1, u_slot = 0;
     int issued = 0;
     for (int64_t i = 0; i < n_tiles; ++i, ++x) {
@@ -494,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (first) {
           // once per unit: which CTAs share it, hence its partial slots
           const int64_t u = (int64_t)b * Hkv + g;
-          const int64_t x_unit = x - t;  // global index of the unit's first tile
+          const int64_t x_unit = x - t;  // virtual index of the unit's first tile
           const int64_t c_first = cta_of(x_unit, Ce, T);
           const int64_t c_last = cta_of(x_unit + ntile - 1, Ce, T);
           u_seg_base = (int)(u + c_first);
@@ -553,9 +600,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       __syncwarp();
       ++issued;
-      // advance to the next tile of the work list
+      // advance to the next tile of the work list (past the unit's end cost)
       if (++t == ntile) {
         t = 0;
+        x += unit_end_cost<kFmt>();
         if (++g == Hkv) {
           g = 0;
           do {
